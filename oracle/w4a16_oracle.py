@@ -1,0 +1,213 @@
+"""CPU oracle for group-wise low-bit weight quantization and the W4A16 GEMV.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code,
+constant table or helper with the CUDA library, and never calls it.
+
+It is the plain, slow, obviously correct statement of what the hot path
+computes: numpy in float64, following the pages step by step.
+
+Pages cited (by title and section):
+
+* [L13] "MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading guide
+  (quidproquo.cc).  §AWQ "why scaling lowers the error" (slides 26, 28):
+  Q(w) = Delta * Round(w / Delta), Delta = max|w| / 2^(N-1), expected Round
+  error about 0.25; the search objective with s = s_X^alpha, s_X the mean
+  activation magnitude; scaling salient channels by s and folding 1/s into the
+  previous op (slides 25-27).  §TinyChat: offline packing so that one AND and
+  one shift unpack the codes (slide 36); dequantization fused into the matmul
+  (slide 37).  §"why W8A8 is not enough": decode is memory-bound (slides 19-20).
+* [CMU] "CMU 11-868 LLM Systems: Model Quantization (L19/L20)" reading guide
+  (quidproquo.cc).  §"absmax and zero-point" and the two PyTorch functions of
+  lecture slide 10: zero-point scale from (max - min) / (2^8 - 1), a rounded
+  zero point, clipping to the code range, dequant = (q - zp) * step, and a
+  zero range replaced by 1.  §"back to the question": batch-1 decode is a GEMV
+  and memory-bound.
+* [Lab4] "MIT 6.5940 Lab 4 + Lab 5" reading guide (quidproquo.cc).  §Lab 4
+  setup: calibration statistic = mean |X| per input channel over 512-token
+  blocks; pseudo quantization (quantize, then dequantize at once); 3-bit,
+  group 128.
+* [ML11] "Learning-ML-DL ch. 11: Quantization for LLMs"
+  (hoangvt2501.github.io).  §11.3: Y = (X diag(s)^-1)(W diag(s))^T;
+  §11.4: AWQ's s = s_X^alpha with s_X the mean channel magnitude.
+
+Readings of points the pages leave open:
+
+1. Symmetric step Delta = max|w| / 2^(N-1) as in [L13]; the signed code is
+   clamped to [-2^(N-1), 2^(N-1)-1] and stored as u = q + 2^(N-1), z = 2^(N-1).
+2. Round = round half to even (numpy ``rint``), matching the pages' ``round``.
+3. Asymmetric codes are u = clamp(Round(w / Delta) + z, 0, 2^N - 1), so that an
+   unclamped element dequantizes to exactly Delta * Round(w / Delta).
+4. Asymmetric step Delta = fp16(fp64((max - min) / (2^N - 1))); zero point
+   z = clamp(Round(-min / Delta), 0, 2^N - 1), stored as an fp16 integer.
+5. A step that would be zero in fp16 (zero range included) is computed as if
+   the range were 1, extending [CMU]'s "range 0 -> 1" rule.
+6. The AWQ-scaled weight is rounded to fp16 once, w' = fp16(W * s), before
+   the group statistics are taken.
+7. s = fp16(s_X ** alpha) with s_X the fp64 mean of |X| over tokens; no other
+   normalisation.
+8. Packed layout v1 (our own design, stated in include/w4a16.h): qweight is
+   u32[N, K/8]; word (n, j) holds k = 8j + i, i = 0..7; nibble slot p (bits
+   4p..4p+3) holds i = [0, 2, 4, 6, 1, 3, 5, 7][p].
+
+Every function here is pinned by tests marked ``not gpu`` against closed
+forms, brute force, invariants the pages state, or special cases.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+F16 = np.float16
+F64 = np.float64
+
+ASYM = 0
+SYM = 1
+
+# layout v1: which element i of an 8-element k-block sits in nibble slot p
+SLOT_TO_ELEM = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
+# ---------------------------------------------------------------------------
+# a0: AWQ activation-aware scale  ([L13] slide 28, [Lab4] setup, [ML11] §11.4)
+# ---------------------------------------------------------------------------
+def act_scale(X: np.ndarray, alpha: float) -> np.ndarray:
+    """s_k = fp16( (mean_t |X[t, k]|) ** alpha ) for calibration tokens X[T, K].
+
+    s_X is the per-input-channel mean activation magnitude ([L13] slide 28,
+    [ML11] §11.4) averaged over the calibration tokens ([Lab4] setup).
+    """
+    X = np.asarray(X)
+    sx = np.abs(X.astype(F64)).mean(axis=0)
+    return (sx ** F64(alpha)).astype(F16)
+
+
+# ---------------------------------------------------------------------------
+# a1: scaled weight  ([L13] slides 25-27, [ML11] §11.3)
+# ---------------------------------------------------------------------------
+def scale_weight(W: np.ndarray, s: np.ndarray | None) -> np.ndarray:
+    """w'[n, k] = fp16(W[n, k] * s[k]): input channel k of the weight times s_k.
+
+    The matching activation is divided by s_k in the previous op, so that
+    (X diag(s)^-1)(W diag(s))^T = X W^T ([ML11] §11.3).
+    """
+    W = np.asarray(W, dtype=F16)
+    if s is None:
+        return W.copy()
+    s = np.asarray(s, dtype=F16)
+    return (W.astype(F64) * s.astype(F64)[None, :]).astype(F16)
+
+
+# ---------------------------------------------------------------------------
+# a2 + a3: group statistics, step Delta and zero point z
+# ---------------------------------------------------------------------------
+def group_params(wp: np.ndarray, bits: int, mode: int, group: int = 128):
+    """Per (row, group) step Delta and zero point z, both returned as fp16.
+
+    Asymmetric ([CMU] zero-point function): Delta = fp16((max - min) / (2^N-1)),
+    z = clamp(Round(-min / Delta), 0, 2^N - 1).
+    Symmetric ([L13] slide 26): Delta = fp16(max|w| / 2^(N-1)), z = 2^(N-1).
+    A zero step is replaced by the step of a unit range (reading 5).
+    """
+    N, K = wp.shape
+    g = wp.astype(F64).reshape(N, K // group, group)
+    qmax = 2 ** bits - 1
+    if mode == ASYM:
+        mx = g.max(axis=-1)
+        mn = g.min(axis=-1)
+        delta = ((mx - mn) / F64(qmax)).astype(F16)
+        delta[delta == 0] = F16(1.0 / qmax)
+        z = np.clip(np.rint(-mn / delta.astype(F64)), 0, qmax)
+    elif mode == SYM:
+        amax = np.abs(g).max(axis=-1)
+        half = 2 ** (bits - 1)
+        delta = (amax / F64(half)).astype(F16)
+        delta[delta == 0] = F16(1.0 / half)
+        z = np.full(delta.shape, F64(half))
+    else:
+        raise ValueError("mode must be ASYM or SYM")
+    return delta, z.astype(F16)
+
+
+# ---------------------------------------------------------------------------
+# a4: round-to-nearest codes  ([L13] slide 26, [CMU] zero-point function)
+# ---------------------------------------------------------------------------
+def quantize_codes(wp: np.ndarray, delta: np.ndarray, z: np.ndarray, bits: int, group: int = 128) -> np.ndarray:
+    """u = clamp(Round(w' / Delta) + z, 0, 2^N - 1) as uint8 [N, K]."""
+    N, K = wp.shape
+    g = wp.astype(F64).reshape(N, K // group, group)
+    d = delta.astype(F64)[..., None]
+    zz = z.astype(F64)[..., None]
+    u = np.clip(np.rint(g / d) + zz, 0, 2 ** bits - 1)
+    return u.reshape(N, K).astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# a5: pack / unpack, layout v1  ([L13] slide 36: offline reordering)
+# ---------------------------------------------------------------------------
+def pack_v1(u: np.ndarray) -> np.ndarray:
+    """Pack codes u[N, K] (values < 16) into qweight u32[N, K/8] (layout v1)."""
+    N, K = u.shape
+    blocks = u.astype(np.uint32).reshape(N, K // 8, 8)
+    words = np.zeros((N, K // 8), dtype=np.uint32)
+    for p, i in enumerate(SLOT_TO_ELEM):
+        words |= blocks[:, :, i] << np.uint32(4 * p)
+    return words
+
+
+def unpack_v1(qweight: np.ndarray) -> np.ndarray:
+    """Inverse of pack_v1: qweight u32[N, K/8] -> codes uint8[N, K]."""
+    qweight = np.asarray(qweight, dtype=np.uint32)
+    N, KW = qweight.shape
+    u = np.zeros((N, KW, 8), dtype=np.uint8)
+    for p, i in enumerate(SLOT_TO_ELEM):
+        u[:, :, i] = (qweight >> np.uint32(4 * p)) & np.uint32(0xF)
+    return u.reshape(N, KW * 8)
+
+
+# ---------------------------------------------------------------------------
+# The quantizer end to end: awq_quantize_pack
+# ---------------------------------------------------------------------------
+def quantize_pack(W: np.ndarray, s: np.ndarray | None, group: int = 128, bits: int = 4, mode: int = ASYM):
+    """(qweight u32[N,K/8], scales fp16[N,K/group], zeros fp16[N,K/group])."""
+    wp = scale_weight(W, s)
+    delta, z = group_params(wp, bits, mode, group)
+    u = quantize_codes(wp, delta, z, bits, group)
+    return pack_v1(u), delta, z
+
+
+# ---------------------------------------------------------------------------
+# a6: dequantization  ([CMU] dequant = (q - zp) * step; [Lab4] pseudo quant)
+# ---------------------------------------------------------------------------
+def dequant(qweight: np.ndarray, scales: np.ndarray, zeros: np.ndarray, group: int = 128) -> np.ndarray:
+    """w_hat[n, k] = (u[n, k] - z[n, g]) * Delta[n, g] in float64 (exact)."""
+    u = unpack_v1(qweight).astype(F64)
+    N, K = u.shape
+    d = np.repeat(scales.astype(F64), group, axis=1)
+    z = np.repeat(zeros.astype(F64), group, axis=1)
+    return (u - z) * d
+
+
+# ---------------------------------------------------------------------------
+# a7 / a8: the GEMV / skinny GEMM  ([L13] slides 19-20, 37; [CMU] slide 23)
+# ---------------------------------------------------------------------------
+def gemm_ref(x: np.ndarray, w_hat: np.ndarray):
+    """y = x @ w_hat^T in float64 and the per-element bound B = |x| @ |w_hat|^T.
+
+    The tolerance the CUDA result must meet is |y - y_ref| <= 2e-3 * B + 1e-3.
+    """
+    x64 = np.asarray(x).astype(F64)
+    y = x64 @ w_hat.T
+    bound = np.abs(x64) @ np.abs(w_hat).T
+    return y, bound
+
+
+def gemm(x, qweight, scales, zeros, group: int = 128):
+    """Pseudo-quantized reference of w4a16_gemm: dequantize, then fp64 matmul."""
+    return gemm_ref(x, dequant(qweight, scales, zeros, group))
+
+
+def gemm_rows(x, qweight, scales, zeros, rows, group: int = 128):
+    """The reference restricted to output channels ``rows`` (for sampled checks)."""
+    rows = np.asarray(rows)
+    w_hat = dequant(qweight[rows], scales[rows], zeros[rows], group)
+    return gemm_ref(x, w_hat)
