@@ -1,0 +1,170 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) group-wise 4-bit weight-only
+ * quantization library and its W4A16 decode GEMV / skinny GEMM.
+ *
+ * What is computed (pages cited by title and section):
+ *
+ *  - AWQ activation-aware scaling: salient input channels of the weight are
+ *    multiplied by s > 1 and the activations divided by s, with s = s_X^alpha
+ *    and s_X the mean activation magnitude per input channel ("MIT 6.5940
+ *    Fall 2024 Lecture 13: LLM Deployment" reading guide, §AWQ, slides 25-28;
+ *    "Learning-ML-DL ch. 11", §11.4).  The 1/s on the activation is folded
+ *    into the previous op, so w4a16_gemm receives x already divided by s.
+ *  - Round-to-nearest group quantization Q(w) = Delta * Round(w / Delta) per
+ *    group of 128 input channels (Lecture 13 guide, §AWQ, slide 26), with the
+ *    zero-point (asymmetric) form of the "CMU 11-868 Model Quantization"
+ *    reading guide (§absmax and zero-point, lecture slide 10).
+ *  - Packing the codes offline into 32-bit words so that one AND (and one
+ *    shift) unpacks them (Lecture 13 guide, §TinyChat, slide 36), and a GEMV
+ *    that dequantizes in registers, fused with the product (slide 37), for
+ *    memory-bound batch-1 decode (§"why W8A8 is not enough", slides 19-20).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensors are dense, row-major, on the current CUDA device, owned by
+ *    the caller.  The library never allocates device or host memory.
+ *  - "fp16" is IEEE binary16 (__half).  Every pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).  A
+ *    return of W4A16_OK means the arguments were valid and the work was
+ *    enqueued; nothing is launched when a negative status is returned.
+ *  - Errors: a negative w4a16_status; w4a16_last_error() gives a message
+ *    (thread-local, valid until the next call on the same thread).
+ *
+ * Packed layout v1 (our own design for sm_100a; w4a16_layout_version() == 1):
+ *    qweight is uint32[N][K/8].  Word (n, j) holds the codes of
+ *    k = 8j + i, i = 0..7.  Nibble slot p (bits 4p..4p+3) holds
+ *    i = {0, 2, 4, 6, 1, 3, 5, 7}[p].  Hence (word >> 4t) & 0x000F000F has the
+ *    codes of k = 8j+2t and 8j+2t+1 in its low and high 16-bit halves, which
+ *    OR 0x64006400 turns into the fp16 pair (1024 + q0, 1024 + q1).
+ *    3-bit codes use the same nibble containers.
+ *    scales[n][g] = Delta and zeros[n][g] = z (an integer held in fp16) for
+ *    the group g = k / group; the dequantized weight is (u - z) * Delta.
+ */
+#ifndef W4A16_H_
+#define W4A16_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A16_API __attribute__((visibility("default")))
+#else
+#define W4A16_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; spelled out so this header needs no CUDA headers. */
+typedef struct CUstream_st* w4a16_stream_t;
+
+typedef enum {
+  W4A16_OK = 0,
+  W4A16_ERR_ARG = -1,          /* null pointer, non-positive size, bad enum, non-finite alpha */
+  W4A16_ERR_ALIGN = -2,        /* a pointer is not 16-byte aligned */
+  W4A16_ERR_SHAPE = -3,        /* K not a multiple of the group, sizes too large */
+  W4A16_ERR_UNSUPPORTED = -4,  /* valid but unsupported: group != 128, bits not in {3,4} */
+  W4A16_ERR_WORKSPACE = -5,    /* workspace missing or smaller than w4a16_gemm_workspace_size */
+  W4A16_ERR_CUDA = -6,         /* a CUDA runtime call or a kernel launch failed */
+  W4A16_ERR_DEVICE = -7        /* a kernel gave up waiting (see w4a16_gemm_check) */
+} w4a16_status;
+
+typedef enum {
+  W4A16_ASYM = 0,  /* Delta = fp16((max-min)/(2^bits-1)), z = clamp(Round(-min/Delta), 0, 2^bits-1) */
+  W4A16_SYM = 1    /* Delta = fp16(max|w|/2^(bits-1)),    z = 2^(bits-1) */
+} w4a16_mode;
+
+/*
+ * awq_act_scale -- per-input-channel AWQ scale from calibration activations.
+ *
+ *   s[k] = fp16( (mean_t |X[t][k]|) ^ alpha ),  t = 0..T-1
+ *
+ * s_X = mean |X| per input channel is the calibration statistic ("MIT 6.5940
+ * Lab 4 + Lab 5" reading guide, §Lab 4 setup: mean |X| over 512-token blocks)
+ * and s = s_X^alpha the scale (Lecture 13 guide, §AWQ, slide 28).  The mean
+ * is formed in fp64 (exact, hence independent of summation order, for T <= 8192)
+ * and the power in fp64; s may differ from a correctly rounded result by one fp16 ulp
+ * only when s_X^alpha lies within a few fp64 ulps of an fp16 rounding boundary.
+ *
+ *   X     fp16 [T][K], device.      s  fp16 [K], device (output).
+ *   T, K  >= 1.   alpha  finite; the pages search it in [0, 1] (any finite value accepted).
+ */
+W4A16_API w4a16_status awq_act_scale(const void* X, int T, int K, double alpha, void* s,
+                           w4a16_stream_t stream);
+
+/*
+ * awq_quantize_pack -- AWQ scaling + group RTN + layout-v1 packing.
+ *
+ *   w'[n][k] = fp16(W[n][k] * s[k])               (one rounding; s == NULL means s = 1)
+ *   per group (n, g) of `group` consecutive k:
+ *     ASYM: Delta = fp16(fp64(max w' - min w') / (2^bits - 1)),
+ *           z = clamp(Round(-min w' / Delta), 0, 2^bits - 1)
+ *     SYM:  Delta = fp16(max |w'| / 2^(bits-1)),   z = 2^(bits-1)
+ *     a Delta that rounds to zero is replaced by the Delta of a unit range
+ *   u[n][k] = clamp(Round(w'[n][k] / Delta) + z, 0, 2^bits - 1)
+ *   Round = round half to even, on the exact quotients.
+ *
+ *   W        fp16 [N][K], device.         s  fp16 [K] or NULL, device.
+ *   qweight  uint32 [N][K/8] (output).    scales, zeros  fp16 [N][K/group] (outputs).
+ *   N >= 1;  K a multiple of group;  group == 128;  bits in {3, 4}.
+ *   W * s must be finite in fp16 (|W*s| <= 65504); other inputs give
+ *   unspecified codes but never fault.
+ * The results are bit-exact: identical on every call and to the reference
+ * definition above.
+ */
+W4A16_API w4a16_status awq_quantize_pack(const void* W, const void* s, int N, int K, int group, int bits,
+                               w4a16_mode mode, uint32_t* qweight, void* scales, void* zeros,
+                               w4a16_stream_t stream);
+
+/*
+ * w4a16_gemm_workspace_size -- bytes of workspace that w4a16_gemm needs.
+ * Returns 0 for invalid sizes.  The workspace holds fp32 split-K partial sums,
+ * per-row-block arrival counters and a device status word.
+ */
+W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
+
+/*
+ * w4a16_gemm -- y = x * dequant(qweight, scales, zeros)^T.
+ *
+ *   y[m][n] = fp16( sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k] )
+ *
+ * with fp32 accumulation.  M < 16 runs the split-K CUDA-core GEMV; M >= 16 the
+ * tensor-core kernel.  x is the activation already divided by the AWQ scale s.
+ * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
+ * y_ref the exact product with the dequantized weight.  The order of the
+ * split-K additions may vary between calls, so y may differ in the last bit.
+ *
+ *   x        fp16 [M][K], device.     y  fp16 [M][N], device (output).
+ *   qweight, scales, zeros as produced by awq_quantize_pack (layout v1).
+ *   1 <= M <= 64;  N >= 1;  K a multiple of group;  group == 128.
+ *   workspace  device memory of at least w4a16_gemm_workspace_size(M, N, K, group)
+ *              bytes, 16-byte aligned, ZERO-FILLED before its first use.  Every
+ *              call that completes leaves it zero-filled again, so it can be reused
+ *              by later calls on the same stream.  Calls that may run concurrently
+ *              need distinct workspaces.  After W4A16_ERR_DEVICE it must be zero-filled
+ *              again by the caller.
+ */
+W4A16_API w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scales,
+                        const void* zeros, int M, int N, int K, int group, void* y,
+                        void* workspace, size_t workspace_bytes, w4a16_stream_t stream);
+
+/*
+ * w4a16_gemm_check -- synchronizes `stream` and reads the workspace's device
+ * status word.  Returns W4A16_ERR_DEVICE if any earlier w4a16_gemm with this
+ * workspace gave up waiting for its weight tiles (bounded waits, about 2 s),
+ * W4A16_ERR_CUDA if the stream reports an error, else W4A16_OK.  The status word is
+ * cleared by this call.
+ */
+W4A16_API w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream);
+
+/* Message for the last error on this thread ("" if none). */
+W4A16_API const char* w4a16_last_error(void);
+
+/* Packed layout version: 1 (see above). */
+W4A16_API int w4a16_layout_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H_ */

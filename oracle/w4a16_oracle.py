@@ -116,7 +116,8 @@ def group_params(wp: np.ndarray, bits: int, mode: int, group: int = 128):
         mn = g.min(axis=-1)
         delta = ((mx - mn) / F64(qmax)).astype(F16)
         delta[delta == 0] = F16(1.0 / qmax)
-        z = np.clip(np.rint(-mn / delta.astype(F64)), 0, qmax)
+        # an integer zero point has no sign of zero: -0.0 (from min = 0) becomes +0.0
+        z = np.clip(np.rint(-mn / delta.astype(F64)), 0, qmax) + 0.0
     elif mode == SYM:
         amax = np.abs(g).max(axis=-1)
         half = 2 ** (bits - 1)

@@ -1,0 +1,116 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/w4a16.h declares, and rejects bad arguments before launching anything.
+
+No test here reaches a kernel launch: every call fails validation first, so
+the fake device addresses below are never dereferenced."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a16_decode_gemv_b200 as w4
+from w4a16_decode_gemv_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+OK, ERR_ARG, ERR_ALIGN, ERR_SHAPE, ERR_UNSUPPORTED, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+A = 0x10000          # a 16-byte aligned fake address (never dereferenced)
+B = 0x20000
+MIS = 0x10008        # 8-byte aligned only
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return w4.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"W4A16_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"awq_act_scale", "awq_quantize_pack", "w4a16_gemm", "w4a16_gemm_workspace_size",
+            "w4a16_gemm_check", "w4a16_last_error", "w4a16_layout_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_layout_version(lib):
+    assert lib.w4a16_layout_version() == 1
+
+
+def _err(lib):
+    return lib.w4a16_last_error().decode()
+
+
+def test_quantize_pack_validation(lib):
+    qp = lib.awq_quantize_pack
+    assert qp(None, None, 8, 128, 128, 4, 0, A, A, A, None) == ERR_ARG
+    assert "null" in _err(lib)
+    assert qp(A, None, 0, 128, 128, 4, 0, A, A, A, None) == ERR_ARG
+    assert qp(A, None, 8, 128, 128, 4, 7, A, A, A, None) == ERR_ARG
+    assert qp(A, None, 8, 128, 64, 4, 0, A, A, A, None) == ERR_UNSUPPORTED
+    assert qp(A, None, 8, 128, 128, 5, 0, A, A, A, None) == ERR_UNSUPPORTED
+    assert qp(A, None, 8, 128, 128, 2, 1, A, A, A, None) == ERR_UNSUPPORTED
+    assert qp(A, None, 8, 200, 128, 4, 0, A, A, A, None) == ERR_SHAPE
+    assert qp(MIS, None, 8, 128, 128, 4, 0, A, A, A, None) == ERR_ALIGN
+    assert qp(A, MIS, 8, 128, 128, 4, 0, A, A, A, None) == ERR_ALIGN
+    assert qp(A, None, 8, 128, 128, 4, 0, A, A, MIS, None) == ERR_ALIGN
+    assert qp(A, None, 1 << 20, 1 << 12, 128, 4, 0, A, A, A, None) == ERR_SHAPE
+
+
+def test_act_scale_validation(lib):
+    f = lib.awq_act_scale
+    assert f(None, 4, 8, 0.5, A, None) == ERR_ARG
+    assert f(A, 0, 8, 0.5, A, None) == ERR_ARG
+    assert f(A, 4, 8, float("nan"), A, None) == ERR_ARG
+    assert f(A, 4, 8, float("inf"), A, None) == ERR_ARG
+    assert f(MIS, 4, 8, 0.5, A, None) == ERR_ALIGN
+
+
+def test_workspace_size(lib):
+    ws = lib.w4a16_gemm_workspace_size
+    assert ws(1, 8192, 8192, 128) > 8192 * 4
+    assert ws(4, 100, 256, 128) >= 4 * 100 * 4
+    assert ws(0, 8, 128, 128) == 0
+    assert ws(65, 8, 128, 128) == 0
+    assert ws(1, 8, 100, 128) == 0
+    assert ws(1, 8, 128, 64) == 0
+
+
+def test_gemm_validation(lib):
+    g = lib.w4a16_gemm
+    need = lib.w4a16_gemm_workspace_size(1, 64, 256, 128)
+    assert g(None, A, A, A, 1, 64, 256, 128, A, B, need, None) == ERR_ARG
+    assert g(A, A, A, A, 0, 64, 256, 128, A, B, need, None) == ERR_ARG
+    assert g(A, A, A, A, 1, 64, 256, 64, A, B, need, None) == ERR_UNSUPPORTED
+    assert g(A, A, A, A, 1, 64, 200, 128, A, B, need, None) == ERR_SHAPE
+    assert g(A, A, A, A, 65, 64, 256, 128, A, B, need, None) == ERR_UNSUPPORTED
+    assert g(MIS, A, A, A, 1, 64, 256, 128, A, B, need, None) == ERR_ALIGN
+    assert g(A, A, A, A, 1, 64, 256, 128, MIS, B, need, None) == ERR_ALIGN
+    assert g(A, A, A, A, 1, 64, 256, 128, A, None, need, None) == ERR_WORKSPACE
+    assert g(A, A, A, A, 1, 64, 256, 128, A, B, need - 1, None) == ERR_WORKSPACE
+    assert "workspace" in _err(lib)
+    assert g(A, A, A, A, 1, 64, 256, 128, A, MIS, need, None) == ERR_ALIGN
+
+
+def test_gemm_check_validation(lib):
+    assert lib.w4a16_gemm_check(None, None) == ERR_ARG
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(w4.W4A16Error):
+        w4.awq_quantize_pack(torch.zeros((8, 128), dtype=torch.float16))
+    with pytest.raises(w4.W4A16Error):
+        w4.w4a16_gemm(torch.zeros((1, 128), dtype=torch.float16), torch.zeros((8, 16), dtype=torch.int32),
+                      torch.zeros((8, 1), dtype=torch.float16), torch.zeros((8, 1), dtype=torch.float16))

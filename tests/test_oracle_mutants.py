@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 MUTANTS = {
     "step_denominator_2^N": ("delta = ((mx - mn) / F64(qmax)).astype(F16)",
                              "delta = ((mx - mn) / F64(qmax + 1)).astype(F16)"),
-    "zero_point_sign": ("z = np.clip(np.rint(-mn / delta.astype(F64)), 0, qmax)",
-                        "z = np.clip(np.rint(mn / delta.astype(F64)), 0, qmax)"),
+    "zero_point_sign": ("z = np.clip(np.rint(-mn / delta.astype(F64)), 0, qmax) + 0.0",
+                        "z = np.clip(np.rint(mn / delta.astype(F64)), 0, qmax) + 0.0"),
     "round_half_up": ("u = np.clip(np.rint(g / d) + zz, 0, 2 ** bits - 1)",
                       "u = np.clip(np.floor(g / d + 0.5) + zz, 0, 2 ** bits - 1)"),
     "joint_rounding": ("u = np.clip(np.rint(g / d) + zz, 0, 2 ** bits - 1)",

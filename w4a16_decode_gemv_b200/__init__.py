@@ -1,0 +1,181 @@
+"""Python binding of the w4a16 C ABI (include/w4a16.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libw4a16.so``.  PyTorch supplies device memory and the current
+stream.  There is no CPU fallback: if the library is missing or the tensors
+are not on a CUDA device, the call raises.
+
+Packed weights are uint32 bit patterns kept in ``torch.int32`` tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+ASYM = 0
+SYM = 1
+GROUP = 128
+LAYOUT_VERSION = 1
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
+_lib = None
+_workspaces: dict = {}
+
+
+class W4A16Error(RuntimeError):
+    pass
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libw4a16.so once and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise W4A16Error(f"{_LIB_PATH} is missing: build it with `python -m w4a16_decode_gemv_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i, d, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+    lib.awq_act_scale.argtypes = [vp, i, i, d, vp, vp]
+    lib.awq_act_scale.restype = i
+    lib.awq_quantize_pack.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp]
+    lib.awq_quantize_pack.restype = i
+    lib.w4a16_gemm_workspace_size.argtypes = [i, i, i, i]
+    lib.w4a16_gemm_workspace_size.restype = sz
+    lib.w4a16_gemm.argtypes = [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
+    lib.w4a16_gemm.restype = i
+    lib.w4a16_gemm_check.argtypes = [vp, vp]
+    lib.w4a16_gemm_check.restype = i
+    lib.w4a16_last_error.argtypes = []
+    lib.w4a16_last_error.restype = ctypes.c_char_p
+    lib.w4a16_layout_version.argtypes = []
+    lib.w4a16_layout_version.restype = i
+    if lib.w4a16_layout_version() != LAYOUT_VERSION:
+        raise W4A16Error("libw4a16.so has an unexpected packed-layout version")
+    _lib = lib
+    return lib
+
+
+def _check(status: int, name: str) -> None:
+    if status != 0:
+        msg = load_library().w4a16_last_error().decode(errors="replace")
+        raise W4A16Error(f"{name} failed with status {status}: {msg}")
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _expect(t: torch.Tensor, dtype, shape, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise W4A16Error(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise W4A16Error(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise W4A16Error(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise W4A16Error(f"{name} must be contiguous")
+
+
+def awq_act_scale(X: torch.Tensor, alpha: float = 0.5, out: torch.Tensor | None = None) -> torch.Tensor:
+    """s[k] = fp16(mean_t |X[t, k]| ** alpha) for calibration activations X fp16 [T, K]."""
+    lib = load_library()
+    if X.dim() != 2:
+        raise W4A16Error("X must be 2-D [T, K]")
+    T, K = X.shape
+    _expect(X, torch.float16, (T, K), "X")
+    s = torch.empty(K, dtype=torch.float16, device=X.device) if out is None else out
+    _expect(s, torch.float16, (K,), "out")
+    with torch.cuda.device(X.device):
+        _check(lib.awq_act_scale(_ptr(X), T, K, float(alpha), _ptr(s), _stream(X.device)), "awq_act_scale")
+    return s
+
+
+def awq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None = None, group: int = GROUP, bits: int = 4,
+                      mode: int = ASYM, out=None):
+    """AWQ-scale, group-quantize and pack W fp16 [N, K].
+
+    Returns (qweight int32 [N, K/8] holding uint32 words of layout v1,
+    scales fp16 [N, K/group], zeros fp16 [N, K/group]).
+    """
+    lib = load_library()
+    if W.dim() != 2:
+        raise W4A16Error("W must be 2-D [N, K]")
+    N, K = W.shape
+    _expect(W, torch.float16, (N, K), "W")
+    if s is not None:
+        _expect(s, torch.float16, (K,), "s")
+    if group <= 0 or K % group:
+        raise W4A16Error(f"K={K} must be a multiple of group={group}")
+    if out is None:
+        qweight = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+        scales = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+        zeros = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+    else:
+        qweight, scales, zeros = out
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(scales, torch.float16, (N, K // group), "scales")
+    _expect(zeros, torch.float16, (N, K // group), "zeros")
+    with torch.cuda.device(W.device):
+        _check(lib.awq_quantize_pack(_ptr(W), _ptr(s), N, K, group, bits, mode, _ptr(qweight), _ptr(scales),
+                                     _ptr(zeros), _stream(W.device)), "awq_quantize_pack")
+    return qweight, scales, zeros
+
+
+def gemm_workspace_size(M: int, N: int, K: int, group: int = GROUP) -> int:
+    return int(load_library().w4a16_gemm_workspace_size(M, N, K, group))
+
+
+def workspace_for(device: torch.device, nbytes: int) -> torch.Tensor:
+    """A zero-filled workspace of at least nbytes for the current stream of device.
+
+    The kernels leave it zero-filled after every completed call, so one buffer
+    per (device, stream) is reused across calls.
+    """
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 16), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+               group: int = GROUP, out: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y fp16 [M, N] = x fp16 [M, K] @ dequant(qweight, scales, zeros)^T."""
+    lib = load_library()
+    if x.dim() != 2 or qweight.dim() != 2:
+        raise W4A16Error("x must be [M, K] and qweight [N, K/8]")
+    M, K = x.shape
+    N = qweight.shape[0]
+    _expect(x, torch.float16, (M, K), "x")
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(scales, torch.float16, (N, K // group), "scales")
+    _expect(zeros, torch.float16, (N, K // group), "zeros")
+    y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
+    _expect(y, torch.float16, (M, N), "out")
+    need = gemm_workspace_size(M, N, K, group)
+    if need == 0:
+        raise W4A16Error(f"unsupported sizes M={M} N={N} K={K} group={group}")
+    ws = workspace_for(x.device, need) if workspace is None else workspace
+    with torch.cuda.device(x.device):
+        _check(lib.w4a16_gemm(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
+                              _ptr(ws), ws.numel() * ws.element_size(), _stream(x.device)), "w4a16_gemm")
+    return y
+
+
+def gemm_check(workspace: torch.Tensor) -> None:
+    """Synchronizes and raises if a kernel that used this workspace gave up waiting."""
+    lib = load_library()
+    with torch.cuda.device(workspace.device):
+        _check(lib.w4a16_gemm_check(_ptr(workspace), _stream(workspace.device)), "w4a16_gemm_check")

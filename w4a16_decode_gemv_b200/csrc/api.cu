@@ -1,0 +1,166 @@
+// C ABI of the w4a16 library: argument checks, error reporting, dispatch.
+// The operations themselves are specified in include/w4a16.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/w4a16.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+namespace {
+
+thread_local std::string g_last_error;
+
+w4a16_status fail(w4a16_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+w4a16_status fail(w4a16_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+w4a16_status ok() {
+  g_last_error.clear();
+  return W4A16_OK;
+}
+
+w4a16_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(W4A16_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr long long kMaxElems = 1ll << 31;  // index arithmetic stays in 64 bits; sizes stay sane
+
+}  // namespace
+
+int device_sm_count() {
+  static int cached[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+size_t workspace_bytes(int M, int N, int K) {
+  (void)K;
+  const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
+  const size_t cnt = (row_blocks * 4 + 15) / 16 * 16;
+  return 16 + cnt + static_cast<size_t>(M) * N * 4;
+}
+
+Workspace carve_workspace(void* base, int M, int N, int K) {
+  (void)M;
+  (void)K;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
+  const size_t cnt = (row_blocks * 4 + 15) / 16 * 16;
+  Workspace w;
+  w.status = reinterpret_cast<uint32_t*>(p);
+  w.counters = reinterpret_cast<uint32_t*>(p + 16);
+  w.acc = reinterpret_cast<float*>(p + 16 + cnt);
+  return w;
+}
+
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" {
+
+const char* w4a16_last_error(void) { return g_last_error.c_str(); }
+
+int w4a16_layout_version(void) { return 1; }
+
+w4a16_status awq_act_scale(const void* X, int T, int K, double alpha, void* s, w4a16_stream_t stream) {
+  if (!X || !s) return fail(W4A16_ERR_ARG, "awq_act_scale: null pointer");
+  if (T < 1 || K < 1) return fail(W4A16_ERR_ARG, "awq_act_scale: T=%d K=%d must be >= 1", T, K);
+  if (static_cast<long long>(T) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "awq_act_scale: T*K too large");
+  if (!std::isfinite(alpha)) return fail(W4A16_ERR_ARG, "awq_act_scale: alpha must be finite");
+  if (!aligned16(X) || !aligned16(s)) return fail(W4A16_ERR_ALIGN, "awq_act_scale: pointers must be 16-byte aligned");
+  cudaError_t e = launch_act_scale(static_cast<const __half*>(X), T, K, alpha, static_cast<__half*>(s),
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "awq_act_scale launch");
+  return ok();
+}
+
+w4a16_status awq_quantize_pack(const void* W, const void* s, int N, int K, int group, int bits, w4a16_mode mode,
+                               uint32_t* qweight, void* scales, void* zeros, w4a16_stream_t stream) {
+  if (!W || !qweight || !scales || !zeros) return fail(W4A16_ERR_ARG, "awq_quantize_pack: null pointer");
+  if (N < 1 || K < 1) return fail(W4A16_ERR_ARG, "awq_quantize_pack: N=%d K=%d must be >= 1", N, K);
+  if (mode != W4A16_ASYM && mode != W4A16_SYM) return fail(W4A16_ERR_ARG, "awq_quantize_pack: bad mode %d", mode);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "awq_quantize_pack: group=%d (only 128)", group);
+  if (bits != 3 && bits != 4) return fail(W4A16_ERR_UNSUPPORTED, "awq_quantize_pack: bits=%d (3 or 4)", bits);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "awq_quantize_pack: K=%d not a multiple of group=%d", K, group);
+  if (static_cast<long long>(N) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "awq_quantize_pack: N*K too large");
+  if (!aligned16(W) || (s && !aligned16(s)) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros))
+    return fail(W4A16_ERR_ALIGN, "awq_quantize_pack: pointers must be 16-byte aligned");
+  cudaError_t e = launch_quantize_pack(static_cast<const __half*>(W), static_cast<const __half*>(s), N, K, bits,
+                                       static_cast<int>(mode), qweight, static_cast<__half*>(scales),
+                                       static_cast<__half*>(zeros), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "awq_quantize_pack launch");
+  return ok();
+}
+
+size_t w4a16_gemm_workspace_size(int M, int N, int K, int group) {
+  if (M < 1 || M > kMaxM || N < 1 || K < 1 || group != kGroup || K % group) return 0;
+  return workspace_bytes(M, N, K);
+}
+
+w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scales, const void* zeros, int M, int N,
+                        int K, int group, void* y, void* workspace, size_t workspace_bytes_, w4a16_stream_t stream) {
+  if (!x || !qweight || !scales || !zeros || !y) return fail(W4A16_ERR_ARG, "w4a16_gemm: null pointer");
+  if (M < 1 || N < 1 || K < 1) return fail(W4A16_ERR_ARG, "w4a16_gemm: M=%d N=%d K=%d must be >= 1", M, N, K);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: group=%d (only 128)", group);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "w4a16_gemm: K=%d not a multiple of group=%d", K, group);
+  if (M > kMaxM) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: M=%d (at most %d)", M, kMaxM);
+  if (static_cast<long long>(N) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "w4a16_gemm: N*K too large");
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
+    return fail(W4A16_ERR_ALIGN, "w4a16_gemm: pointers must be 16-byte aligned");
+  const size_t need = workspace_bytes(M, N, K);
+  if (!workspace || workspace_bytes_ < need)
+    return fail(W4A16_ERR_WORKSPACE, "w4a16_gemm: workspace of %zu bytes needed, %zu given", need, workspace_bytes_);
+  if (!aligned16(workspace)) return fail(W4A16_ERR_ALIGN, "w4a16_gemm: workspace must be 16-byte aligned");
+  GemmProblem p{static_cast<const __half*>(x), qweight, static_cast<const __half*>(scales),
+                static_cast<const __half*>(zeros), static_cast<__half*>(y), M, N, K};
+  const Workspace ws = carve_workspace(workspace, M, N, K);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M < 16 && gemv_supports(M, K)) {
+    e = launch_gemv(p, ws, st);
+  } else {
+    e = launch_gemm_tc(p, ws, st);
+  }
+  if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: M=%d K=%d not supported yet", M, K);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm launch");
+  return ok();
+}
+
+w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream) {
+  if (!workspace) return fail(W4A16_ERR_ARG, "w4a16_gemm_check: null workspace");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm_check: stream");
+  uint32_t flag = 0;
+  e = cudaMemcpy(&flag, workspace, sizeof(flag), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm_check: read status");
+  if (flag != kDevOk) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm_check: clear status");
+    return fail(W4A16_ERR_DEVICE, "w4a16_gemm: a kernel gave up waiting for its weight tiles (status %u)", flag);
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace w4a16 {
+
+constexpr int kGroup = 128;        // group size along K (the only one supported)
+constexpr int kMaxGemvM = 4;       // largest M the CUDA-core GEMV handles
+constexpr int kMaxM = 64;          // largest M of w4a16_gemm
+
+// Streaming-multiprocessor count of the current device (cached per device).
+int device_sm_count();
+
+cudaError_t launch_act_scale(const __half* X, int T, int K, double alpha, __half* s, cudaStream_t st);
+
+cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K, int bits, int mode,
+                                 uint32_t* qweight, __half* scales, __half* zeros, cudaStream_t st);
+
+// Workspace of the split-K kernels: [status word | padding to 16 B]
+// [row-block counters, padded to 16 B] [fp32 partial sums M x N].
+struct Workspace {
+  uint32_t* status;
+  uint32_t* counters;
+  float* acc;
+};
+size_t workspace_bytes(int M, int N, int K);
+Workspace carve_workspace(void* base, int M, int N, int K);
+
+struct GemmProblem {
+  const __half* x;
+  const uint32_t* qweight;
+  const __half* scales;
+  const __half* zeros;
+  __half* y;
+  int M, N, K;
+};
+
+// Can the CUDA-core GEMV run this problem (M and shared-memory budget)?
+bool gemv_supports(int M, int K);
+cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+
+}  // namespace w4a16

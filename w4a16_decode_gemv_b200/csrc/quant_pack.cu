@@ -1,0 +1,219 @@
+// AWQ calibration scale and the quantize + pack kernel.
+//
+// Pages (by title and section):
+//  - "MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading guide, §AWQ:
+//    scale salient input channels by s = s_X^alpha (slides 25-28) and quantize
+//    with Q(w) = Delta * Round(w / Delta) per group of 128 (slide 26).
+//  - "CMU 11-868 Model Quantization" reading guide, §absmax and zero-point
+//    (lecture slide 10): step from (max - min) / (2^N - 1), a rounded zero point,
+//    clipping to the code range; a zero range is replaced by 1.
+//  - "MIT 6.5940 Lab 4 + Lab 5" reading guide, §Lab 4 setup: calibration
+//    statistic = mean |X| per input channel.
+//  - Lecture 13 guide, §TinyChat (slide 36): codes packed offline so that the
+//    GEMV unpacks them with an AND and a shift (layout v1, include/w4a16.h).
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+namespace {
+
+// ---------------------------------------------------------------------------
+// s[k] = fp16((mean_t |X[t][k]|)^alpha).  One CTA per 64 channels; warp w sums
+// the tokens t = w, w + 8, ...  The fp64 sums of fp16 magnitudes are exact for
+// T <= 8192 (every term is a multiple of 2^-24 below 2^16), so the order of the
+// additions does not change the result.
+// ---------------------------------------------------------------------------
+constexpr int kAsWarps = 8;
+constexpr int kAsChannels = 64;
+
+__global__ void __launch_bounds__(kAsWarps * 32) act_scale_kernel(const __half* __restrict__ X, int T, int K,
+                                                                   double alpha, __half* __restrict__ s) {
+  __shared__ double part[kAsWarps][kAsChannels];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k0 = blockIdx.x * kAsChannels + 2 * lane;
+  double a0 = 0.0, a1 = 0.0;
+  for (int t = warp; t < T; t += kAsWarps) {
+    const __half* row = X + static_cast<size_t>(t) * K;
+    if (k0 < K) a0 += fabs(static_cast<double>(__half2float(row[k0])));
+    if (k0 + 1 < K) a1 += fabs(static_cast<double>(__half2float(row[k0 + 1])));
+  }
+  part[warp][2 * lane] = a0;
+  part[warp][2 * lane + 1] = a1;
+  __syncthreads();
+  if (threadIdx.x < kAsChannels) {
+    const int k = blockIdx.x * kAsChannels + threadIdx.x;
+    if (k < K) {
+      double sum = 0.0;
+#pragma unroll
+      for (int w = 0; w < kAsWarps; ++w) sum += part[w][threadIdx.x];
+      const double mean = sum / static_cast<double>(T);
+      s[k] = __double2half(pow(mean, alpha));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quantize + pack.  A group of 128 input channels is handled by a half-warp:
+// lane h of the half-warp owns channels 8h .. 8h+7, i.e. exactly one packed
+// word of layout v1.  Group statistics are shuffle reductions over the 16 lanes.
+// Each warp iteration covers two groups; kQpUnroll iterations are loaded before
+// any is computed so that enough bytes are in flight.
+// ---------------------------------------------------------------------------
+constexpr int kQpThreads = 256;
+constexpr int kQpHalfWarps = kQpThreads / 16;
+constexpr int kQpUnroll = 4;
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Round(w / d) with Round = half to even, on the exact quotient.  The IEEE fp32
+// quotient decides every half-integer boundary exactly: for fp16 w and d with
+// |w / d| < 2^5 a non-tie quotient lies at least 2^-14 from a half-integer,
+// far beyond the fp32 rounding error, and an exact tie is representable.
+__device__ __forceinline__ float round_quotient(float w, float d) { return rintf(__fdiv_rn(w, d)); }
+
+template <int BITS, int MODE, bool HAS_S>
+__global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half* __restrict__ W,
+                                                                   const __half* __restrict__ s, int N, int K,
+                                                                   uint32_t* __restrict__ qweight,
+                                                                   __half* __restrict__ scales,
+                                                                   __half* __restrict__ zeros) {
+  constexpr int kQmax = (1 << BITS) - 1;
+  constexpr int kHalfRange = 1 << (BITS - 1);
+  const int Kg = K / kGroup;
+  const int Kw = K / 8;
+  const long long total = static_cast<long long>(N) * Kg;
+  const int hl = threadIdx.x & 15;
+  const long long stride = static_cast<long long>(gridDim.x) * kQpHalfWarps;
+  long long g0 = static_cast<long long>(blockIdx.x) * kQpHalfWarps + (threadIdx.x >> 4);
+
+  for (; g0 - (threadIdx.x >> 4) % 2 < total; g0 += stride * kQpUnroll) {
+    uint4 wv[kQpUnroll];
+    uint4 sv[kQpUnroll];
+#pragma unroll
+    for (int u = 0; u < kQpUnroll; ++u) {
+      const long long g = g0 + u * stride;
+      wv[u] = make_uint4(0, 0, 0, 0);
+      sv[u] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // 1.0
+      if (g < total) {
+        const long long n = g / Kg;
+        const int k = static_cast<int>(g - n * Kg) * kGroup + hl * 8;
+        wv[u] = ldg_stream(W + n * K + k);
+        if (HAS_S) sv[u] = __ldg(reinterpret_cast<const uint4*>(s + k));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQpUnroll; ++u) {
+      const long long g = g0 + u * stride;
+      // a1: w' = fp16(W * s), the exact product rounded once (mul.rn.f16x2)
+      __half2 w2[4];
+      w2[0] = as_h2(wv[u].x);
+      w2[1] = as_h2(wv[u].y);
+      w2[2] = as_h2(wv[u].z);
+      w2[3] = as_h2(wv[u].w);
+      if (HAS_S) {
+        w2[0] = __hmul2(w2[0], as_h2(sv[u].x));
+        w2[1] = __hmul2(w2[1], as_h2(sv[u].y));
+        w2[2] = __hmul2(w2[2], as_h2(sv[u].z));
+        w2[3] = __hmul2(w2[3], as_h2(sv[u].w));
+      }
+      // a2: group statistics over the half-warp (all 32 lanes take part)
+      __half d;
+      float zf;
+      if (MODE == 0) {
+        __half2 hi = __hmax2(__hmax2(w2[0], w2[1]), __hmax2(w2[2], w2[3]));
+        __half2 lo = __hmin2(__hmin2(w2[0], w2[1]), __hmin2(w2[2], w2[3]));
+        // (max, min) of this lane's 8 values in one register
+        __half2 mm = __halves2half2(__hmax(__low2half(hi), __high2half(hi)), __hmin(__low2half(lo), __high2half(lo)));
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) {
+          const __half2 other = as_h2(__shfl_xor_sync(0xffffffffu, as_u32(mm), o));
+          mm = __halves2half2(__hmax(__low2half(mm), __low2half(other)), __hmin(__high2half(mm), __high2half(other)));
+        }
+        // a3: Delta = fp16(fp64(max - min) / (2^N - 1)); zero step -> unit range
+        const double mx = static_cast<double>(__low2float(mm));
+        const double mn = static_cast<double>(__high2float(mm));
+        d = __double2half((mx - mn) / static_cast<double>(kQmax));
+        if (__heq(d, __float2half(0.0f))) d = __double2half(1.0 / static_cast<double>(kQmax));
+        // z = clamp(Round(-min / Delta), 0, 2^N - 1) as a non-negative integer
+        const double zq = rint(-mn / static_cast<double>(__half2float(d)));
+        zf = static_cast<float>(static_cast<int>(fmin(fmax(zq, 0.0), static_cast<double>(kQmax))));
+      } else {
+        __half2 a = __hmax2(__hmax2(__habs2(w2[0]), __habs2(w2[1])), __hmax2(__habs2(w2[2]), __habs2(w2[3])));
+        __half am = __hmax(__low2half(a), __high2half(a));
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) {
+          const __half other = __ushort_as_half(
+              static_cast<unsigned short>(__shfl_xor_sync(0xffffffffu, static_cast<unsigned>(__half_as_ushort(am)), o)));
+          am = __hmax(am, other);
+        }
+        // a3: Delta = fp16(max|w'| / 2^(N-1)), z = 2^(N-1)
+        d = __double2half(static_cast<double>(__half2float(am)) / static_cast<double>(kHalfRange));
+        if (__heq(d, __float2half(0.0f))) d = __double2half(1.0 / static_cast<double>(kHalfRange));
+        zf = static_cast<float>(kHalfRange);
+      }
+      if (g >= total) continue;
+      // a4: u = clamp(Round(w' / Delta) + z, 0, 2^N - 1);  a5: pack into layout v1
+      const float df = __half2float(d);
+      uint32_t word = 0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 wf = __half22float2(w2[t]);
+        const float u0 = fminf(fmaxf(round_quotient(wf.x, df) + zf, 0.0f), static_cast<float>(kQmax));
+        const float u1 = fminf(fmaxf(round_quotient(wf.y, df) + zf, 0.0f), static_cast<float>(kQmax));
+        word |= (static_cast<uint32_t>(u0) << (4 * t)) | (static_cast<uint32_t>(u1) << (16 + 4 * t));
+      }
+      const long long n = g / Kg;
+      const int gi = static_cast<int>(g - n * Kg);
+      qweight[n * Kw + gi * 16 + hl] = word;
+      if (hl == 0) {
+        scales[n * Kg + gi] = d;
+        zeros[n * Kg + gi] = __float2half_rn(zf);
+      }
+    }
+  }
+}
+
+template <int BITS, int MODE, bool HAS_S>
+cudaError_t launch_qp(const __half* W, const __half* s, int N, int K, uint32_t* qw, __half* sc, __half* zr,
+                      cudaStream_t st) {
+  const long long groups = static_cast<long long>(N) * (K / kGroup);
+  const long long half_warps_needed = (groups + kQpUnroll - 1) / kQpUnroll;
+  long long blocks = (half_warps_needed + kQpHalfWarps - 1) / kQpHalfWarps;
+  const long long cap = static_cast<long long>(device_sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  quantize_pack_kernel<BITS, MODE, HAS_S>
+      <<<static_cast<unsigned>(blocks), kQpThreads, 0, st>>>(W, s, N, K, qw, sc, zr);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_act_scale(const __half* X, int T, int K, double alpha, __half* s, cudaStream_t st) {
+  const int blocks = (K + kAsChannels - 1) / kAsChannels;
+  act_scale_kernel<<<blocks, kAsWarps * 32, 0, st>>>(X, T, K, alpha, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K, int bits, int mode,
+                                 uint32_t* qw, __half* sc, __half* zr, cudaStream_t st) {
+  const bool hs = s != nullptr;
+#define W4A16_QP_CASE(B, MO)                                                         \
+  if (bits == B && mode == MO)                                                       \
+    return hs ? launch_qp<B, MO, true>(W, s, N, K, qw, sc, zr, st)                   \
+              : launch_qp<B, MO, false>(W, s, N, K, qw, sc, zr, st);
+  W4A16_QP_CASE(4, 0)
+  W4A16_QP_CASE(4, 1)
+  W4A16_QP_CASE(3, 0)
+  W4A16_QP_CASE(3, 1)
+#undef W4A16_QP_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace w4a16
