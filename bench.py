@@ -20,6 +20,7 @@ during the timed region.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import hashlib
 import json
 import os
@@ -31,6 +32,13 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+
+faulthandler.enable()
+
+
+def log(msg):
+    print(f"[bench {time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
+
 
 METRIC = "W4A16 GEMV effective GB/s & % of B200 HBM peak (M=1, K=N=8192); us/layer"
 LAYERS = 16
@@ -111,11 +119,17 @@ class ClockSampler:
             import pynvml
             import torch
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(torch_device).pci_bus_id
-            try:
-                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-            except Exception:
-                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            # match the CUDA device to its NVML handle by UUID (robust to CUDA_VISIBLE_DEVICES)
+            want = str(torch.cuda.get_device_properties(torch_device).uuid).lower().replace("gpu-", "")
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else str(u)).lower().replace("gpu-", "")
+                if u == want:
+                    self._h = h
+                    break
+            if self._h is None:
+                raise RuntimeError(f"no NVML device with UUID {want}")
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self._nv = pynvml
         except Exception as e:  # no NVML: report that instead of clocks
@@ -195,12 +209,16 @@ def run_ours(args, dist):
     torch.manual_seed(0)
 
     # ---- inputs: the 8192^2 layer of the LLaMA-65B set, quantized on the GPU
+    log("drawing inputs")
     (layer,) = inputs.layer_set(inputs.LLAMA65B, only="attn_8192x8192")
     W = torch.from_numpy(layer.W).to(dev)
+    log("quantize")
     q0, s0, z0 = w4.awq_quantize_pack(W)
     del W
     # parity first: sampled rows against the oracle
+    log("parity")
     parity = check_parity(layer, q0, s0, z0, dev)
+    log("copies")
     layers = []
     for l in range(args.layers):
         if l == 0:
@@ -217,13 +235,16 @@ def run_ours(args, dist):
         for l, (q, s, z) in enumerate(layers):
             w4.w4a16_gemm(xbufs[l], q, s, z, out=xbufs[l + 1], workspace=ws)
 
+    log("eager token")
     with torch.cuda.stream(stream):
         xbufs[0].copy_(x0)
         token()
         torch.cuda.synchronize()
+        log("capture")
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             token()
+        log("warmup")
         for _ in range(args.warmup):
             graph.replay()
         torch.cuda.synchronize()
@@ -233,6 +254,7 @@ def run_ours(args, dist):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
+    log("timed region")
     with ClockSampler(dev) as clk:
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -250,6 +272,7 @@ def run_ours(args, dist):
     us_layer = ms_per_step * 1e3 / L
 
     # ---- e2e through the public API (eager), pinned host input/output every step
+    log("e2e")
     e2e = measure_e2e(args, layers, ws, x0, dev, stream, dist)
 
     out = None
@@ -272,8 +295,10 @@ def run_ours(args, dist):
                "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * L,
                "clocks": clk.summary(), "parity": parity}
         if not args.skip_extras:
+            log("other workloads")
             out["workloads"] = other_workloads(args, dev)
         if dist.world == 1 and not args.skip_cpu:
+            log("cpu baseline")
             out["cpu_baseline"] = cpu_baseline(layer, q0, s0, z0, args.cpu_seconds)
     del graph
     dist.close()

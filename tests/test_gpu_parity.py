@@ -143,9 +143,12 @@ def test_quantize_edge_groups(dev, bits, mode):
     G = _edge_groups()
     W = G.reshape(-1, 256) if G.shape[0] % 2 == 0 else G
     assert_bit_exact(*quantize_both(W, None, bits, mode, dev), "edge groups")
-    # AWQ scale that hits exact fp16 product ties
-    s = np.full(W.shape[1], 1.5, dtype=F16)
-    assert_bit_exact(*quantize_both(W, s, bits, mode, dev), "edge groups, s=1.5")
+    # AWQ scale that hits exact fp16 product ties; the near-65504 group is left
+    # out because W * 1.5 would overflow fp16 (outside the stated precondition)
+    G2 = np.delete(G, 7, axis=0)
+    W2 = G2.reshape(-1, 256) if G2.shape[0] % 2 == 0 else G2
+    s = np.full(W2.shape[1], 1.5, dtype=F16)
+    assert_bit_exact(*quantize_both(W2, s, bits, mode, dev), "edge groups, s=1.5")
 
 
 def _sweep_weight():
@@ -153,18 +156,22 @@ def _sweep_weight():
     allv = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16).view(F16)
     allv = allv[np.isfinite(allv)].astype(np.float64)
     rows = []
-    for e in range(-24, 16):
-        hi = 2.0 ** (e + 1)
-        lo = -1.5 * 2.0 ** e
-        vals = allv[(allv >= lo) & (allv <= hi)]
+
+    def add(lo, hi, vals):
         for start in range(0, len(vals), 126):
-            chunk = vals[start:start + 126]
-            g = np.full(128, 0.0)
+            g = np.zeros(128)
             g[0], g[1] = lo, hi
+            chunk = vals[start:start + 126]
             g[2:2 + len(chunk)] = chunk
             rows.append(g)
-    rows.append(np.concatenate([[-65504.0, 65504.0], np.linspace(-65504, 65504, 126)]))
+
+    for e in range(-24, 15):
+        lo, hi = float(F16(-1.5 * 2.0 ** e)), float(F16(2.0 ** (e + 1)))
+        add(lo, hi, allv[(allv >= lo) & (allv <= hi)])
+    add(-65504.0, 65504.0, allv[np.abs(allv) >= 2.0 ** 14])   # top binades, widest anchors
     W = np.stack(rows)
+    covered = np.unique(W.astype(F16).view(np.uint16))
+    assert np.isin(allv.astype(F16).view(np.uint16), covered).all()
     if W.shape[0] % 2:
         W = np.vstack([W, np.zeros((1, 128))])
     return W.reshape(-1, 256).astype(F16)

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <string>
 
 #include "../../include/w4a16.h"
@@ -50,6 +51,14 @@ int device_sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("W4A16_NO_PDL");
+    return !(v && v[0]);
+  }();
+  return on;
 }
 
 size_t workspace_bytes(int M, int N, int K) {
@@ -136,7 +145,9 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   const Workspace ws = carve_workspace(workspace, M, N, K);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (M < 16 && gemv_supports(M, K)) {
+  if (M == 1 && gemv_m1_supports(N, K)) {
+    e = launch_gemv_m1(p, ws.status, st);
+  } else if (M < 16 && gemv_supports(M, K)) {
     e = launch_gemv(p, ws, st);
   } else {
     e = launch_gemm_tc(p, ws, st);

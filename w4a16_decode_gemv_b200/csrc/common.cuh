@@ -87,6 +87,18 @@ __device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// 2-D tiled tensor copy global -> this CTA's shared memory (TMA), completion
+// counted on `bar` in bytes.  x is the innermost coordinate (elements); x times
+// the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy) accesses to the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -125,5 +137,58 @@ __device__ __forceinline__ void fma2_f16_f32(uint32_t a, uint32_t b, float& acc_
       : "+f"(acc_lo), "+f"(acc_hi)
       : "r"(a), "r"(b));
 }
+
+
+// ---- packed fp32 pairs (sm_100: one instruction for two fp32 lanes) ----------
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return f2_pack(__float_as_uint(lo), __float_as_uint(hi));
+}
+
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// ---- programmatic dependent launch ---------------------------------------------
+// Lets the next kernel on the stream begin launching (it still waits for this
+// grid's completion in griddep_wait before using its results).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Blocks until the previous grid on the stream has completed and its memory
+// operations are visible.  A no-op when the kernel was not launched with
+// programmatic stream serialization.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Magic-number unpack into fp32: (w & m) | 0x4B000000 reads as 2^23 + (w & m)
+// for any mask m below bit 23, so a nibble at bit 4t becomes 2^23 + 2^(4t) q.
+constexpr uint32_t kMagic23 = 0x4B000000u;
 
 }  // namespace w4a16

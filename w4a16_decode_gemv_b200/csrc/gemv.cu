@@ -1,27 +1,31 @@
-// Split-K W4A16 GEMV on CUDA cores, for M <= kMaxGemvM.
+// Split-K W4A16 GEMV on CUDA cores for small M (up to kMaxGemvM).
 //
 //   y[m][n] = sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k]
 //
 // Decode is a GEMV: every weight is read once per token and the time goes into
 // reading weights ("MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading
 // guide, §"why W8A8 is not enough", slides 19-20; "CMU 11-868 Model
-// Quantization" guide, §"back to the question").  So the kernel is built to
-// stream the packed weights at HBM speed and to keep the dequantization (AND,
-// OR, one fp16 subtract per pair: Lecture 13 guide, §TinyChat, slides 36-37)
-// and the fp32 multiply-adds under the memory time.
+// Quantization" guide, §"back to the question").  The kernels stream the packed
+// weights at HBM speed and keep the dequantization (an AND/OR per code and one
+// subtraction per pair: Lecture 13 guide, §TinyChat, slides 36-37) and the fp32
+// multiply-adds under the memory time.
 //
-// Work split.  The weight is cut into units of 4 rows x 1024 input channels
-// (2 KiB of codes).  Units are ordered row-block-major and dealt to all warps
-// of a persistent grid (one 16-warp CTA per SM) in contiguous, equal ranges.
-// Each warp streams its own units through a private ring of shared-memory
-// stages filled by bulk copies (TMA) that complete on an mbarrier, so every SM
-// keeps about 100 KiB of weights in flight.  Lane l owns 32 consecutive input
-// channels (a quarter group) of each unit row: one 16-byte shared-memory read
-// yields its 4 words.  Partial sums stay in registers while a warp's units
-// share a row block; when the row block changes the warp reduces them with
-// shuffles and either writes y (it covered the whole row) or adds them into the
-// fp32 workspace, the last contributor of a row block converting to fp16 and
-// zeroing the workspace behind it.
+// Work split.  The weight is cut into units of R rows x 1024 input channels.
+// Units are ordered row-block-major and dealt to all warps of a persistent grid
+// (one 16-warp CTA per SM) in contiguous, equal ranges.  Each warp streams its
+// own units through a private ring of shared-memory stages filled by bulk copies
+// (TMA) that complete on an mbarrier, so every SM keeps ~100-190 KiB of weights
+// in flight.  Lane l owns 32 consecutive input channels (a quarter group) of
+// each unit row: one 16-byte shared-memory read yields its 4 words.  Partial
+// sums stay in registers while a warp's units share a row block; when the row
+// block changes the warp reduces them with shuffles and either writes y (it
+// covered the whole row) or adds them into the fp32 workspace, the last
+// contributor of a row block converting to fp16 and zeroing the workspace behind it.
+//
+// This file holds the kernel for M = 2..4 (and for M = 1 when K is too large
+// for the dedicated M = 1 kernel of gemv_m1.cu): units of 4 rows, codes
+// unpacked into exact fp16 pairs (u - z) and mixed fp16 x fp16 -> fp32
+// multiply-adds.
 #include "common.cuh"
 #include "internal.h"
 
@@ -30,9 +34,7 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kUnitRows = 4;
-constexpr int kUnitWords = 128;                          // 1024 input channels
-constexpr int kUnitBytes = kUnitRows * kUnitWords * 4;   // 2 KiB
+constexpr int kUnitWords = 128;  // 1024 input channels per unit row
 constexpr int kMaxSmem = 227 * 1024;
 
 struct GemvArgs {
@@ -48,7 +50,7 @@ struct GemvArgs {
   int Kw, Kg;          // words and groups per row
   int units_k;         // units per row block
   int total_units;
-  int x_bytes;         // shared-memory bytes reserved for x (multiple of 128)
+  int x_bytes;         // shared-memory bytes reserved for the activations
 };
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -65,15 +67,24 @@ __device__ __forceinline__ uint32_t ld_nc_u16(const __half* p) {
   return v;
 }
 
-// Issues the bulk copies of unit u into a ring slot.  Lane r < rows copies row r.
-__device__ __forceinline__ void issue_unit(const GemvArgs& a, int u, uint8_t* slot, uint64_t* bar, int lane,
-                                           uint64_t pol) {
-  const int rb = u / a.units_k;
-  const int kc = u - rb * a.units_k;
-  const int n0 = rb * kUnitRows;
+// This warp's contiguous range [u0, u0 + cnt) of the units.
+__device__ __forceinline__ void warp_range(const GemvArgs& a, int warp, int& u0, int& cnt) {
+  const int gw = blockIdx.x * kWarps + warp;
+  const int nw = gridDim.x * kWarps;
+  const int base = a.total_units / nw;
+  const int rem = a.total_units - base * nw;
+  u0 = gw * base + min(gw, rem);
+  cnt = base + (gw < rem ? 1 : 0);
+}
+
+// Issues the bulk copies of unit (rb, kc) of R rows into a ring slot.  Lane r < rows copies row r.
+template <int R>
+__device__ __forceinline__ void issue_unit(const GemvArgs& a, int rb, int kc, uint8_t* slot, uint64_t* bar,
+                                           int lane, uint64_t pol) {
+  const int n0 = rb * R;
   const int j0 = kc * kUnitWords;
-  const int rows = min(kUnitRows, a.N - n0);
-  const int words = min(kUnitWords, a.Kw - j0);   // a multiple of 16
+  const int rows = min(R, a.N - n0);
+  const int words = min(kUnitWords, a.Kw - j0);  // a multiple of 16
   const uint32_t row_bytes = static_cast<uint32_t>(words) * 4u;
   if (lane == 0) mbar_arrive_expect_tx(bar, row_bytes * static_cast<uint32_t>(rows));
   __syncwarp();
@@ -83,48 +94,61 @@ __device__ __forceinline__ void issue_unit(const GemvArgs& a, int u, uint8_t* sl
 }
 
 // Delta (low 16 bits) and z (high 16 bits) of this lane's group for each unit row.
-__device__ __forceinline__ void load_dz(const GemvArgs& a, int u, int lane, uint32_t (&dz)[kUnitRows]) {
-  const int rb = u / a.units_k;
-  const int kc = u - rb * a.units_k;
+template <int R>
+__device__ __forceinline__ void load_dz(const GemvArgs& a, int rb, int kc, int lane, uint32_t (&dz)[R]) {
   const int g = kc * (kUnitWords / 16) + (lane >> 2);
+  const int n0 = rb * R;
+  const __half* sp = a.scales + static_cast<size_t>(n0) * a.Kg + g;
+  const __half* zp = a.zeros + static_cast<size_t>(n0) * a.Kg + g;
 #pragma unroll
-  for (int r = 0; r < kUnitRows; ++r) {
-    const int n = rb * kUnitRows + r;
+  for (int r = 0; r < R; ++r) {
     dz[r] = 0;
-    if (n < a.N && g < a.Kg) {
-      const size_t o = static_cast<size_t>(n) * a.Kg + g;
-      dz[r] = ld_nc_u16(a.scales + o) | (ld_nc_u16(a.zeros + o) << 16);
-    }
+    if (n0 + r < a.N && g < a.Kg) dz[r] = ld_nc_u16(sp + r * a.Kg) | (ld_nc_u16(zp + r * a.Kg) << 16);
   }
 }
 
-// Reduces acc[4][MT] over the warp and writes / accumulates the row block.
-template <int MT>
-__device__ __forceinline__ void flush_rows(const GemvArgs& a, int rb, int contrib, float (&acc)[kUnitRows][MT],
+// Sums v[R] (one partial per unit row) over the 32 lanes.  Lane bits 0..log2(R)-1
+// select the row whose total the lane returns; lanes 0..R-1 hold distinct rows.
+template <int R>
+__device__ __forceinline__ float butterfly_rows(const float (&v)[R], int lane, int& row) {
+  float t[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) t[j] = v[j];
+  row = 0;
+  int level = 0;
+#pragma unroll
+  for (int h = R / 2; h >= 1; h /= 2, ++level) {
+    const bool b = (lane >> level) & 1;
+#pragma unroll
+    for (int j = 0; j < h; ++j) {
+      const float keep = b ? t[h + j] : t[j];
+      const float send = b ? t[j] : t[h + j];
+      t[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << level);
+    }
+    row += b ? h : 0;
+  }
+  float k = t[0];
+#pragma unroll
+  for (int o = R; o < 32; o <<= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+  return k;
+}
+
+// Reduces acc[R][MT] over the warp and writes (the warp covered the whole row
+// block) or accumulates into the workspace (the last contributor converts).
+template <int R, int MT>
+__device__ __forceinline__ void flush_rows(const GemvArgs& a, int rb, int contrib, const float (&acc)[R][MT],
                                            int lane) {
-  const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
   float tot[MT];
+  int r = 0;
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
-    // xor 1: even lanes keep rows {0,1}, odd lanes rows {2,3}
-    float k0 = b0 ? acc[2][m] : acc[0][m];
-    float k1 = b0 ? acc[3][m] : acc[1][m];
-    const float s0 = b0 ? acc[0][m] : acc[2][m];
-    const float s1 = b0 ? acc[1][m] : acc[3][m];
-    k0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-    k1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-    // xor 2: keep one of the two rows
-    float k = b1 ? k1 : k0;
-    const float s = b1 ? k0 : k1;
-    k += __shfl_xor_sync(0xffffffffu, s, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 16);
-    tot[m] = k;
+    float v[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) v[j] = acc[j][m];
+    tot[m] = butterfly_rows<R>(v, lane, r);
   }
-  const int r = (b0 ? 2 : 0) + (b1 ? 1 : 0);
-  const int n = rb * kUnitRows + r;
-  const bool writer = lane < 4 && n < a.N;
+  const int n = rb * R + r;
+  const bool writer = lane < R && n < a.N;
   if (contrib == a.units_k) {
     if (writer) {
 #pragma unroll
@@ -141,8 +165,8 @@ __device__ __forceinline__ void flush_rows(const GemvArgs& a, int rb, int contri
   __threadfence();
   __syncwarp();
   uint32_t last = 0;
-  if (lane == 0) last = (atomicAdd(a.ws_cnt + rb, static_cast<uint32_t>(contrib)) + contrib ==
-                         static_cast<uint32_t>(a.units_k));
+  if (lane == 0)
+    last = (atomicAdd(a.ws_cnt + rb, static_cast<uint32_t>(contrib)) + contrib == static_cast<uint32_t>(a.units_k));
   last = __shfl_sync(0xffffffffu, last, 0);
   if (last) {
     __threadfence();
@@ -158,22 +182,32 @@ __device__ __forceinline__ void flush_rows(const GemvArgs& a, int rb, int contri
   }
 }
 
-template <int MT, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs a) {
+// Records a timed-out wait and lets the copies already in flight land.
+template <int STAGES>
+__device__ void bail_out(const GemvArgs& a, uint64_t* bars, int i, int cnt, int lane) {
+  if (lane == 0) atomicOr(a.ws_status, kDevWaitTimeout);
+  for (int j = i + 1; j < cnt && j < i + STAGES; ++j)
+    mbar_wait_bounded(&bars[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u);
+}
+
+// ===========================================================================
+// M = 1..4 (M = 1 only when the dedicated kernel in gemv_m1.cu cannot run)
+// ===========================================================================
+constexpr int kRm = 4;
+constexpr int kUnitMBytes = kRm * kUnitWords * 4;  // 2 KiB
+
+// XS: x is staged in shared memory (when M*K fp16 fits); otherwise each lane
+// reads its activations from global memory (L1/L2 resident).
+template <int MT, int STAGES, bool XS>
+__global__ void __launch_bounds__(kThreads, 1) gemv_multi_kernel(const GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const __half* xs = reinterpret_cast<const __half*>(smem);
-  uint8_t* ring = smem + a.x_bytes + warp * (STAGES * kUnitBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.x_bytes + kWarps * STAGES * kUnitBytes) + warp * STAGES;
+  uint8_t* ring = smem + a.x_bytes + warp * (STAGES * kUnitMBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.x_bytes + kWarps * STAGES * kUnitMBytes) + warp * STAGES;
 
-  // this warp's contiguous unit range
-  const int gw = blockIdx.x * kWarps + warp;
-  const int nw = gridDim.x * kWarps;
-  const int base = a.total_units / nw;
-  const int rem = a.total_units - base * nw;
-  const int u0 = gw * base + min(gw, rem);
-  const int cnt = base + (gw < rem ? 1 : 0);
-
+  int u0, cnt;
+  warp_range(a, warp, u0, cnt);
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
@@ -181,12 +215,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs 
   }
   __syncwarp();
   const uint64_t pol = l2_evict_first_policy();
-#pragma unroll
-  for (int i = 0; i < STAGES; ++i)
-    if (i < cnt) issue_unit(a, u0 + i, ring + i * kUnitBytes, &bars[i], lane, pol);
-
-  // x -> shared memory, once per CTA (M*K fp16; K is a multiple of 128)
   {
+    int rb = u0 / a.units_k, kc = u0 - (u0 / a.units_k) * a.units_k;
+#pragma unroll
+    for (int i = 0; i < STAGES; ++i) {
+      if (i < cnt) issue_unit<kRm>(a, rb, kc, ring + i * kUnitMBytes, &bars[i], lane, pol);
+      if (++kc == a.units_k) kc = 0, ++rb;
+    }
+  }
+
+  if (XS) {  // x -> shared memory, once per CTA (M*K fp16; K is a multiple of 128)
     const int chunks = a.M * a.K / 8;
     const uint4* src = reinterpret_cast<const uint4*>(a.x);
     uint4* dst = reinterpret_cast<uint4*>(smem);
@@ -195,31 +233,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs 
   __syncthreads();
   if (cnt == 0) return;
 
-  float acc[kUnitRows][MT];
+  float acc[kRm][MT];
 #pragma unroll
-  for (int r = 0; r < kUnitRows; ++r)
+  for (int r = 0; r < kRm; ++r)
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
-  int cur_rb = u0 / a.units_k;
+  int rb = u0 / a.units_k;
+  int kc = u0 - rb * a.units_k;
+  int cur_rb = rb;
   int contrib = 0;
-  uint32_t dz_next[kUnitRows];
-  load_dz(a, u0, lane, dz_next);
+  int rb_f = rb, kc_f = kc;
+  for (int j = 0; j < STAGES; ++j)
+    if (++kc_f == a.units_k) kc_f = 0, ++rb_f;
+  uint32_t dz_next[kRm];
+  load_dz<kRm>(a, rb, kc, lane, dz_next);
 
   for (int i = 0; i < cnt; ++i) {
-    const int u = u0 + i;
     const int slot = i % STAGES;
     const uint32_t parity = static_cast<uint32_t>(i / STAGES) & 1u;
-    const int rb = u / a.units_k;
-    const int kc = u - rb * a.units_k;
-    uint32_t dz[kUnitRows];
+    uint32_t dz[kRm];
 #pragma unroll
-    for (int r = 0; r < kUnitRows; ++r) dz[r] = dz_next[r];
-    if (i + 1 < cnt) load_dz(a, u + 1, lane, dz_next);
-
+    for (int r = 0; r < kRm; ++r) dz[r] = dz_next[r];
+    {
+      int rb_n = rb, kc_n = kc + 1;
+      if (kc_n == a.units_k) kc_n = 0, ++rb_n;
+      if (i + 1 < cnt) load_dz<kRm>(a, rb_n, kc_n, lane, dz_next);
+    }
     if (rb != cur_rb) {
-      flush_rows<MT>(a, cur_rb, contrib, acc, lane);
+      flush_rows<kRm, MT>(a, cur_rb, contrib, acc, lane);
 #pragma unroll
-      for (int r = 0; r < kUnitRows; ++r)
+      for (int r = 0; r < kRm; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
       cur_rb = rb;
@@ -228,17 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs 
 
     const int words = min(kUnitWords, a.Kw - kc * kUnitWords);
     const bool active = lane * 4 < words;
-    // this lane's 32 activations of each token, as fp16 pairs
     uint32_t xr[MT][16];
     if (active) {
       const int k0 = kc * (kUnitWords * 8) + lane * 32;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         if (m < a.M) {
-          const uint4* p = reinterpret_cast<const uint4*>(xs + static_cast<size_t>(m) * a.K + k0);
+          const uint4* p = reinterpret_cast<const uint4*>((XS ? xs : a.x) + static_cast<size_t>(m) * a.K + k0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 v = p[c];
+            const uint4 v = XS ? p[c] : ld_nc_v4(p + c);
             xr[m][4 * c + 0] = v.x;
             xr[m][4 * c + 1] = v.y;
             xr[m][4 * c + 2] = v.z;
@@ -252,17 +294,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs 
     }
 
     if (!mbar_wait_bounded(&bars[slot], parity)) {
-      if (lane == 0) atomicOr(a.ws_status, kDevWaitTimeout);
-      // let the copies already in flight land before the CTA can exit
-      for (int j = i + 1; j < cnt && j < i + STAGES; ++j)
-        mbar_wait_bounded(&bars[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u);
+      bail_out<STAGES>(a, bars, i, cnt, lane);
       return;
     }
 
     if (active) {
-      const uint4* wq = reinterpret_cast<const uint4*>(ring + slot * kUnitBytes);
+      const uint4* wq = reinterpret_cast<const uint4*>(ring + slot * kUnitMBytes);
 #pragma unroll
-      for (int r = 0; r < kUnitRows; ++r) {
+      for (int r = 0; r < kRm; ++r) {
         const uint4 w4 = wq[r * (kUnitWords / 4) + lane];
         const __half2 z2 = __half2half2(__ushort_as_half(static_cast<unsigned short>(dz[r] >> 16)));
         const uint32_t nz_lo = as_u32(__hneg2(__hadd2(z2, __floats2half2_rn(1024.0f, 1024.0f))));
@@ -296,39 +335,57 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_w4a16_kernel(const GemvArgs 
       }
     }
     ++contrib;
+    if (++kc == a.units_k) kc = 0, ++rb;
     __syncwarp();
-    if (i + STAGES < cnt) {
-      fence_proxy_async_smem();
-      issue_unit(a, u + STAGES, ring + slot * kUnitBytes, &bars[slot], lane, pol);
-    }
+    if (i + STAGES < cnt) issue_unit<kRm>(a, rb_f, kc_f, ring + slot * kUnitMBytes, &bars[slot], lane, pol);
+    if (++kc_f == a.units_k) kc_f = 0, ++rb_f;
   }
-  flush_rows<MT>(a, cur_rb, contrib, acc, lane);
+  flush_rows<kRm, MT>(a, cur_rb, contrib, acc, lane);
 }
 
-int pick_stages(int x_bytes) {
+// ===========================================================================
+// host side
+// ===========================================================================
+int round128(int b) { return (b + 127) / 128 * 128; }
+
+// Largest ring depth (<= 4) whose shared memory fits next to x_bytes.
+int pick_stages(int x_bytes, int unit_bytes) {
   for (int st = 4; st >= 2; --st)
-    if (x_bytes + kWarps * st * (kUnitBytes + 8) <= kMaxSmem) return st;
+    if (x_bytes + kWarps * st * (unit_bytes + 8) <= kMaxSmem) return st;
   return 0;
 }
 
-int x_smem_bytes(int M, int K) { return (M * K * 2 + 127) / 128 * 128; }
-
-template <int MT, int STAGES>
-cudaError_t launch_t(const GemvArgs& a, int grid, cudaStream_t st) {
-  const int smem = a.x_bytes + kWarps * STAGES * (kUnitBytes + 8);
-  auto kern = gemv_w4a16_kernel<MT, STAGES>;
+// Launches with programmatic stream serialization when `pdl` is set: the
+// kernel may then start while the previous kernel on the stream is finishing,
+// and waits for it (griddepcontrol.wait) before touching x, y or the workspace.
+template <typename Kern>
+cudaError_t launch_kernel(Kern kern, const GemvArgs& a, int grid, int threads, int smem, cudaStream_t st,
+                          bool pdl = false) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int MT>
-cudaError_t launch_m(const GemvArgs& a, int grid, int stages, cudaStream_t st) {
+cudaError_t launch_multi(const GemvArgs& a, int grid, int stages, cudaStream_t st) {
+  const int smem = a.x_bytes + kWarps * stages * (kUnitMBytes + 8);
+  if (a.x_bytes == 0) return launch_kernel(gemv_multi_kernel<MT, 4, false>, a, grid, kThreads, smem, st);
   switch (stages) {
-    case 4: return launch_t<MT, 4>(a, grid, st);
-    case 3: return launch_t<MT, 3>(a, grid, st);
-    case 2: return launch_t<MT, 2>(a, grid, st);
+    case 4: return launch_kernel(gemv_multi_kernel<MT, 4, true>, a, grid, kThreads, smem, st);
+    case 3: return launch_kernel(gemv_multi_kernel<MT, 3, true>, a, grid, kThreads, smem, st);
+    case 2: return launch_kernel(gemv_multi_kernel<MT, 2, true>, a, grid, kThreads, smem, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -336,8 +393,8 @@ cudaError_t launch_m(const GemvArgs& a, int grid, int stages, cudaStream_t st) {
 }  // namespace
 
 bool gemv_supports(int M, int K) {
-  if (M < 1 || M > kMaxGemvM) return false;
-  return pick_stages(x_smem_bytes(M, K)) > 0;
+  (void)K;
+  return M >= 1 && M <= kMaxGemvM;
 }
 
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
@@ -356,18 +413,20 @@ cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t 
   a.Kw = p.K / 8;
   a.Kg = p.K / kGroup;
   a.units_k = (a.Kw + kUnitWords - 1) / kUnitWords;
-  const int row_blocks = (p.N + kUnitRows - 1) / kUnitRows;
-  a.total_units = row_blocks * a.units_k;
-  a.x_bytes = x_smem_bytes(p.M, p.K);
-  const int stages = pick_stages(a.x_bytes);
-  if (stages == 0) return cudaErrorInvalidValue;
   const int sms = device_sm_count();
-  int grid = (a.total_units + kWarps - 1) / kWarps;
-  if (grid > sms) grid = sms;
-  switch (p.M <= 1 ? 1 : p.M <= 2 ? 2 : 4) {
-    case 1: return launch_m<1>(a, grid, stages, st);
-    case 2: return launch_m<2>(a, grid, stages, st);
-    default: return launch_m<4>(a, grid, stages, st);
+  const int row_blocks = (p.N + kRm - 1) / kRm;
+  a.total_units = row_blocks * a.units_k;
+  a.x_bytes = round128(p.M * p.K * 2);
+  int stages = pick_stages(a.x_bytes, kUnitMBytes);
+  if (stages == 0) {  // x does not fit next to a 2-stage ring: read it from global memory
+    a.x_bytes = 0;
+    stages = 4;
+  }
+  const int grid = min(sms, (a.total_units + kWarps - 1) / kWarps);
+  switch (p.M) {
+    case 1: return launch_multi<1>(a, grid, stages, st);
+    case 2: return launch_multi<2>(a, grid, stages, st);
+    default: return launch_multi<4>(a, grid, stages, st);
   }
 }
 

@@ -1,0 +1,384 @@
+// W4A16 decode GEMV for M = 1 on CUDA cores.
+//
+//   y[n] = sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[k]
+//
+// Decode is a GEMV: every weight is read once per token and the time goes into
+// reading weights ("MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading
+// guide, §"why W8A8 is not enough", slides 19-20; "CMU 11-868 Model
+// Quantization" guide, §"back to the question").  The codes are unpacked with
+// bit masks and the dequantization is fused into the product (Lecture 13 guide,
+// §TinyChat, slides 36-37).
+//
+// Work split.  Row blocks of 4 rows are dealt to the CTAs (one per SM) in
+// contiguous, balanced ranges, so a CTA owns whole rows and no partial sum
+// leaves the SM.  A CTA's row blocks are cut into units of 4 rows x 2048 input
+// channels (4 KiB of codes plus the 4 x 16 Delta and z of those rows), and warp
+// w of the CTA takes units w, w + 16, w + 32, ...  Each warp streams its own
+// units through a private ring of shared-memory stages: one lane issues a 2-D
+// tensor copy (TMA, box of 4 rows x 256 words, zero fill past the matrix edge)
+// per unit and all lanes copy the Delta / z tile with cp.async, all completing
+// on the stage's mbarrier.  Many warps issuing copies
+// at once keep far more bytes in flight than one producer could.  Each warp
+// reduces a unit's 4 row partials across its lanes with shuffles and stores
+// them in a shared slot of their own; at the end the CTA adds the slots of each
+// row in a fixed order, so y does not depend on timing.
+//
+// Arithmetic.  Codes are unpacked straight into fp32 by one AND each: a nibble
+// at bit position b <= 19 of a word w, isolated as (w & 0xF<<b), reads as the
+// fp32 subnormal q 2^(b-149) (subnormals are kept; nothing here flushes them).
+// The two words of a 64-bit half of a lane's 16-byte shared-memory read are
+// processed as one fp32 pair (the same nibble slot of word j and word j+1), so
+// each AND is one 64-bit op on a register pair.  Subtracting the pair
+// (z 2^(b-149), z 2^(b-149)) is exact, and the activations are staged
+// pre-scaled by 2^(109-b), so one packed FMA adds (q - z) x 2^-40 exactly into
+// fp32; 2^40 is folded into Delta.  Slots 5..7 (bits 20..31) are first shifted
+// down by 12.  Per 16 codes: 2 shifts and 16 ANDs on the ALU pipe (which issues
+// at half rate on sm_100, so they bound the inner loop), 8 sub.f32x2 and
+// 8 fma.f32x2 on the FMA pipe.  Lane l owns 64 consecutive input channels
+// (8 words, half a group) of each unit row.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+namespace {
+
+constexpr int kWarps = 16;                    // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kR = 4;                         // rows per unit (= rows per row block)
+constexpr int kUW = 256;                      // words per unit row (2048 channels)
+constexpr int kUB = kR * kUW * 4;             // 4 KiB of codes per unit
+constexpr int kUG = kUW / 16;                 // 16 groups per unit row
+constexpr int kStage = kUB + 2 * kR * kUG * 2;  // + Delta and z tiles (4 x 16 fp16 each)
+constexpr int kSlice = 68;                    // floats per 64-channel lane slice (+4 pad)
+constexpr int kMaxSmem = 227 * 1024;
+constexpr float kTwo40 = 1099511627776.0f;   // 2^40
+
+struct M1Args {
+  const __half* x;
+  const uint32_t* qw;
+  const __half* scales;
+  const __half* zeros;
+  __half* y;
+  uint32_t* status;  // device status word (wait timeouts)
+  int N, K, Kw, Kg;
+  int units_k;     // units per row block
+  int row_blocks;  // ceil(N / kR)
+  int max_units;   // most units any CTA gets
+  int x_bytes;     // staged activations (multiple of 128)
+  int stages;      // ring depth of each warp
+};
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+
+// Slot p of layout v1 holds element i = (p < 4 ? 2p : 2(p-4)+1) of its word.
+// Bit offset of slot p after the optional shift by 12: 4p (p <= 4), 4p - 12.
+__device__ __forceinline__ int slot_bit(int p) { return p <= 4 ? 4 * p : 4 * p - 12; }
+
+// Staged activations: channels are grouped in 64-channel lane slices kSlice
+// floats apart (the 16-byte pad makes the quarter-warp phases of a 128-bit read
+// hit distinct banks); inside a slice, block b = words 2b and 2b+1, and float
+// 16b + 2p + (j & 1) holds the element of word j in slot p.
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
+
+// 2^(b-149) for b = 0..16 is subnormal: build it from its bit pattern.
+__device__ __forceinline__ float sub2pow(int b) { return __uint_as_float(1u << b); }
+
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Arrives on `bar` once this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Issues the copies of unit (rb, kc) into a stage: lane 0 the 4 x 256-word
+// code box (one TMA op; rows past N and words past K/8 arrive as zeros), every
+// lane 4 bytes of the Delta tile and 4 of the z tile with cp.async (the group
+// count per row is even, so these pairs are 4-byte aligned).
+__device__ __forceinline__ void issue_unit(const M1Args& a, const CUtensorMap* tmap, int rb, int kc, uint8_t* dst,
+                                           uint64_t* bar, int lane, uint64_t pol) {
+  const int n0 = rb * kR;
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kUB));
+    tma_load_2d(dst, tmap, kc * kUW, n0, bar, pol);
+  }
+  const int rows = min(kR, a.N - n0);
+  const int words = min(kUW, a.Kw - kc * kUW);
+  const int tr = lane >> 3, tc = lane & 7;  // tile row and group pair of this lane
+  if (tr < rows && 2 * tc < words / 16) {
+    const size_t o = static_cast<size_t>(n0 + tr) * a.Kg + kc * kUG + 2 * tc;
+    __half* tile = reinterpret_cast<__half*>(dst + kUB);
+    cp_async_4(tile + tr * kUG + 2 * tc, a.scales + o);
+    cp_async_4(tile + kR * kUG + tr * kUG + 2 * tc, a.zeros + o);
+  }
+  cp_async_arrive(bar);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.stages;
+  float* xs = reinterpret_cast<float*>(smem);
+  uint8_t* ring = smem + a.x_bytes + static_cast<size_t>(warp) * S * kStage;
+  float* part = reinterpret_cast<float*>(smem + a.x_bytes + static_cast<size_t>(kWarps) * S * kStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(part + a.max_units * kR) + warp * S;
+
+  // this CTA's row blocks [rb0, rb1); this warp's units are warp, warp + 8, ...
+  const int rb0 = static_cast<int>(static_cast<long long>(blockIdx.x) * a.row_blocks / gridDim.x);
+  const int rb1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * a.row_blocks / gridDim.x);
+  const int U = (rb1 - rb0) * a.units_k;
+  const int dkc = kWarps % a.units_k, drb = kWarps / a.units_k;
+
+  // the next kernel on the stream may start its own prologue right away
+  griddep_launch_dependents();
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 33);  // expect-tx arrival + 32 cp.async arrivals
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = l2_evict_first_policy();
+  // prologue: fill the ring (codes, Delta and z are read-only)
+  int rb_f = rb0 + warp / a.units_k, kc_f = warp % a.units_k;
+  int jf = warp;
+  for (int s = 0; s < S && jf < U; ++s, jf += kWarps) {
+    issue_unit(a, &tmap, rb_f, kc_f, ring + static_cast<size_t>(s) * kStage, &full[s], lane, pol);
+    rb_f += drb, kc_f += dkc;
+    if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
+  }
+
+  // x, y and anything earlier kernels produce are touched only after this
+  griddep_wait();
+
+  // x'' = x * 2^(109 - b(slot)), fp32, in pair order.  Word c (8 channels) is
+  // word c & 7 of lane slice c >> 3: block (c >> 1) & 3, pair half c & 1;
+  // element 2t sits in slot t, element 2t + 1 in slot 4 + t.
+  for (int c = threadIdx.x; c < a.K / 8; c += kThreads) {
+    const uint4 v = ld_nc_v4(a.x + 8 * c);
+    const uint32_t hv[4] = {v.x, v.y, v.z, v.w};
+    float* dst = xs + (c >> 3) * kSlice + 16 * ((c >> 1) & 3) + (c & 1);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float2 f = __half22float2(as_h2(hv[t]));
+      dst[2 * t] = f.x * pow2f(109 - slot_bit(t));
+      dst[8 + 2 * t] = f.y * pow2f(109 - slot_bit(4 + t));
+    }
+  }
+  __syncthreads();
+
+  // Lanes with bit 2 set read the second half of their slice first (weights
+  // and activations alike) so that the 32-byte lane stride does not put two
+  // lanes of a quarter-warp phase on the same banks.
+  const int swap1 = (lane >> 2) & 1;
+  bool failed = false;
+  int kc = warp % a.units_k;
+  for (int j = warp, i = 0; j < U; j += kWarps, ++i) {
+    const int s = i % S;
+    const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
+    const int ckc = kc;
+    kc += dkc;
+    if (kc >= a.units_k) kc -= a.units_k;
+
+    const bool act = lane * 8 < min(kUW, a.Kw - ckc * kUW);
+    uint64_t xp[32];
+    if (act) {
+      const ulonglong2* xb =
+          reinterpret_cast<const ulonglong2*>(xs + (ckc * (kUW / 8) + lane) * kSlice) + swap1 * 8;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const ulonglong2 v = xb[c];
+        xp[2 * c] = v.x;
+        xp[2 * c + 1] = v.y;
+      }
+      xb += 8 - 16 * swap1;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const ulonglong2 v = xb[c];
+        xp[16 + 2 * c] = v.x;
+        xp[16 + 2 * c + 1] = v.y;
+      }
+    }
+
+    if (!mbar_wait_bounded(&full[s], parity)) {
+      if (lane == 0) atomicOr(a.status, kDevWaitTimeout);
+      failed = true;
+      break;
+    }
+
+    float acc[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) acc[r] = 0.0f;
+    uint8_t* stage = ring + static_cast<size_t>(s) * kStage;
+    if (act) {
+      const ulonglong2* wq = reinterpret_cast<const ulonglong2*>(stage) + 2 * lane + swap1;
+      const __half* tile = reinterpret_cast<const __half*>(stage + kUB) + (lane >> 1);
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        const ulonglong2 wa = wq[r * (kUW / 4)];
+        const ulonglong2 wb = wq[r * (kUW / 4) + 1 - 2 * swap1];
+        const float zf = __half2float(tile[kR * kUG + r * kUG]);
+        const float df = __half2float(tile[r * kUG]) * kTwo40;
+        const uint64_t zz = f2_pack(zf, zf);
+        // (z 2^(b-149), z 2^(b-149)) for b = 0, 4, 8, 12, 16 (exact subnormals)
+        const uint64_t z0 = f2_mul(zz, f2_pack(sub2pow(0), sub2pow(0)));
+        const uint64_t z4 = f2_mul(zz, f2_pack(sub2pow(4), sub2pow(4)));
+        const uint64_t z8 = f2_mul(zz, f2_pack(sub2pow(8), sub2pow(8)));
+        const uint64_t z12 = f2_mul(zz, f2_pack(sub2pow(12), sub2pow(12)));
+        const uint64_t z16 = f2_mul(zz, f2_pack(sub2pow(16), sub2pow(16)));
+        uint64_t pa = 0, pb = 0;
+        const uint64_t blk[4] = {wa.x, wa.y, wb.x, wb.y};
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const uint64_t w = blk[b];
+          const uint64_t h = f2_pack(static_cast<uint32_t>(w) >> 12, static_cast<uint32_t>(w >> 32) >> 12);
+          const uint64_t* x8 = xp + 8 * b;
+          pa = f2_fma(f2_sub(w & 0x0000000F0000000Full, z0), x8[0], pa);
+          pb = f2_fma(f2_sub(w & 0x000000F0000000F0ull, z4), x8[1], pb);
+          pa = f2_fma(f2_sub(w & 0x00000F0000000F00ull, z8), x8[2], pa);
+          pb = f2_fma(f2_sub(w & 0x0000F0000000F000ull, z12), x8[3], pb);
+          pa = f2_fma(f2_sub(w & 0x000F0000000F0000ull, z16), x8[4], pa);
+          pb = f2_fma(f2_sub(h & 0x00000F0000000F00ull, z8), x8[5], pb);
+          pa = f2_fma(f2_sub(h & 0x0000F0000000F000ull, z12), x8[6], pa);
+          pb = f2_fma(f2_sub(h & 0x000F0000000F0000ull, z16), x8[7], pb);
+        }
+        const float2 fa = f2_unpack(pa), fb = f2_unpack(pb);
+        acc[r] = df * ((fa.x + fb.x) + (fa.y + fb.y));
+      }
+    }
+    // refill the stage with this warp's unit i + S (its reads above are done)
+    __syncwarp();
+    if (jf < U) {
+      issue_unit(a, &tmap, rb_f, kc_f, stage, &full[s], lane, pol);
+      jf += kWarps;
+      rb_f += drb, kc_f += dkc;
+      if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
+    }
+    // reduce the unit's 4 row partials over the lanes
+    const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
+    float k0 = b0 ? acc[2] : acc[0];
+    float k1 = b0 ? acc[3] : acc[1];
+    k0 += __shfl_xor_sync(0xffffffffu, b0 ? acc[0] : acc[2], 1);
+    k1 += __shfl_xor_sync(0xffffffffu, b0 ? acc[1] : acc[3], 1);
+    float t = b1 ? k1 : k0;
+    t += __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 8);
+    t += __shfl_xor_sync(0xffffffffu, t, 16);
+    if (lane < 4) part[j * kR + 2 * b0 + b1] = t;  // lane bits -> row 2*b0 + b1
+  }
+  if (failed) {
+    // let this warp's copies in flight land before the CTA can exit
+    for (int i2 = 0; i2 < S; ++i2) mbar_wait_bounded(&full[i2], 0u);
+  }
+  __syncthreads();
+  if (failed) return;
+
+  // y[n] = sum over the units of row block (n / 4), in unit order
+  const int rows = (rb1 - rb0) * kR;
+  for (int i = threadIdx.x; i < rows; i += kThreads) {
+    const int n = rb0 * kR + i;
+    if (n >= a.N) continue;
+    const int rbl = i / kR, r = i - rbl * kR;
+    float v = 0.0f;
+    for (int c = 0; c < a.units_k; ++c) v += part[(rbl * a.units_k + c) * kR + r];
+    a.y[n] = __float2half_rn(v);
+  }
+}
+
+int round128(int b) { return (b + 127) / 128 * 128; }
+
+int x_bytes_for(int K) { return round128((K / 64) * kSlice * 4); }
+
+int smem_for(int stages, int x_bytes, int max_units) {
+  return x_bytes + kWarps * stages * kStage + round128(max_units * kR * 4) + kWarps * stages * 8;
+}
+
+}  // namespace
+
+bool gemv_m1_supports(int N, int K) {
+  if ((K / kGroup) % 2) return false;  // Delta/z pairs are copied 4 bytes at a time
+  const int sms = device_sm_count();
+  const int row_blocks = (N + kR - 1) / kR;
+  const int grid = min(sms, row_blocks);
+  const int max_units = ((row_blocks + grid - 1) / grid) * ((K / 8 + kUW - 1) / kUW);
+  return smem_for(2, x_bytes_for(K), max_units) <= kMaxSmem;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda); looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t st) {
+  M1Args a;
+  a.status = status;
+  a.x = p.x;
+  a.qw = p.qweight;
+  a.scales = p.scales;
+  a.zeros = p.zeros;
+  a.y = p.y;
+  a.N = p.N;
+  a.K = p.K;
+  a.Kw = p.K / 8;
+  a.Kg = p.K / kGroup;
+  a.units_k = (a.Kw + kUW - 1) / kUW;
+  a.row_blocks = (p.N + kR - 1) / kR;
+  const int grid = min(device_sm_count(), a.row_blocks);
+  a.max_units = ((a.row_blocks + grid - 1) / grid) * a.units_k;
+  a.x_bytes = x_bytes_for(p.K);
+  // deepest per-warp ring that fits
+  int stages = 6;
+  while (stages > 2 && smem_for(stages, a.x_bytes, a.max_units) > kMaxSmem) --stages;
+  if (smem_for(stages, a.x_bytes, a.max_units) > kMaxSmem) return cudaErrorNotSupported;
+  a.stages = stages;
+  const int smem = smem_for(stages, a.x_bytes, a.max_units);
+
+  // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256
+  CUtensorMap tmap;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.Kw), static_cast<cuuint64_t>(p.N)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.Kw) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kUW), static_cast<cuuint32_t>(kR)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  cudaError_t e = cudaFuncSetAttribute(gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, gemv_m1_kernel, a, tmap);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace w4a16

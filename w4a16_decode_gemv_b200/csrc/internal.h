@@ -16,6 +16,10 @@ constexpr int kMaxM = 64;          // largest M of w4a16_gemm
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();
 
+// Whether the GEMV kernels are launched with programmatic dependent launch
+// (on unless the environment variable W4A16_NO_PDL is set to a non-empty value).
+bool pdl_enabled();
+
 cudaError_t launch_act_scale(const __half* X, int T, int K, double alpha, __half* s, cudaStream_t st);
 
 cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K, int bits, int mode,
@@ -40,7 +44,11 @@ struct GemmProblem {
   int M, N, K;
 };
 
-// Can the CUDA-core GEMV run this problem (M and shared-memory budget)?
+// The M = 1 decode GEMV (gemv_m1.cu): whole rows per CTA, no workspace.
+bool gemv_m1_supports(int N, int K);
+cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t st);
+
+// The split-K CUDA-core GEMV for small M (gemv.cu).
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
