@@ -157,6 +157,33 @@ W4A16_API w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const 
  */
 W4A16_API w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream);
 
+/*
+ * w4a16_gemv_noalloc -- the split-K CUDA-core GEMV of w4a16_gemm (1 <= M <= 4)
+ * for callers that cannot allocate device memory: inference servers that
+ * reserve every buffer at start-up, plug-ins handed only the tensors they work
+ * on, and hosts linking this library without a device allocator.  The pages
+ * have no counterpart; it exists for those callers only.
+ *
+ * Instead of a caller workspace it uses a scratch array of
+ * w4a16_gemv_noalloc_max_scratch() bytes (512 KiB) that is part of this
+ * library's device data: every GPU that loads the library holds it until the
+ * process exits.  The scratch needed is that of w4a16_gemm_workspace_size;
+ * larger M * N is rejected with W4A16_ERR_SHAPE and a message.  The call
+ * allocates nothing.  Its first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current) and caches it;
+ * make that first call before any stream capture.  Each call clears the part
+ * of the array it uses with an asynchronous memset on `stream`.  All calls
+ * share the one array, so calls whose work may overlap on the GPU (streams
+ * without ordering between them) race and must not be made.
+ * Arguments, layouts and accuracy are those of w4a16_gemm.
+ */
+W4A16_API w4a16_status w4a16_gemv_noalloc(const void* x, const uint32_t* qweight, const void* scales,
+                                          const void* zeros, int M, int N, int K, int group, void* y,
+                                          w4a16_stream_t stream);
+
+/* Size in bytes of the fixed scratch array used by w4a16_gemv_noalloc. */
+W4A16_API size_t w4a16_gemv_noalloc_max_scratch(void);
+
 /* Message for the last error on this thread ("" if none). */
 W4A16_API const char* w4a16_last_error(void);
 

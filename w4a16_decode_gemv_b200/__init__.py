@@ -49,6 +49,10 @@ def load_library():
     lib.w4a16_gemm_workspace_size.restype = sz
     lib.w4a16_gemm.argtypes = [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]
     lib.w4a16_gemm.restype = i
+    lib.w4a16_gemv_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, vp, vp]
+    lib.w4a16_gemv_noalloc.restype = i
+    lib.w4a16_gemv_noalloc_max_scratch.argtypes = []
+    lib.w4a16_gemv_noalloc_max_scratch.restype = sz
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
     lib.w4a16_last_error.argtypes = []
@@ -171,6 +175,28 @@ def w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zer
     with torch.cuda.device(x.device):
         _check(lib.w4a16_gemm(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
                               _ptr(ws), ws.numel() * ws.element_size(), _stream(x.device)), "w4a16_gemm")
+    return y
+
+
+def w4a16_gemv_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                       group: int = GROUP, out: torch.Tensor | None = None) -> torch.Tensor:
+    """The split-K GEMV (M <= 4) with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory; ``out`` may be given so
+    that this call allocates nothing either.
+    """
+    lib = load_library()
+    M, K = x.shape
+    N = qweight.shape[0]
+    _expect(x, torch.float16, (M, K), "x")
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(scales, torch.float16, (N, K // group), "scales")
+    _expect(zeros, torch.float16, (N, K // group), "zeros")
+    y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
+    _expect(y, torch.float16, (M, N), "out")
+    with torch.cuda.device(x.device):
+        _check(lib.w4a16_gemv_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
+                                      _stream(x.device)), "w4a16_gemv_noalloc")
     return y
 
 

@@ -41,6 +41,8 @@ constexpr long long kMaxElems = 1ll << 31;  // index arithmetic stays in 64 bits
 
 }  // namespace
 
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 int device_sm_count() {
   static int cached[128] = {0};
   int dev = 0;

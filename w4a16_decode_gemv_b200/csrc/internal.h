@@ -13,6 +13,9 @@ constexpr int kGroup = 128;        // group size along K (the only one supported
 constexpr int kMaxGemvM = 4;       // largest M the CUDA-core GEMV handles
 constexpr int kMaxM = 64;          // largest M of w4a16_gemm
 
+// Replaces the calling thread's message returned by w4a16_last_error().
+void set_last_error(const char* msg);
+
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();
 
