@@ -279,8 +279,8 @@ def run_ours(args, dist):
     if dist.rank == 0:
         peak, peak_src = measured_peaks()
         achieved = WEIGHT_BYTES / (us_layer * 1e-6) / 1e9
-        traffic = profiled_traffic("gemv_w4a16_kernel M=1 8192x8192")
-        roof = {"bound": "hbm", "kernel": "gemv_w4a16_kernel<1,4> (split-K CUDA-core GEMV)",
+        traffic = profiled_traffic("gemv_m1_kernel M=1 8192x8192")
+        roof = {"bound": "hbm", "kernel": "gemv_m1_kernel (M=1 CUDA-core GEMV, CTA-owned rows)",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "algorithmic_bytes_per_launch": WEIGHT_BYTES,
