@@ -45,6 +45,7 @@ LAYERS = 16
 M1, N1, K1 = 1, 8192, 8192
 WEIGHT_BYTES = N1 * K1 // 2 + 2 * N1 * (K1 // 128) * 2       # codes + scales + zeros = 35,651,584
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_TFLOPS = 1590.0
 
 
 def layer_bytes(N, K):
@@ -172,6 +173,16 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
     return FALLBACK_HBM_GBS, "fallback 6650 GB/s (earlier measurement on this pool)"
+
+
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s for a kernel timed alone (burst), and where it came from."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst; fp16 runs at the bf16 rate)"
+    return FALLBACK_TFLOPS, "fallback 1590 TFLOP/s (earlier measurement on this pool)"
 
 
 def profiled_traffic(kernel_key):
@@ -391,6 +402,9 @@ def other_workloads(args, dev):
     import w4a16_decode_gemv_b200 as w4
     from w4a16_decode_gemv_b200 import inputs
     res = {}
+    hbm_peak, _ = measured_peaks()
+    tc_peak, tc_src = measured_tensor_peak()
+    res["peaks"] = {"hbm_gbs": hbm_peak, "tensor_tflops": tc_peak, "tensor_source": tc_src}
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
 
@@ -431,8 +445,12 @@ def other_workloads(args, dev):
             try:
                 us = gemm_us(M, N, K)
                 b = layer_bytes(N, K)
-                entries.append({"M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(b / us / 1e3, 1),
-                                "tflops": round(2 * M * N * K / us / 1e6, 2)})
+                e = {"M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(b / us / 1e3, 1),
+                     "hbm_frac": round(b / us / 1e3 / hbm_peak, 4), "tflops": round(2 * M * N * K / us / 1e6, 2)}
+                if M > 4:
+                    e["path"] = "tcgen05 tensor cores"
+                    e["tensor_frac"] = round(2 * M * N * K / us / 1e6 / tc_peak, 4)
+                entries.append(e)
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries

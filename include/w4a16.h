@@ -118,8 +118,9 @@ W4A16_API w4a16_status awq_quantize_pack(const void* W, const void* s, int N, in
 
 /*
  * w4a16_gemm_workspace_size -- bytes of workspace that w4a16_gemm needs.
- * Returns 0 for invalid sizes.  The workspace holds fp32 split-K partial sums,
- * per-row-block arrival counters and a device status word.
+ * Returns 0 for invalid sizes.  The workspace holds fp32 split-K partial sums
+ * (M x N for M <= 4, N x round_up(M, 16) for M >= 5), per-row-block arrival
+ * counters and a device status word.
  */
 W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
 
@@ -128,8 +129,11 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  *
  *   y[m][n] = fp16( sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k] )
  *
- * with fp32 accumulation.  M < 16 runs the split-K CUDA-core GEMV; M >= 16 the
- * tensor-core kernel.  x is the activation already divided by the AWQ scale s.
+ * with fp32 accumulation.  M = 1..4 runs on the CUDA cores (M = 1: whole rows
+ * per SM, no partial sums; M = 2..4: split-K); M = 5..64 runs on the tensor
+ * cores (tcgen05), with w_hat = Delta * (u - z) rounded once to fp16 before the
+ * MMA (so |w_hat| must stay below 65504).  x is the activation already divided
+ * by the AWQ scale s.
  * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
  * y_ref the exact product with the dequantized weight.  The order of the
  * split-K additions may vary between calls, so y may differ in the last bit.

@@ -1,0 +1,116 @@
+"""Parity of the tensor-core skinny GEMM (M = 5..64) with the CPU oracle.
+
+Every case goes through the C ABI (``w4a16_gemm``).  The output must satisfy,
+per element, |y - y_ref| <= 2e-3 * B + 1e-3 with B = sum_k |x * w_hat| and
+y_ref the fp64 product with the oracle's dequantized weight.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w4a16_decode_gemv_b200 as w4
+from w4a16_decode_gemv_b200 import build, inputs
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 2e-3, 1e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    w4.load_library()
+    return torch.device("cuda:0")
+
+
+def to_dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def check(y, x, qw, sc, zr, rows=None):
+    if rows is None:
+        y_ref, B = oracle.gemm(x, qw, sc, zr)
+        y = y.astype(np.float64)
+    else:
+        y_ref, B = oracle.gemm_rows(x, qw, sc, zr, rows)
+        y = y[:, rows].astype(np.float64)
+    assert np.all(np.isfinite(y)), "non-finite output"
+    err = np.abs(y - y_ref)
+    lim = RTOL * B + ATOL
+    worst = np.unravel_index(np.argmax(err - lim), err.shape)
+    assert np.all(err <= lim), f"max excess at {worst}: |{y[worst]} - {y_ref[worst]}| > {lim[worst]}"
+
+
+def case(dev, M, N, K, seed, bits=4, mode=oracle.ASYM, workspace=None):
+    W, x = inputs.random_case(seed, N, K, M)
+    qo, so, zo = oracle.quantize_pack(W, None, 128, bits, mode)
+    args = (to_dev(x, dev), to_dev(qo.view(np.int32), dev), to_dev(so, dev), to_dev(zo, dev))
+    y = w4.w4a16_gemm(*args, workspace=workspace)
+    torch.cuda.synchronize()
+    check(y.cpu().numpy(), x, qo, so, zo)
+    return args, (x, qo, so, zo)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (5, 1, 128),          # one row, one group, MP = 16
+    (8, 300, 1024),       # ragged row block (300 = 256 + 44)
+    (16, 256, 128),       # one unit per row block
+    (16, 1000, 2048),
+    (17, 513, 1152),      # MP = 32, odd groups per row
+    (32, 64, 8192),       # many CTAs share one row block
+    (48, 129, 4096),      # MP = 48
+    (64, 256, 11008),     # 86 groups per row
+    (64, 2048, 256),
+    (64, 300, 22016),     # 172 groups per row
+])
+def test_tc_small_shapes(dev, M, N, K):
+    case(dev, M, N, K, seed=M * 7919 + N)
+
+
+def test_tc_whole_row_blocks_written_directly(dev):
+    """K = 128: every CTA covers whole row blocks and writes y without the workspace."""
+    case(dev, 33, 40960, 128, seed=11)
+
+
+def test_tc_3bit_symmetric_codes(dev):
+    case(dev, 16, 200, 2048, seed=5, bits=3, mode=oracle.SYM)
+
+
+@pytest.mark.parametrize("M", [16, 32, 64])
+def test_tc_skinny_workload_sampled_rows(dev, M):
+    """K = N = 8192 quantized on the GPU, the launch the bench times; 256 sampled rows checked."""
+    (layer,) = inputs.layer_set(inputs.SKINNY)
+    x = layer.x[:M]
+    qg, sg, zg = w4.awq_quantize_pack(to_dev(layer.W, dev))
+    y = w4.w4a16_gemm(to_dev(x, dev), qg, sg, zg)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.random.default_rng(M).choice(layer.N, 252, replace=False),
+                                     [0, 255, 256, layer.N - 1]]))
+    qw = qg.cpu().numpy().view(np.uint32)[rows]
+    y_ref, B = oracle.gemm_ref(x, oracle.dequant(qw, sg.cpu().numpy()[rows], zg.cpu().numpy()[rows]))
+    err = np.abs(y.cpu().numpy()[:, rows].astype(np.float64) - y_ref)
+    assert np.all(err <= RTOL * B + ATOL)
+    qo, _, _ = oracle.quantize_pack(layer.W[rows], None, 128, 4, oracle.ASYM)
+    assert np.array_equal(qw, qo)
+
+
+def test_tc_workspace_left_zeroed_across_paths(dev):
+    """One workspace serves M = 1, 32, 4 and 64 in turn; each result is right and it ends zeroed."""
+    N, K = 700, 4096
+    ws = torch.zeros(w4.gemm_workspace_size(64, N, K), dtype=torch.uint8, device=dev)
+    for i, M in enumerate((1, 32, 4, 64, 32)):
+        case(dev, M, N, K, seed=100 + i, workspace=ws)
+    w4.gemm_check(ws)
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_tc_repeated_calls_identical(dev):
+    """Calls repeat on the same inputs; partial sums may add in another order, so each is checked."""
+    args, ref = case(dev, 64, 512, 8192, seed=7)
+    y1 = w4.w4a16_gemm(*args).cpu().numpy()
+    y2 = w4.w4a16_gemm(*args).cpu().numpy()
+    check(y1, *ref)
+    check(y2, *ref)

@@ -63,23 +63,27 @@ bool pdl_enabled() {
   return on;
 }
 
+// fp32 partial sums per output: M for the CUDA-core GEMV, M rounded up to 16 for the tensor-core path.
+static size_t acc_columns(int M) { return M <= kMaxGemvM ? static_cast<size_t>(M) : (static_cast<size_t>(M) + 15) / 16 * 16; }
+
+static size_t counter_bytes(int N) {
+  const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
+  return (row_blocks * 4 + 15) / 16 * 16;
+}
+
 size_t workspace_bytes(int M, int N, int K) {
   (void)K;
-  const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
-  const size_t cnt = (row_blocks * 4 + 15) / 16 * 16;
-  return 16 + cnt + static_cast<size_t>(M) * N * 4;
+  return 16 + counter_bytes(N) + acc_columns(M) * N * 4;
 }
 
 Workspace carve_workspace(void* base, int M, int N, int K) {
   (void)M;
   (void)K;
   uint8_t* p = static_cast<uint8_t*>(base);
-  const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
-  const size_t cnt = (row_blocks * 4 + 15) / 16 * 16;
   Workspace w;
   w.status = reinterpret_cast<uint32_t*>(p);
   w.counters = reinterpret_cast<uint32_t*>(p + 16);
-  w.acc = reinterpret_cast<float*>(p + 16 + cnt);
+  w.acc = reinterpret_cast<float*>(p + 16 + counter_bytes(N));
   return w;
 }
 
@@ -149,7 +153,7 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   cudaError_t e;
   if (M == 1 && gemv_m1_supports(N, K)) {
     e = launch_gemv_m1(p, ws.status, st);
-  } else if (M < 16 && gemv_supports(M, K)) {
+  } else if (M <= kMaxGemvM && gemv_supports(M, K)) {
     e = launch_gemv(p, ws, st);
   } else {
     e = launch_gemm_tc(p, ws, st);

@@ -3,6 +3,7 @@
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstddef>
 #include <cstdint>
@@ -29,7 +30,9 @@ cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K,
                                  uint32_t* qweight, __half* scales, __half* zeros, cudaStream_t st);
 
 // Workspace of the split-K kernels: [status word | padding to 16 B]
-// [row-block counters, padded to 16 B] [fp32 partial sums M x N].
+// [row-block counters, padded to 16 B] [fp32 partial sums]: M x N for the
+// CUDA-core GEMV (M <= 4), N x MP (MP = M rounded up to 16) for the
+// tensor-core path.
 struct Workspace {
   uint32_t* status;
   uint32_t* counters;
@@ -54,6 +57,11 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
 // The split-K CUDA-core GEMV for small M (gemv.cu).
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+
+// The tensor-core skinny GEMM (gemm_tc.cu), M = 5..64.
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 }  // namespace w4a16
