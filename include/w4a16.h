@@ -118,9 +118,11 @@ W4A16_API w4a16_status awq_quantize_pack(const void* W, const void* s, int N, in
 
 /*
  * w4a16_gemm_workspace_size -- bytes of workspace that w4a16_gemm needs.
- * Returns 0 for invalid sizes.  The workspace holds fp32 split-K partial sums
- * (M x N for M <= 4, N x round_up(M, 16) for M >= 5), per-row-block arrival
- * counters and a device status word.
+ * Returns 0 for invalid sizes.  The workspace holds a device status word,
+ * per-row-block arrival counters and fp32 split-K partial sums (M x N for
+ * M <= 4); for M >= 5 it adds, after room for the M = 4 partial sums, two
+ * 256 x round_up(M, 16) fp32 slots per streaming multiprocessor of the current
+ * device for the tensor-core path's partial sums.
  */
 W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
 
@@ -143,8 +145,10 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  *   1 <= M <= 64;  N >= 1;  K a multiple of group;  group == 128.
  *   workspace  device memory of at least w4a16_gemm_workspace_size(M, N, K, group)
  *              bytes, 16-byte aligned, ZERO-FILLED before its first use.  Every
- *              call that completes leaves it zero-filled again, so it can be reused
- *              by later calls on the same stream.  Calls that may run concurrently
+ *              call that completes leaves the part that must start at zero (the
+ *              first w4a16_gemm_workspace_size(min(M, 4), N, K, group) bytes)
+ *              zero-filled again, so it can be reused by later calls on the same
+ *              stream; the rest is scratch.  Calls that may run concurrently
  *              need distinct workspaces.  After W4A16_ERR_DEVICE it must be zero-filled
  *              again by the caller.
  */

@@ -63,27 +63,32 @@ bool pdl_enabled() {
   return on;
 }
 
-// fp32 partial sums per output: M for the CUDA-core GEMV, M rounded up to 16 for the tensor-core path.
-static size_t acc_columns(int M) { return M <= kMaxGemvM ? static_cast<size_t>(M) : (static_cast<size_t>(M) + 15) / 16 * 16; }
-
 static size_t counter_bytes(int N) {
   const size_t row_blocks = (static_cast<size_t>(N) + 3) / 4;
   return (row_blocks * 4 + 15) / 16 * 16;
 }
 
+// Room for the CUDA-core GEMV partial sums (M x N fp32, at most kMaxGemvM rows).
+static size_t gemv_acc_bytes(int M, int N) {
+  const size_t m = static_cast<size_t>(M < kMaxGemvM ? M : kMaxGemvM);
+  return (m * N * 4 + 15) / 16 * 16;
+}
+
 size_t workspace_bytes(int M, int N, int K) {
   (void)K;
-  return 16 + counter_bytes(N) + acc_columns(M) * N * 4;
+  if (M <= kMaxGemvM) return 16 + counter_bytes(N) + static_cast<size_t>(M) * N * 4;
+  return 16 + counter_bytes(N) + gemv_acc_bytes(kMaxGemvM, N) + tc_partial_bytes(M);
 }
 
 Workspace carve_workspace(void* base, int M, int N, int K) {
-  (void)M;
   (void)K;
   uint8_t* p = static_cast<uint8_t*>(base);
   Workspace w;
   w.status = reinterpret_cast<uint32_t*>(p);
   w.counters = reinterpret_cast<uint32_t*>(p + 16);
   w.acc = reinterpret_cast<float*>(p + 16 + counter_bytes(N));
+  w.part = M <= kMaxGemvM ? nullptr
+                          : reinterpret_cast<float*>(p + 16 + counter_bytes(N) + gemv_acc_bytes(kMaxGemvM, N));
   return w;
 }
 

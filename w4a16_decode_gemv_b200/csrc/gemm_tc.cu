@@ -11,16 +11,24 @@
 //
 // Swap-AB.  The weight rows are the MMA's M dimension (128 rows per MMA) and the
 // tokens its N dimension (MP = M rounded up to 16): D[n][m] = sum_k A[n][k] B[m][k]
-// with A = w_hat (fp16, K-major) and B = x (fp16, K-major), fp32 accumulators in
-// tensor memory (TMEM lane = weight row, column = token).
+// with A = w_hat (fp16) and B = x (fp16, K-major in shared memory), fp32
+// accumulators in tensor memory (TMEM lane = weight row, column = token).
+//
+// w_hat lives in tensor memory, not shared memory: the dequantizing thread of a
+// weight row writes its fp16 pairs straight into that row's TMEM lane
+// (tcgen05.st) and the MMA reads A from there.  Shared memory then only carries
+// the codes and x, so its bandwidth (which a shared-memory A tile of fp16 would
+// exhaust: 4x the bytes of the codes, written once and read once) is not the
+// bound, and four w_hat buffers fit beside the accumulators in the 512 columns.
 //
 // Work split.  Units are (row block of 256 rows, group of 128 inputs), ordered
 // row-block-major and dealt to a persistent grid (one CTA per SM) in contiguous,
 // equal ranges.  A CTA accumulates its units of one row block in two 128 x MP
 // TMEM accumulators (double-buffered, so the next row block's MMAs overlap the
 // epilogue of the last).  A CTA that covers a whole row block writes y directly;
-// otherwise its fp32 partials are added into the workspace and the last
-// contributor of the row block converts them to fp16 and zeroes the workspace.
+// otherwise its fp32 partials are added into the workspace (vector reductions in
+// L2) and the last contributor of the row block converts them to fp16 and
+// zeroes the workspace.
 //
 // Roles (16 warps):
 //   warp 0     one thread issues the tensor copies (TMA) of each unit into a ring
@@ -30,9 +38,9 @@
 //   warp 1     allocates TMEM; one thread issues tcgen05.mma (8 per 64-input half)
 //              and tcgen05.commit;
 //   warps 4-7  epilogue: tcgen05.ld of the accumulators, y or workspace;
-//   warps 8-15 dequantization: thread r owns weight row r of the block and turns
-//              its codes into w_hat in a 128-byte-swizzled K-major tile, the
-//              layout the MMA's shared-memory descriptor reads.
+//   warps 8-15 dequantization: thread r owns weight row r of the block (warp
+//              8 + 4t + q holds tile t, TMEM lane quarter q) and writes its w_hat
+//              for 64 inputs at a time into one of the TMEM w_hat buffers.
 // Dequantization of a code pair: (w >> 4t) & 0x000F000F | 0x64006400 (one LOP3)
 // reads as the fp16 pair 1024 + q; subtracting 1024 + z is exact and the
 // multiply by Delta rounds once (Lecture 13 guide, §TinyChat, slides 36-37;
@@ -47,22 +55,25 @@
 namespace w4a16 {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kDqWarps = 16;                    // dequantization + epilogue warps
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 32 * 18;
 constexpr int kRows = 256;                      // weight rows per row block (two MMA tiles)
 constexpr int kCodeBytes = kRows * 16 * 4;      // 16 KiB: one group of codes for the block
-constexpr int kWBytes = kRows * 64 * 2;         // 32 KiB: w_hat for 64 inputs of the block
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kMaxStages = 8;
-constexpr int kCtrlBytes = 256;
+constexpr int kMaxStages = 12;
+constexpr int kCtrlBytes = 512;
 
 struct TcArgs {
+  const uint32_t* qweight;
   const __half* scales;
   const __half* zeros;
   __half* y;
-  float* ws_acc;        // [N][MP]
-  uint32_t* ws_cnt;     // [row blocks]
+  float4* ws_part;      // [2 x grid slots][MP / 4][256 rows] partial sums
   uint32_t* ws_status;
-  int M, N, Kg;
+  int M, N, Kw, Kg;
+  int dz_w;             // groups per Delta / z load: the largest of 8, 4, 2, 1 dividing Kg
   int total_units;
   int stages;
 };
@@ -81,15 +92,35 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, fp16 inputs, fp32 accumulation.
-__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (128 rows x 16 inputs, fp16 pairs in 8
+// columns) is read from tensor memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           bool accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
       : "memory");
 }
+
+// The w_hat of one code word: 4 fp16 pairs, inputs 8j .. 8j + 7 in order.
+struct Word4 {
+  uint32_t v[4];
+};
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const Word4& a, const Word4& b, const Word4& c,
+                                          const Word4& d) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(a.v[0]), "r"(a.v[1]), "r"(a.v[2]), "r"(a.v[3]), "r"(b.v[0]), "r"(b.v[1]), "r"(b.v[2]), "r"(b.v[3]),
+      "r"(c.v[0]), "r"(c.v[1]), "r"(c.v[2]), "r"(c.v[3]), "r"(d.v[0]), "r"(d.v[1]), "r"(d.v[2]), "r"(d.v[3])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Arrives once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -97,18 +128,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns: thread i gets lane (base + i), columns c..c+15.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
-      "[%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+// 32 lanes x 8 consecutive 32-bit columns: thread i gets lane (base + i), columns c..c+7.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+  for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -164,16 +192,44 @@ __device__ __forceinline__ bool epi_bar_or(bool pred) {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Adds four fp32 values into global memory without returning the old ones, so
+// the thread does not wait for the L2 round trip (a later fence orders them).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 __device__ __forceinline__ uint32_t lop3_nib(uint32_t w) {
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
   return r;
 }
 
+// A 16-bit load zero-extended into a 32-bit register, so that nothing reads the
+// destination (and waits for it) until the value is used.
 __device__ __forceinline__ uint32_t ld_nc_u16(const __half* p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  uint32_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
+}
+
+// W consecutive fp16 values (W = 1, 2, 4 or 8, the address aligned to 2W bytes)
+// into the low halves of w[0..3], lowest address first.
+__device__ __forceinline__ void ld_nc_halves(const __half* p, int W, uint32_t (&w)[4]) {
+  w[0] = w[1] = w[2] = w[3] = 0;
+  if (W == 8)
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "l"(p));
+  else if (W == 4)
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "l"(p));
+  else if (W == 2)
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
+  else
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(w[0]) : "l"(p));
+}
+
+// The idx-th fp16 value (0..7) of four packed words, zero-extended.
+__device__ __forceinline__ uint32_t pick_half(const uint32_t (&w)[4], int idx) {
+  const uint32_t v = (idx & 4) ? ((idx & 2) ? w[3] : w[2]) : ((idx & 2) ? w[1] : w[0]);
+  return (idx & 1) ? (v >> 16) : (v & 0xFFFFu);
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -182,12 +238,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
 __device__ __forceinline__ uint32_t dq_pair(uint32_t v, __half2 zz, __half2 dd) {
   return as_u32(__hmul2(__hsub2(as_h2(lop3_nib(v)), zz), dd));
+}
+
+__device__ __forceinline__ Word4 dq_word(uint32_t w, __half2 zz, __half2 dd) {
+  return Word4{{dq_pair(w, zz, dd), dq_pair(w >> 4, zz, dd), dq_pair(w >> 8, zz, dd), dq_pair(w >> 12, zz, dd)}};
 }
 
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
@@ -196,30 +252,45 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return p;
 }
 
+// Tensor-memory columns: [0, 4 MP) hold the accumulators (2 buffers x 2 tiles x
+// MP columns); from 4 MP on, as many w_hat buffers of 64 columns as fit (2 tiles
+// x 32 columns, one column = the fp16 pair of inputs 2c, 2c + 1 of one row):
+// 7 for MP = 16 down to 4 for MP = 64.
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxABufs = 7;
+__host__ __device__ constexpr int a_bufs(int mp) { return (512 - 4 * mp) / 64; }
+
+// Unit u of the range partition: the CTA whose range holds it.
+__host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
+  const int big = rem * (base + 1);
+  return u < big ? u / (base + 1) : rem + (u - big) / base;
+}
+
 template <int MP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(96)
     gemm_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tx) {
   constexpr int kXHalf = MP * 128;                // one 64-input half of the x tile
   constexpr int kStageBytes = kCodeBytes + 2 * kXHalf;
-  constexpr uint32_t kCols = 4 * MP <= 32 ? 32 : (4 * MP <= 64 ? 64 : (4 * MP <= 128 ? 128 : 256));
   constexpr uint32_t kIdesc = idesc_f16(MP);
+  constexpr uint32_t kACol0 = 4 * MP;
+  constexpr int kABufs = a_bufs(MP);
+  static_assert(kACol0 + kABufs * 64 <= kTmemCols, "accumulators and w_hat buffers exceed tensor memory");
+  static_assert(kABufs >= 4, "a unit writes two w_hat buffers; four keep the MMAs one unit behind");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
-  uint8_t* wbuf = smem;                          // 2 x kWBytes
-  uint8_t* stages = smem + 2 * kWBytes;          // S x kStageBytes
+  uint8_t* stages = smem;                        // S x kStageBytes: code tile, then x tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(stages + S * kStageBytes);
-  uint64_t* full = bars;                         // [S] codes + x landed
-  uint64_t* rempty = bars + kMaxStages;          // [S] codes read, x consumed
-  uint64_t* wfull = bars + 2 * kMaxStages;       // [2] w_hat half written
-  uint64_t* wempty = wfull + 2;                  // [2] w_hat half consumed by the MMAs
-  uint64_t* afull = wfull + 4;                   // [2] accumulator complete
-  uint64_t* aempty = wfull + 6;                  // [2] accumulator read out
-  uint64_t* tdown = wfull + 8;                   // teardown: all MMAs complete
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(wfull + 9);
+  uint64_t* full = bars;                         // [S] codes and x landed
+  uint64_t* rempty = bars + kMaxStages;          // [S] codes read and x consumed
+  uint64_t* wfull = bars + 2 * kMaxStages;       // [kABufs] w_hat half written to tensor memory
+  uint64_t* wempty = wfull + kMaxABufs;          // [kABufs] w_hat half consumed by the MMAs
+  uint64_t* afull = wempty + kMaxABufs;          // [2] accumulator complete
+  uint64_t* aempty = afull + 2;                  // [2] accumulator read out
+  uint64_t* tdown = aempty + 2;                  // teardown: all MMAs complete
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tdown + 1);
   volatile uint32_t* abort_flag = tslot + 1;
-  volatile uint32_t* last_flag = tslot + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int base = a.total_units / static_cast<int>(gridDim.x);
@@ -227,59 +298,76 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bx = static_cast<int>(blockIdx.x);
   const int u0 = bx * base + min(bx, rem);
   const int cnt = base + (bx < rem ? 1 : 0);
+  const int rb0 = u0 / a.Kg;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&rempty[s], 9);  // 8 dequantization warps + 1 MMA commit
+      mbar_init(&rempty[s], kDqWarps + 1);  // dequantization warps + 1 MMA commit
+    }
+    for (int b = 0; b < kABufs; ++b) {
+      mbar_init(&wfull[b], kDqWarps);
+      mbar_init(&wempty[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&wfull[b], 8);
-      mbar_init(&wempty[b], 1);
       mbar_init(&afull[b], 1);
-      mbar_init(&aempty[b], 4);
+      mbar_init(&aempty[b], kDqWarps);
     }
     mbar_init(tdown, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tslot, kCols);
+  if (warp == kMmaWarp) tmem_alloc(tslot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
+  // the next kernel on the stream (the partial-sum finalize) may begin launching
+  griddep_launch_dependents();
 
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
     // ---------------- producer: tensor copies of codes and x ----------------
     if (lane == 0) {
       const uint64_t pol_q = l2_evict_first_policy();
       const uint64_t pol_x = l2_evict_last_policy();
-      int issued = 0;
-      for (int i = 0; i < cnt; ++i) {
-        const int s = i % S;
-        if (i >= S && !wait_or_abort(&rempty[s], static_cast<uint32_t>(i / S - 1) & 1u, abort_flag, a.ws_status))
-          break;
+      auto code_copy = [&](int i) {
         const int u = u0 + i, rb = u / a.Kg, g = u - rb * a.Kg;
-        uint8_t* st = stages + s * kStageBytes;
+        const int s = i % S;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(st, &tq, g * 16, rb * kRows, &full[s], pol_q);
-        tma_load_2d(st + kCodeBytes, &tx, g * 128, 0, &full[s], pol_x);
-        tma_load_2d(st + kCodeBytes + kXHalf, &tx, g * 128 + 64, 0, &full[s], pol_x);
+        tma_load_2d(stages + s * kStageBytes, &tq, g * 16, rb * kRows, &full[s], pol_q);
+      };
+      auto x_copy = [&](int i) {
+        const int g = (u0 + i) % a.Kg;
+        const int s = i % S;
+        uint8_t* xs = stages + s * kStageBytes + kCodeBytes;
+        tma_load_2d(xs, &tx, g * 128, 0, &full[s], pol_x);
+        tma_load_2d(xs + kXHalf, &tx, g * 128 + 64, 0, &full[s], pol_x);
+      };
+      // the weights do not depend on the previous kernel: start streaming them first
+      const int pre = min(S, cnt);
+      for (int i = 0; i < pre; ++i) code_copy(i);
+      griddep_wait();  // x may be the previous kernel's output
+      for (int i = 0; i < pre; ++i) x_copy(i);
+      int issued = pre;
+      for (int i = pre; i < cnt; ++i) {
+        const int s = i % S;
+        if (!wait_or_abort(&rempty[s], static_cast<uint32_t>(i / S - 1) & 1u, abort_flag, a.ws_status)) break;
+        code_copy(i);
+        x_copy(i);
         issued = i + 1;
       }
       // copies still in flight must land before the CTA may exit
       for (int j = max(0, issued - S); j < issued; ++j)
         mbar_wait_bounded(&full[j % S], static_cast<uint32_t>(j / S) & 1u);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       bool any = false;
       int hb = 0, f = 0;
       for (int i = 0; i < cnt; ++i) {
         const int s = i % S;
-        const int u = u0 + i, rb = u / a.Kg, g = u - rb * a.Kg;
-        (void)rb;
+        const int g = (u0 + i) % a.Kg;
         const bool first = (i == 0) || (g == 0);
         const bool last = (i == cnt - 1) || (g == a.Kg - 1);
         const int ab = f & 1;
@@ -289,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         const uint8_t* xs = stages + s * kStageBytes + kCodeBytes;
         for (int h = 0; h < 2; ++h) {
-          const int b = hb & 1;
-          if (!wait_or_abort(&wfull[b], static_cast<uint32_t>(hb / 2) & 1u, abort_flag, a.ws_status)) {
+          const int b = hb % kABufs;
+          if (!wait_or_abort(&wfull[b], static_cast<uint32_t>(hb / kABufs) & 1u, abort_flag, a.ws_status)) {
             ok = false;
             break;
           }
@@ -300,9 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d = tbase + static_cast<uint32_t>(ab * 2 * MP + t * MP);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sw128_desc(wbuf + b * kWBytes + t * (128 * 128) + kk * 32);
+              const uint32_t at = tbase + kACol0 + static_cast<uint32_t>(b * 64 + t * 32 + kk * 8);
               const uint64_t bd = sw128_desc(xs + h * kXHalf + kk * 32);
-              mma_f16(d, ad, bd, kIdesc, !(first && h == 0 && kk == 0));
+              mma_f16_ts(d, at, bd, kIdesc, !(first && h == 0 && kk == 0));
             }
           }
           any = true;
@@ -321,148 +409,185 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(tdown, 0);
       }
     }
-  } else if (warp >= 8) {
-    // ---------------- dequantization: thread r owns row r of the block ----------------
-    const int r = threadIdx.x - 256;
-    const uint32_t wb0 = smem_u32(wbuf);
+  } else if (warp < kDqWarps) {
+    // ---------------- dequantization and epilogue ----------------
+    // Warp w: tile t = (w >> 2) & 1, TMEM lane quarter q = w & 3, part p = w >> 3.
+    // Its lanes own rows t*128 + q*32 + lane of the block; of each 64-input half
+    // of a group it converts words 4p .. 4p + 3 (TMEM columns 16p .. 16p + 15 of
+    // the tile), and at the end of a row block it reads out accumulator columns
+    // p*MP/2 .. (p+1)*MP/2 - 1 of its rows.
+    const int t = (warp >> 2) & 1, q = warp & 3, p = warp >> 3;
+    const int rloc = t * 128 + q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t acol = tbase + lane_addr + kACol0 + static_cast<uint32_t>(t * 32 + p * 16);
     const uint32_t st0 = smem_u32(stages);
-    const uint32_t sw_st = static_cast<uint32_t>(r & 7) << 4;          // 128-byte swizzle of w_hat row r
-    const uint32_t sw_ld = static_cast<uint32_t>((r >> 1) & 3);          // 64-byte swizzle of code row r
-    uint32_t d_next = 0, z_next = 0;
-    auto load_dz = [&](int u, uint32_t& dv, uint32_t& zv) {
-      const int rb = u / a.Kg, g = u - rb * a.Kg;
-      const int n = rb * kRows + r;
-      dv = 0;
-      zv = 0;
+    const uint32_t sw_ld = static_cast<uint32_t>((rloc >> 1) & 3);
+    // Delta and z come a block of W groups at a time (W = 1, 2, 4 or 8 divides
+    // K / 128, so the W values of a row are one aligned load), one block ahead.
+    const int W = a.dz_w;
+    uint32_t dc[4], zc[4], dn[4], zn[4];
+    auto issue_dz = [&](int ub) {
+      const int rb = ub / a.Kg, g = ub - rb * a.Kg, g0 = g & ~(W - 1);
+      const int n = rb * kRows + rloc;
       if (n < a.N) {
-        const size_t o = static_cast<size_t>(n) * a.Kg + g;
-        dv = ld_nc_u16(a.scales + o);
-        zv = ld_nc_u16(a.zeros + o);
+        const size_t o = static_cast<size_t>(n) * a.Kg + g0;
+        ld_nc_halves(a.scales + o, W, dn);
+        ld_nc_halves(a.zeros + o, W, zn);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dn[j] = zn[j] = 0;
       }
     };
-    load_dz(u0, d_next, z_next);
-    int hb = 0;
-    for (int i = 0; i < cnt; ++i) {
-      const int s = i % S;
-      const uint32_t dv = d_next, zv = z_next;
-      if (i + 1 < cnt) load_dz(u0 + i + 1, d_next, z_next);
-      if (!wait_or_abort(&full[s], static_cast<uint32_t>(i / S) & 1u, abort_flag, a.ws_status)) break;
-      const __half2 dd = as_h2(dv | (dv << 16));
-      // 1024 + z as an fp16 pair (z is a small non-negative integer held in fp16)
-      const __half zh = __hadd(__ushort_as_half(static_cast<unsigned short>(zv)), __float2half_rn(1024.0f));
-      const __half2 zz = __halves2half2(zh, zh);
-      const uint32_t row = st0 + s * kStageBytes + r * 64;
-      uint4 c[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) c[q] = lds128(row + ((static_cast<uint32_t>(q) ^ sw_ld) << 4));
-      bool ok = true;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int b = hb & 1;
-        if (hb >= 2 && !wait_or_abort(&wempty[b], static_cast<uint32_t>(hb / 2 - 1) & 1u, abort_flag, a.ws_status)) {
-          ok = false;
-          break;
-        }
-        const uint32_t dst = wb0 + b * kWBytes + r * 128;
-        const uint32_t wv[8] = {c[2 * h].x,     c[2 * h].y,     c[2 * h].z,     c[2 * h].w,
-                                c[2 * h + 1].x, c[2 * h + 1].y, c[2 * h + 1].z, c[2 * h + 1].w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t w = wv[j];
-          sts128(dst + ((static_cast<uint32_t>(j) << 4) ^ sw_st), dq_pair(w, zz, dd), dq_pair(w >> 4, zz, dd),
-                 dq_pair(w >> 8, zz, dd), dq_pair(w >> 12, zz, dd));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&wfull[b]);
-        ++hb;
+    int hb = 0, f = 0, start = 0;
+    int pend = -1, pend_rb = 0, pend_contrib = 0;  // a row block whose accumulator awaits read-out
+    bool ok = true;
+    // Read-out of the accumulator of flush number f (row block rb, `contrib` units).
+    auto flush = [&](int fl, int rb, int contrib) {
+      const int ab = fl & 1;
+      const bool okw = wait_or_abort(&afull[ab], static_cast<uint32_t>(fl / 2) & 1u, abort_flag, a.ws_status);
+      if (__any_sync(0xffffffffu, !okw)) {
+        ok = false;
+        return;
       }
-      if (!ok) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rempty[s]);
-    }
-  } else if (warp >= 4) {
-    // ---------------- epilogue: accumulators -> y or workspace ----------------
-    const int q = warp - 4;  // TMEM lane quarter
-    const int te = threadIdx.x - 128;
-    int f = 0, start = 0;
-    for (int i = 0; i < cnt; ++i) {
-      const int u = u0 + i, rb = u / a.Kg, g = u - rb * a.Kg;
-      if (i == 0 || g == 0) start = i;
-      if (!(i == cnt - 1 || g == a.Kg - 1)) continue;
-      const int ab = f & 1;
-      const bool ok = wait_or_abort(&afull[ab], static_cast<uint32_t>(f / 2) & 1u, abort_flag, a.ws_status);
-      if (epi_bar_or(!ok || *abort_flag)) break;
       tc_fence_after();
-      const int contrib = i - start + 1;
       const bool owner = contrib == a.Kg;
+      const int n = rb * kRows + rloc;
+      // a CTA has at most two partial row blocks: the one its range starts in
+      // (slot 0) and the one it ends in (slot 1); blocks in between are whole
+      float4* slot = a.ws_part + static_cast<size_t>(bx * 2 + (rb == rb0 ? 0 : 1)) * (kRows * MP / 4);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int n = rb * kRows + t * 128 + q * 32 + lane;
+      for (int c = 0; c < MP / 16; ++c) {
+        const int m0 = p * (MP / 2) + c * 8;
+        float v[8];
+        tmem_ld8(tbase + lane_addr + static_cast<uint32_t>(ab * 2 * MP + t * MP + m0), v);
+        if (n < a.N) {
+          if (owner) {
 #pragma unroll
-        for (int c = 0; c < MP / 16; ++c) {
-          float v[16];
-          tmem_ld16(tbase + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * 2 * MP + t * MP + c * 16),
-                    v);
-          if (n < a.N) {
-            if (owner) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (c * 16 + j < a.M) a.y[static_cast<size_t>(c * 16 + j) * a.N + n] = __float2half_rn(v[j]);
-            } else {
-              float4* dst = reinterpret_cast<float4*>(a.ws_acc + static_cast<size_t>(n) * MP + c * 16);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                atomicAdd(dst + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-            }
+            for (int j = 0; j < 8; ++j)
+              if (m0 + j < a.M) a.y[static_cast<size_t>(m0 + j) * a.N + n] = __float2half_rn(v[j]);
+          } else {
+            slot[(m0 / 4) * kRows + rloc] = make_float4(v[0], v[1], v[2], v[3]);
+            slot[(m0 / 4 + 1) * kRows + rloc] = make_float4(v[4], v[5], v[6], v[7]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&aempty[ab]);
-      ++f;
-      if (!owner) {
-        __threadfence();
-        epi_bar();
-        if (te == 0)
-          *last_flag = (atomicAdd(a.ws_cnt + rb, static_cast<uint32_t>(contrib)) + contrib ==
-                        static_cast<uint32_t>(a.Kg));
-        epi_bar();
-        if (*last_flag) {
-          __threadfence();
-          for (int rr = te; rr < kRows; rr += 128) {
-            const int n = rb * kRows + rr;
-            if (n >= a.N) continue;
-            float4* src = reinterpret_cast<float4*>(a.ws_acc + static_cast<size_t>(n) * MP);
+    };
+    const int uend = u0 + cnt;
+    int cur_end = u0;  // the Delta / z block in dc / zc covers units up to cur_end - 1
+    issue_dz(u0);
+    for (int i = 0; i < cnt && ok; ++i) {
+      const int u = u0 + i;
+      const int g = u % a.Kg;
+      if (u >= cur_end) {
 #pragma unroll
-            for (int c4 = 0; c4 < MP / 4; ++c4) {
-              const float4 v = __ldcg(src + c4);
-              const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (c4 * 4 + j < a.M) a.y[static_cast<size_t>(c4 * 4 + j) * a.N + n] = __float2half_rn(vv[j]);
-              src[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-          if (te == 0) a.ws_cnt[rb] = 0;
+        for (int j = 0; j < 4; ++j) {
+          dc[j] = dn[j];
+          zc[j] = zn[j];
         }
-        epi_bar();
+        cur_end = u + min(W - (g & (W - 1)), a.Kg - g);
+        if (cur_end < uend) issue_dz(cur_end);
+      }
+      const int s = i % S;
+      const bool okf = wait_or_abort(&full[s], static_cast<uint32_t>(i / S) & 1u, abort_flag, a.ws_status);
+      if (__any_sync(0xffffffffu, !okf)) {
+        ok = false;
+        break;
+      }
+      const uint32_t row = st0 + static_cast<uint32_t>(s * kStageBytes + rloc * 64);
+      const uint4 c0 = lds128(row + ((static_cast<uint32_t>(p) ^ sw_ld) << 4));
+      const uint4 c1 = lds128(row + ((static_cast<uint32_t>(2 + p) ^ sw_ld) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty[s]);  // codes are in registers
+      const uint32_t dv = pick_half(dc, g & (W - 1)), zv = pick_half(zc, g & (W - 1));
+      const __half2 dd = as_h2(dv | (dv << 16));
+      // 1024 + z as an fp16 pair (z is a small non-negative integer held in fp16)
+      const __half zh = __hadd(__ushort_as_half(static_cast<unsigned short>(zv)), __float2half_rn(1024.0f));
+      const __half2 zz = __halves2half2(zh, zh);
+      const int b0 = hb % kABufs, b1 = (hb + 1) % kABufs;
+      bool okw = hb < kABufs ||
+                 wait_or_abort(&wempty[b0], static_cast<uint32_t>(hb / kABufs - 1) & 1u, abort_flag, a.ws_status);
+      okw = okw && (hb + 1 < kABufs || wait_or_abort(&wempty[b1], static_cast<uint32_t>((hb + 1) / kABufs - 1) & 1u,
+                                                    abort_flag, a.ws_status));
+      if (__any_sync(0xffffffffu, !okw)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(acol + static_cast<uint32_t>(b0 * 64), dq_word(c0.x, zz, dd), dq_word(c0.y, zz, dd),
+                dq_word(c0.z, zz, dd), dq_word(c0.w, zz, dd));
+      tmem_st16(acol + static_cast<uint32_t>(b1 * 64), dq_word(c1.x, zz, dd), dq_word(c1.y, zz, dd),
+                dq_word(c1.z, zz, dd), dq_word(c1.w, zz, dd));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&wfull[b0]);
+        mbar_arrive(&wfull[b1]);
+      }
+      hb += 2;
+      // the previous row block's accumulator is complete by now: read it out
+      if (pend >= 0) {
+        flush(pend, pend_rb, pend_contrib);
+        pend = -1;
+        if (!ok) break;
+      }
+      if (i == 0 || g == 0) start = i;
+      if (i == cnt - 1 || g == a.Kg - 1) {
+        pend = f++;
+        pend_rb = u / a.Kg;
+        pend_contrib = i - start + 1;
       }
     }
+    if (ok && pend >= 0) flush(pend, pend_rb, pend_contrib);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tbase, kCols);
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// Sums the partial-sum slots of the row blocks no single CTA covered, in CTA
+// order (so y does not depend on timing), and writes y.  Block (rb, cy): the
+// 256 rows of row block rb, tokens 16 cy .. 16 cy + 15.
+template <int MP>
+__global__ void __launch_bounds__(kRows) gemm_tc_finalize(const TcArgs a, int grid_main) {
+  griddep_wait();
+  const int rb = blockIdx.x;
+  const int base = a.total_units / grid_main;
+  const int rem = a.total_units - base * grid_main;
+  const int c0 = owner_cta(rb * a.Kg, base, rem);
+  const int c1 = owner_cta(rb * a.Kg + a.Kg - 1, base, rem);
+  if (c0 == c1) return;  // one CTA covered the row block and wrote y itself
+  const int r = threadIdx.x;
+  const int n = rb * kRows + r;
+  if (n >= a.N) return;
+  for (int cg = blockIdx.y * 4; cg < blockIdx.y * 4 + 4 && cg < MP / 4; ++cg) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    for (int c = c0; c <= c1; ++c) {
+      const int rbc = (c * base + min(c, rem)) / a.Kg;  // row block where c's range starts
+      const float4 v =
+          __ldcg(a.ws_part + static_cast<size_t>(c * 2 + (rb == rbc ? 0 : 1)) * (kRows * MP / 4) + cg * kRows + r);
+      s0 += v.x;
+      s1 += v.y;
+      s2 += v.z;
+      s3 += v.w;
+    }
+    const float sv[4] = {s0, s1, s2, s3};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (cg * 4 + j < a.M) a.y[static_cast<size_t>(cg * 4 + j) * a.N + n] = __float2half_rn(sv[j]);
   }
 }
 
 int stages_for(int mp) {
   const int stage = kCodeBytes + 2 * mp * 128;
-  int s = (kMaxSmem - 1024 - 2 * kWBytes - kCtrlBytes) / stage;
+  int s = (kMaxSmem - 1024 - kCtrlBytes) / stage;
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -471,27 +596,57 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   TcArgs a = a0;
   a.stages = stages_for(MP);
   if (a.stages < 2) return cudaErrorNotSupported;
-  const int smem = 1024 + 2 * kWBytes + a.stages * (kCodeBytes + 2 * MP * 128) + kCtrlBytes;
+  const int smem = 1024 + a.stages * (kCodeBytes + 2 * MP * 128) + kCtrlBytes;
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<MP><<<grid, kThreads, smem, st>>>(a, tq, tx);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<MP>, a, tq, tx);
+  if (e != cudaSuccess) return e;
+  // the partial sums of row blocks shared by several CTAs; asking for the same
+  // shared-memory carveout as the main kernel spares the SMs a reconfiguration
+  // between the two launches
+  e = cudaFuncSetAttribute(gemm_tc_finalize<MP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  const int row_blocks = (a.N + kRows - 1) / kRows;
+  cudaLaunchConfig_t fin = {};
+  fin.gridDim = dim3(row_blocks, (MP / 4 + 3) / 4);
+  fin.blockDim = dim3(kRows);
+  fin.stream = st;
+  fin.attrs = attr;
+  fin.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&fin, gemm_tc_finalize<MP>, a, grid);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t tc_partial_bytes(int M) {
+  const size_t mp = (static_cast<size_t>(M) + 15) / 16 * 16;
+  return 2 * static_cast<size_t>(device_sm_count()) * kRows * mp * 4;
+}
+
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
-  if (p.M < 1 || p.M > kMaxM) return cudaErrorNotSupported;
+  if (p.M < 1 || p.M > kMaxM || !ws.part) return cudaErrorNotSupported;
   const int mp = (p.M + 15) / 16 * 16;
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  const int Kw = p.K / 8;
 
   // codes: u32 [N][K/8], boxes of 256 rows x 16 words (one group), 64-byte swizzle
   CUtensorMap tq, tx;
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kw), static_cast<cuuint64_t>(p.N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kw) * 4};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K / 8), static_cast<cuuint64_t>(p.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 8) * 4};
     const cuuint32_t box[2] = {16, static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box, estr,
@@ -512,15 +667,17 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
   }
 
   TcArgs a;
+  a.qweight = p.qweight;
   a.scales = p.scales;
   a.zeros = p.zeros;
   a.y = p.y;
-  a.ws_acc = ws.acc;
-  a.ws_cnt = ws.counters;
+  a.ws_part = reinterpret_cast<float4*>(ws.part);
   a.ws_status = ws.status;
   a.M = p.M;
   a.N = p.N;
+  a.Kw = p.K / 8;
   a.Kg = p.K / kGroup;
+  a.dz_w = a.Kg % 8 == 0 ? 8 : (a.Kg % 4 == 0 ? 4 : (a.Kg % 2 == 0 ? 2 : 1));
   const int row_blocks = (p.N + kRows - 1) / kRows;
   a.total_units = row_blocks * a.Kg;
   a.stages = 0;

@@ -29,14 +29,17 @@ cudaError_t launch_act_scale(const __half* X, int T, int K, double alpha, __half
 cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K, int bits, int mode,
                                  uint32_t* qweight, __half* scales, __half* zeros, cudaStream_t st);
 
-// Workspace of the split-K kernels: [status word | padding to 16 B]
-// [row-block counters, padded to 16 B] [fp32 partial sums]: M x N for the
-// CUDA-core GEMV (M <= 4), N x MP (MP = M rounded up to 16) for the
-// tensor-core path.
+// Workspace: [status word | padding to 16 B] [row-block counters, padded to
+// 16 B] [fp32 partial sums M x N of the CUDA-core GEMV, M <= 4] and, for
+// M >= 5, after room for 4 x N GEMV partials: the tensor-core path's
+// partial-sum slots (2 per CTA of 256 x MP fp32, MP = M rounded up to 16).
+// The counters and GEMV partials must be zero when a kernel starts and are
+// left zero; the slots are scratch, written before they are read.
 struct Workspace {
   uint32_t* status;
   uint32_t* counters;
   float* acc;
+  float* part;  // tensor-core partial-sum slots (M >= 5 only), after the GEMV region
 };
 size_t workspace_bytes(int M, int N, int K);
 Workspace carve_workspace(void* base, int M, int N, int K);
@@ -58,7 +61,9 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 
-// The tensor-core skinny GEMM (gemm_tc.cu), M = 5..64.
+// The tensor-core skinny GEMM (gemm_tc.cu), M = 5..64, and the bytes of its
+// partial-sum slots on the current device.
+size_t tc_partial_bytes(int M);
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
