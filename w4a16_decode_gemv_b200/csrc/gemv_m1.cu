@@ -25,17 +25,18 @@
 //
 // Arithmetic.  Codes are unpacked straight into fp32 by one AND each: a nibble
 // at bit position b <= 19 of a word w, isolated as (w & 0xF<<b), reads as the
-// fp32 subnormal q 2^(b-149) (subnormals are kept; nothing here flushes them).
+// fp32 subnormal u 2^(b-149) (subnormals are kept; nothing here flushes them).
 // The two words of a 64-bit half of a lane's 16-byte shared-memory read are
 // processed as one fp32 pair (the same nibble slot of word j and word j+1), so
-// each AND is one 64-bit op on a register pair.  Subtracting the pair
-// (z 2^(b-149), z 2^(b-149)) is exact, and the activations are staged
-// pre-scaled by 2^(109-b), so one packed FMA adds (q - z) x 2^-40 exactly into
-// fp32; 2^40 is folded into Delta.  Slots 5..7 (bits 20..31) are first shifted
+// each AND is one 64-bit op on a register pair.  The activations are staged
+// pre-scaled by 2^(109-b), so one packed FMA adds u x 2^-40 exactly into fp32.
+// The zero point is taken out once per row and lane: sum (u - z) x =
+// sum u x - z sum x, with 2^-40 sum x of the lane's 64 channels staged beside
+// them; 2^40 is folded into Delta.  Slots 5..7 (bits 20..31) are first shifted
 // down by 12.  Per 16 codes: 2 shifts and 16 ANDs on the ALU pipe (which issues
-// at half rate on sm_100, so they bound the inner loop), 8 sub.f32x2 and
-// 8 fma.f32x2 on the FMA pipe.  Lane l owns 64 consecutive input channels
-// (8 words, half a group) of each unit row.
+// at half rate on sm_100, so they bound the inner loop) and 8 fma.f32x2 on the
+// FMA pipe.  Lane l owns 64 consecutive input channels (8 words, half a group)
+// of each unit row.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -89,8 +90,6 @@ __device__ __forceinline__ int slot_bit(int p) { return p <= 4 ? 4 * p : 4 * p -
 // 16b + 2p + (j & 1) holds the element of word j in slot p.
 __device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
 
-// 2^(b-149) for b = 0..16 is subnormal: build it from its bit pattern.
-__device__ __forceinline__ float sub2pow(int b) { return __uint_as_float(1u << b); }
 
 __device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -162,16 +161,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
   // x'' = x * 2^(109 - b(slot)), fp32, in pair order.  Word c (8 channels) is
   // word c & 7 of lane slice c >> 3: block (c >> 1) & 3, pair half c & 1;
   // element 2t sits in slot t, element 2t + 1 in slot 4 + t.
+  // The pad float 64 of each slice holds 2^-40 times the sum of its 64 channels.
+  // K / 8 is a multiple of 16, so the 8 words of a slice are 8 aligned lanes.
   for (int c = threadIdx.x; c < a.K / 8; c += kThreads) {
     const uint4 v = ld_nc_v4(a.x + 8 * c);
     const uint32_t hv[4] = {v.x, v.y, v.z, v.w};
     float* dst = xs + (c >> 3) * kSlice + 16 * ((c >> 1) & 3) + (c & 1);
+    float sum = 0.0f;
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const float2 f = __half22float2(as_h2(hv[t]));
       dst[2 * t] = f.x * pow2f(109 - slot_bit(t));
       dst[8 + 2 * t] = f.y * pow2f(109 - slot_bit(4 + t));
+      sum += f.x + f.y;
     }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+    if ((c & 7) == 0) xs[(c >> 3) * kSlice + 64] = sum * pow2f(-40);
   }
   __syncthreads();
 
@@ -190,7 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
 
     const bool act = lane * 8 < min(kUW, a.Kw - ckc * kUW);
     uint64_t xp[32];
+    float xsum = 0.0f;  // 2^-40 x the sum of this lane's 64 activations
     if (act) {
+      xsum = xs[(ckc * (kUW / 8) + lane) * kSlice + 64];
       const ulonglong2* xb =
           reinterpret_cast<const ulonglong2*>(xs + (ckc * (kUW / 8) + lane) * kSlice) + swap1 * 8;
 #pragma unroll
@@ -227,13 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
         const ulonglong2 wb = wq[r * (kUW / 4) + 1 - 2 * swap1];
         const float zf = __half2float(tile[kR * kUG + r * kUG]);
         const float df = __half2float(tile[r * kUG]) * kTwo40;
-        const uint64_t zz = f2_pack(zf, zf);
-        // (z 2^(b-149), z 2^(b-149)) for b = 0, 4, 8, 12, 16 (exact subnormals)
-        const uint64_t z0 = f2_mul(zz, f2_pack(sub2pow(0), sub2pow(0)));
-        const uint64_t z4 = f2_mul(zz, f2_pack(sub2pow(4), sub2pow(4)));
-        const uint64_t z8 = f2_mul(zz, f2_pack(sub2pow(8), sub2pow(8)));
-        const uint64_t z12 = f2_mul(zz, f2_pack(sub2pow(12), sub2pow(12)));
-        const uint64_t z16 = f2_mul(zz, f2_pack(sub2pow(16), sub2pow(16)));
         uint64_t pa = 0, pb = 0;
         const uint64_t blk[4] = {wa.x, wa.y, wb.x, wb.y};
 #pragma unroll
@@ -241,17 +243,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
           const uint64_t w = blk[b];
           const uint64_t h = f2_pack(static_cast<uint32_t>(w) >> 12, static_cast<uint32_t>(w >> 32) >> 12);
           const uint64_t* x8 = xp + 8 * b;
-          pa = f2_fma(f2_sub(w & 0x0000000F0000000Full, z0), x8[0], pa);
-          pb = f2_fma(f2_sub(w & 0x000000F0000000F0ull, z4), x8[1], pb);
-          pa = f2_fma(f2_sub(w & 0x00000F0000000F00ull, z8), x8[2], pa);
-          pb = f2_fma(f2_sub(w & 0x0000F0000000F000ull, z12), x8[3], pb);
-          pa = f2_fma(f2_sub(w & 0x000F0000000F0000ull, z16), x8[4], pa);
-          pb = f2_fma(f2_sub(h & 0x00000F0000000F00ull, z8), x8[5], pb);
-          pa = f2_fma(f2_sub(h & 0x0000F0000000F000ull, z12), x8[6], pa);
-          pb = f2_fma(f2_sub(h & 0x000F0000000F0000ull, z16), x8[7], pb);
+          pa = f2_fma(w & 0x0000000F0000000Full, x8[0], pa);
+          pb = f2_fma(w & 0x000000F0000000F0ull, x8[1], pb);
+          pa = f2_fma(w & 0x00000F0000000F00ull, x8[2], pa);
+          pb = f2_fma(w & 0x0000F0000000F000ull, x8[3], pb);
+          pa = f2_fma(w & 0x000F0000000F0000ull, x8[4], pa);
+          pb = f2_fma(h & 0x00000F0000000F00ull, x8[5], pb);
+          pa = f2_fma(h & 0x0000F0000000F000ull, x8[6], pa);
+          pb = f2_fma(h & 0x000F0000000F0000ull, x8[7], pb);
         }
         const float2 fa = f2_unpack(pa), fb = f2_unpack(pb);
-        acc[r] = df * ((fa.x + fb.x) + (fa.y + fb.y));
+        // sum (u - z) x = sum u x - z sum x, all scaled by 2^-40
+        acc[r] = df * fmaf(-zf, xsum, (fa.x + fb.x) + (fa.y + fb.y));
       }
     }
     // refill the stage with this warp's unit i + S (its reads above are done)
