@@ -53,6 +53,7 @@ constexpr int kUB = kR * kUW * 4;             // 4 KiB of codes per unit
 constexpr int kUG = kUW / 16;                 // 16 groups per unit row
 constexpr int kStage = kUB + 2 * kR * kUG * 2;  // + Delta and z tiles (4 x 16 fp16 each)
 constexpr int kSlice = 68;                    // floats per 64-channel lane slice (+4 pad)
+constexpr int kXBatch = 4;                    // activation words a thread loads at once while staging
 constexpr int kMaxSmem = 227 * 1024;
 constexpr float kTwo40 = 1099511627776.0f;   // 2^40
 
@@ -163,22 +164,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
   // element 2t sits in slot t, element 2t + 1 in slot 4 + t.
   // The pad float 64 of each slice holds 2^-40 times the sum of its 64 channels.
   // K / 8 is a multiple of 16, so the 8 words of a slice are 8 aligned lanes.
-  for (int c = threadIdx.x; c < a.K / 8; c += kThreads) {
-    const uint4 v = ld_nc_v4(a.x + 8 * c);
-    const uint32_t hv[4] = {v.x, v.y, v.z, v.w};
-    float* dst = xs + (c >> 3) * kSlice + 16 * ((c >> 1) & 3) + (c & 1);
-    float sum = 0.0f;
+  // All of a thread's loads are issued before any is used, so the staging costs
+  // one trip to L2 rather than one per word.
+  // The loop bound is the warp's first word, so every lane runs every shuffle;
+  // lanes past the end contribute nothing.
+  for (int c0 = threadIdx.x; c0 - lane < a.K / 8; c0 += kXBatch * kThreads) {
+    uint4 v[kXBatch];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const float2 f = __half22float2(as_h2(hv[t]));
-      dst[2 * t] = f.x * pow2f(109 - slot_bit(t));
-      dst[8 + 2 * t] = f.y * pow2f(109 - slot_bit(4 + t));
-      sum += f.x + f.y;
+    for (int q = 0; q < kXBatch; ++q) {
+      const int c = c0 + q * kThreads;
+      v[q] = c < a.K / 8 ? ld_nc_v4(a.x + 8 * c) : make_uint4(0, 0, 0, 0);
     }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-    if ((c & 7) == 0) xs[(c >> 3) * kSlice + 64] = sum * pow2f(-40);
+#pragma unroll
+    for (int q = 0; q < kXBatch; ++q) {
+      const int c = c0 + q * kThreads;
+      if (c - lane >= a.K / 8) break;  // uniform over the warp
+      const bool valid = c < a.K / 8;
+      const uint32_t hv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+      float* dst = xs + (c >> 3) * kSlice + 16 * ((c >> 1) & 3) + (c & 1);
+      float sum = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __half22float2(as_h2(hv[t]));
+        if (valid) {
+          dst[2 * t] = f.x * pow2f(109 - slot_bit(t));
+          dst[8 + 2 * t] = f.y * pow2f(109 - slot_bit(4 + t));
+        }
+        sum += f.x + f.y;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      if (valid && (c & 7) == 0) xs[(c >> 3) * kSlice + 64] = sum * pow2f(-40);
+    }
   }
   __syncthreads();
 
@@ -188,6 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
   const int swap1 = (lane >> 2) & 1;
   bool failed = false;
   int kc = warp % a.units_k;
+  // this lane's staged activations for channel block xkc (reloaded only when the
+  // warp's block changes; with 16 warps and K / 2048 dividing 16 it never does)
+  int xkc = -1;
+  uint64_t xp[32];
+  float xsum = 0.0f;  // 2^-40 x the sum of this lane's 64 activations
   for (int j = warp, i = 0; j < U; j += kWarps, ++i) {
     const int s = i % S;
     const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
@@ -196,24 +219,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
     if (kc >= a.units_k) kc -= a.units_k;
 
     const bool act = lane * 8 < min(kUW, a.Kw - ckc * kUW);
-    uint64_t xp[32];
-    float xsum = 0.0f;  // 2^-40 x the sum of this lane's 64 activations
-    if (act) {
-      xsum = xs[(ckc * (kUW / 8) + lane) * kSlice + 64];
-      const ulonglong2* xb =
-          reinterpret_cast<const ulonglong2*>(xs + (ckc * (kUW / 8) + lane) * kSlice) + swap1 * 8;
+    if (ckc != xkc) {
+      xkc = ckc;
+      if (act) {
+        xsum = xs[(ckc * (kUW / 8) + lane) * kSlice + 64];
+        const ulonglong2* xb =
+            reinterpret_cast<const ulonglong2*>(xs + (ckc * (kUW / 8) + lane) * kSlice) + swap1 * 8;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const ulonglong2 v = xb[c];
-        xp[2 * c] = v.x;
-        xp[2 * c + 1] = v.y;
-      }
-      xb += 8 - 16 * swap1;
+        for (int c = 0; c < 8; ++c) {
+          const ulonglong2 v = xb[c];
+          xp[2 * c] = v.x;
+          xp[2 * c + 1] = v.y;
+        }
+        xb += 8 - 16 * swap1;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const ulonglong2 v = xb[c];
-        xp[16 + 2 * c] = v.x;
-        xp[16 + 2 * c + 1] = v.y;
+        for (int c = 0; c < 8; ++c) {
+          const ulonglong2 v = xb[c];
+          xp[16 + 2 * c] = v.x;
+          xp[16 + 2 * c + 1] = v.y;
+        }
       }
     }
 
