@@ -147,14 +147,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
   }
   __syncwarp();
   const uint64_t pol = l2_evict_first_policy();
-  // prologue: fill the ring (codes, Delta and z are read-only)
+  // prologue: the first stage of the ring (codes, Delta and z are read-only, so
+  // this overlaps the previous kernel's tail).  Only one: the activations are
+  // loaded right after griddep_wait and should not queue behind more weights.
   int rb_f = rb0 + warp / a.units_k, kc_f = warp % a.units_k;
   int jf = warp;
-  for (int s = 0; s < S && jf < U; ++s, jf += kWarps) {
+  auto issue_next = [&](int s) {
     issue_unit(a, &tmap, rb_f, kc_f, ring + static_cast<size_t>(s) * kStage, &full[s], lane, pol);
+    jf += kWarps;
     rb_f += drb, kc_f += dkc;
     if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
-  }
+  };
+  if (jf < U) issue_next(0);
 
   // x, y and anything earlier kernels produce are touched only after this
   griddep_wait();
@@ -199,6 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
     }
   }
   __syncthreads();
+  // the rest of the ring
+  for (int s = 1; s < S && jf < U; ++s) issue_next(s);
 
   // Lanes with bit 2 set read the second half of their slice first (weights
   // and activations alike) so that the 32-byte lane stride does not put two
@@ -283,12 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, co
     }
     // refill the stage with this warp's unit i + S (its reads above are done)
     __syncwarp();
-    if (jf < U) {
-      issue_unit(a, &tmap, rb_f, kc_f, stage, &full[s], lane, pol);
-      jf += kWarps;
-      rb_f += drb, kc_f += dkc;
-      if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
-    }
+    if (jf < U) issue_next(s);
     // reduce the unit's 4 row partials over the lanes
     const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
     float k0 = b0 ? acc[2] : acc[0];
