@@ -158,6 +158,8 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   cudaError_t e;
   if (M == 1 && gemv_m1_supports(N, K)) {
     e = launch_gemv_m1(p, ws.status, st);
+  } else if (gemv_mt_supports(M, N, K)) {
+    e = launch_gemv_mt(p, ws.status, st);
   } else if (M <= kMaxGemvM && gemv_supports(M, K)) {
     e = launch_gemv(p, ws, st);
   } else {

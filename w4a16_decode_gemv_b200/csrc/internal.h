@@ -57,6 +57,11 @@ struct GemmProblem {
 bool gemv_m1_supports(int N, int K);
 cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t st);
 
+// The M = 2..4 GEMV (gemv_mt.cu): whole rows per CTA, no workspace; false when
+// the staged activations of M tokens do not fit in shared memory.
+bool gemv_mt_supports(int M, int N, int K);
+cudaError_t launch_gemv_mt(const GemmProblem& p, uint32_t* status, cudaStream_t st);
+
 // The split-K CUDA-core GEMV for small M (gemv.cu).
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
