@@ -13,7 +13,8 @@
 // contiguous, balanced ranges, so a CTA owns whole rows and no partial sum
 // leaves the SM.  A CTA's row blocks are cut into units of 4 rows x 2048 input
 // channels (4 KiB of codes plus the 4 x 16 Delta and z of those rows), and warp
-// w of the CTA takes units w, w + 16, w + 32, ...  Each warp streams its own
+// w of the CTA takes units w, w + W, w + 2W, ... (W = 16 warps, or 12 when
+// the staged activations of a large K leave room for only 12 rings)  Each warp streams its own
 // units through a private ring of shared-memory stages: one lane issues a 2-D
 // tensor copy (TMA, box of 4 rows x 256 words, zero fill past the matrix edge)
 // per unit and all lanes copy the Delta / z tile with cp.async, all completing
@@ -45,8 +46,6 @@
 namespace w4a16 {
 namespace {
 
-constexpr int kWarps = 16;                    // warps per CTA
-constexpr int kThreads = kWarps * 32;
 constexpr int kR = 4;                         // rows per unit (= rows per row block)
 constexpr int kUW = 256;                      // words per unit row (2048 channels)
 constexpr int kUB = kR * kUW * 4;             // 4 KiB of codes per unit
@@ -124,7 +123,13 @@ __device__ __forceinline__ void issue_unit(const M1Args& a, const CUtensorMap* t
   cp_async_arrive(bar);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1Args a, const __grid_constant__ CUtensorMap tmap) {
+// WARPS = 16, or 12 when 16 rings do not fit beside the staged activations
+// (large K).
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+    gemv_m1_kernel(const M1Args a, const __grid_constant__ CUtensorMap tmap) {
+  constexpr int kWarps = WARPS;
+  constexpr int kThreads = WARPS * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
@@ -326,19 +331,27 @@ int round128(int b) { return (b + 127) / 128 * 128; }
 
 int x_bytes_for(int K) { return round128((K / 64) * kSlice * 4); }
 
-int smem_for(int stages, int x_bytes, int max_units) {
-  return x_bytes + kWarps * stages * kStage + round128(max_units * kR * 4) + kWarps * stages * 8;
+int smem_for(int warps, int stages, int x_bytes, int max_units) {
+  return x_bytes + warps * stages * kStage + round128(max_units * kR * 4) + warps * stages * 8;
+}
+
+// Warps per CTA: 16 if two ring stages per warp fit, else 12, else 0.
+int m1_warps(int N, int K, int& max_units) {
+  const int sms = device_sm_count();
+  const int row_blocks = (N + kR - 1) / kR;
+  const int grid = min(sms, row_blocks);
+  max_units = ((row_blocks + grid - 1) / grid) * ((K / 8 + kUW - 1) / kUW);
+  for (int w : {16, 12})
+    if (smem_for(w, 2, x_bytes_for(K), max_units) <= kMaxSmem) return w;
+  return 0;
 }
 
 }  // namespace
 
 bool gemv_m1_supports(int N, int K) {
   if ((K / kGroup) % 2) return false;  // Delta/z pairs are copied 4 bytes at a time
-  const int sms = device_sm_count();
-  const int row_blocks = (N + kR - 1) / kR;
-  const int grid = min(sms, row_blocks);
-  const int max_units = ((row_blocks + grid - 1) / grid) * ((K / 8 + kUW - 1) / kUW);
-  return smem_for(2, x_bytes_for(K), max_units) <= kMaxSmem;
+  int max_units;
+  return m1_warps(N, K, max_units) != 0;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -372,12 +385,14 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   const int grid = min(device_sm_count(), a.row_blocks);
   a.max_units = ((a.row_blocks + grid - 1) / grid) * a.units_k;
   a.x_bytes = x_bytes_for(p.K);
+  int mu;
+  const int warps = m1_warps(p.N, p.K, mu);
+  if (warps == 0) return cudaErrorNotSupported;
   // deepest per-warp ring that fits
   int stages = 6;
-  while (stages > 2 && smem_for(stages, a.x_bytes, a.max_units) > kMaxSmem) --stages;
-  if (smem_for(stages, a.x_bytes, a.max_units) > kMaxSmem) return cudaErrorNotSupported;
+  while (stages > 2 && smem_for(warps, stages, a.x_bytes, a.max_units) > kMaxSmem) --stages;
   a.stages = stages;
-  const int smem = smem_for(stages, a.x_bytes, a.max_units);
+  const int smem = smem_for(warps, stages, a.x_bytes, a.max_units);
 
   // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256
   CUtensorMap tmap;
@@ -392,11 +407,12 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
-  cudaError_t e = cudaFuncSetAttribute(gemv_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  auto kern = warps == 16 ? gemv_m1_kernel<16> : gemv_m1_kernel<12>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(warps * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -404,7 +420,7 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, gemv_m1_kernel, a, tmap);
+  e = cudaLaunchKernelEx(&cfg, kern, a, tmap);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
