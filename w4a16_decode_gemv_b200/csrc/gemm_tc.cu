@@ -176,28 +176,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
-// Named barrier over the four epilogue warps; returns the OR of `pred` over them.
-__device__ __forceinline__ bool epi_bar_or(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred))
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// Adds four fp32 values into global memory without returning the old ones, so
-// the thread does not wait for the L2 round trip (a later fence orders them).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
 __device__ __forceinline__ uint32_t lop3_nib(uint32_t w) {
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
@@ -238,8 +216,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t dq_pair(uint32_t v, __half2 zz, __half2 dd) {
-  return as_u32(__hmul2(__hsub2(as_h2(lop3_nib(v)), zz), dd));
+// (1024 + u) - (1024 + z) = u - z exactly, computed as an FMA with 1 (the fp16
+// add and subtract instructions issue far slower than FMA on sm_100a), then one
+// rounding in the multiply by Delta.  nz = -(1024 + z).
+__device__ __forceinline__ uint32_t dq_pair(uint32_t v, __half2 nz, __half2 dd) {
+  return as_u32(__hmul2(__hfma2(as_h2(lop3_nib(v)), __float2half2_rn(1.0f), nz), dd));
 }
 
 __device__ __forceinline__ Word4 dq_word(uint32_t w, __half2 zz, __half2 dd) {
@@ -503,8 +484,8 @@ __global__ void __maxnreg__(96)
       if (lane == 0) mbar_arrive(&rempty[s]);  // codes are in registers
       const uint32_t dv = pick_half(dc, g & (W - 1)), zv = pick_half(zc, g & (W - 1));
       const __half2 dd = as_h2(dv | (dv << 16));
-      // 1024 + z as an fp16 pair (z is a small non-negative integer held in fp16)
-      const __half zh = __hadd(__ushort_as_half(static_cast<unsigned short>(zv)), __float2half_rn(1024.0f));
+      // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
+      const __half zh = __hneg(__hadd(__ushort_as_half(static_cast<unsigned short>(zv)), __float2half_rn(1024.0f)));
       const __half2 zz = __halves2half2(zh, zh);
       const int b0 = hb % kABufs, b1 = (hb + 1) % kABufs;
       bool okw = hb < kABufs ||

@@ -307,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_multi_kernel(const GemvArgs 
         const uint32_t nz_lo = as_u32(__hneg2(__hadd2(z2, __floats2half2_rn(1024.0f, 1024.0f))));
         const uint32_t nz_hi = as_u32(__hneg2(__hadd2(z2, __floats2half2_rn(64.0f, 64.0f))));
         const __half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+        // the adds are FMAs with 1: fp16 add issues far slower than FMA on sm_100a
+        const __half2 one = __floats2half2_rn(1.0f, 1.0f);
         // (u - z) for the 32 channels, as exact fp16 pairs
         uint32_t dq[16];
         const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
@@ -314,9 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_multi_kernel(const GemvArgs 
         for (int c = 0; c < 4; ++c) {
           const uint32_t w = wv[c];
           const uint32_t w8 = w >> 8;
-          dq[4 * c + 0] = as_u32(__hadd2(as_h2(nib_to_f16x2(w, 0x000F000Fu)), as_h2(nz_lo)));
+          dq[4 * c + 0] = as_u32(__hfma2(as_h2(nib_to_f16x2(w, 0x000F000Fu)), one, as_h2(nz_lo)));
           dq[4 * c + 1] = as_u32(__hfma2(as_h2(nib_to_f16x2(w, 0x00F000F0u)), sixteenth, as_h2(nz_hi)));
-          dq[4 * c + 2] = as_u32(__hadd2(as_h2(nib_to_f16x2(w8, 0x000F000Fu)), as_h2(nz_lo)));
+          dq[4 * c + 2] = as_u32(__hfma2(as_h2(nib_to_f16x2(w8, 0x000F000Fu)), one, as_h2(nz_lo)));
           dq[4 * c + 3] = as_u32(__hfma2(as_h2(nib_to_f16x2(w8, 0x00F000F0u)), sixteenth, as_h2(nz_hi)));
         }
         const float delta = __half2float(__ushort_as_half(static_cast<unsigned short>(dz[r] & 0xFFFFu)));
