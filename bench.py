@@ -64,6 +64,11 @@ def workload_config(layers=LAYERS):
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
+def whole_job_gbps(world, bytes_per_step, ms_per_step):
+    """Weak scaling: every rank streams bytes_per_step per step; the step time is the max over ranks."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
+
+
 class Dist:
     def __init__(self, gpus):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -279,7 +284,7 @@ def run_ours(args, dist):
     ms_per_step = ms / args.steps
     w4.gemm_check(ws)
     bytes_step = L * WEIGHT_BYTES
-    value = dist.world * bytes_step / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbps(dist.world, bytes_step, ms_per_step)
     us_layer = ms_per_step * 1e3 / L
 
     # ---- e2e through the public API (eager), pinned host input/output every step
