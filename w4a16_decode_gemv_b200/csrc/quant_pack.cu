@@ -75,7 +75,22 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // quotient decides every half-integer boundary exactly: for fp16 w and d with
 // |w / d| < 2^5 a non-tie quotient lies at least 2^-14 from a half-integer,
 // far beyond the fp32 rounding error, and an exact tie is representable.
-__device__ __forceinline__ float round_quotient(float w, float d) { return rintf(__fdiv_rn(w, d)); }
+//
+// The quotient itself comes from the correctly rounded reciprocal of d (one per
+// group): q = w * rcp_rn(d) is within 2^-18 of w / d for |w / d| < 2^5 (two
+// fp32 roundings), so rint(q) is already the right decision unless q lies
+// within 2^-16 of a half-integer k + 1/2; only then is w compared with
+// (k + 1/2) d, which is exact in fp32 (an 11-bit by 7-bit product).  Equality
+// is an exact tie (round half to even); otherwise the side of w decides.
+// Quotients of 2^5 and more only reach clamped codes.
+__device__ __forceinline__ float round_quotient(float w, float d, float inv_d) {
+  const float q = w * inv_d;
+  const float k = floorf(q);
+  if (fabsf(q - k - 0.5f) >= 0x1p-16f) return rintf(q);
+  const float t = (k + 0.5f) * d;
+  if (w == t) return rintf(k + 0.5f);
+  return w > t ? k + 1.0f : k;  // d > 0
+}
 
 template <int BITS, int MODE, bool HAS_S>
 __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half* __restrict__ W,
@@ -160,12 +175,13 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half*
       if (g >= total) continue;
       // a4: u = clamp(Round(w' / Delta) + z, 0, 2^N - 1);  a5: pack into layout v1
       const float df = __half2float(d);
+      const float inv_d = __frcp_rn(df);
       uint32_t word = 0;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 wf = __half22float2(w2[t]);
-        const float u0 = fminf(fmaxf(round_quotient(wf.x, df) + zf, 0.0f), static_cast<float>(kQmax));
-        const float u1 = fminf(fmaxf(round_quotient(wf.y, df) + zf, 0.0f), static_cast<float>(kQmax));
+        const float u0 = fminf(fmaxf(round_quotient(wf.x, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax));
+        const float u1 = fminf(fmaxf(round_quotient(wf.y, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax));
         word |= (static_cast<uint32_t>(u0) << (4 * t)) | (static_cast<uint32_t>(u1) << (16 + 4 * t));
       }
       const long long n = g / Kg;
