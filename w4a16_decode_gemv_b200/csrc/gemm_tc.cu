@@ -364,16 +364,20 @@ __global__ void __maxnreg__(96)
             break;
           }
           tc_fence_after();
+          // Addresses computed once per half: the B descriptor's start-address
+          // field advances by 32 bytes (2 in 16-byte units) per 16 inputs, A
+          // and D are tensor-memory columns at fixed offsets.  This thread
+          // shares its scheduler with dequantizing warps, so few instructions
+          // per MMA matter.
+          const uint64_t bd0 = sw128_desc(xs + h * kXHalf);
+          const uint32_t at0 = tbase + kACol0 + static_cast<uint32_t>(b * 64);
+          const uint32_t d0 = tbase + static_cast<uint32_t>(ab * 2 * MP);
+          const bool acc0 = !(first && h == 0);
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const uint32_t d = tbase + static_cast<uint32_t>(ab * 2 * MP + t * MP);
+          for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t at = tbase + kACol0 + static_cast<uint32_t>(b * 64 + t * 32 + kk * 8);
-              const uint64_t bd = sw128_desc(xs + h * kXHalf + kk * 32);
-              mma_f16_ts(d, at, bd, kIdesc, !(first && h == 0 && kk == 0));
-            }
-          }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts(d0 + t * MP, at0 + t * 32 + kk * 8, bd0 + 2 * kk, kIdesc, kk > 0 || acc0);
           any = true;
           mma_commit(&wempty[b]);
           ++hb;
