@@ -24,20 +24,20 @@
 // them in a shared slot of their own; at the end the CTA adds the slots of each
 // row in a fixed order, so y does not depend on timing.
 //
-// Arithmetic.  Codes are unpacked straight into fp32 by one AND each: a nibble
-// at bit position b <= 19 of a word w, isolated as (w & 0xF<<b), reads as the
-// fp32 subnormal u 2^(b-149) (subnormals are kept; nothing here flushes them).
-// The two words of a 64-bit half of a lane's 16-byte shared-memory read are
-// processed as one fp32 pair (the same nibble slot of word j and word j+1), so
-// each AND is one 64-bit op on a register pair.  The activations are staged
-// pre-scaled by 2^(109-b), so one packed FMA adds u x 2^-40 exactly into fp32.
-// The zero point is taken out once per row and lane: sum (u - z) x =
-// sum u x - z sum x, with 2^-40 sum x of the lane's 64 channels staged beside
-// them; 2^40 is folded into Delta.  Slots 5..7 (bits 20..31) are first shifted
-// down by 12.  Per 16 codes: 2 shifts and 16 ANDs on the ALU pipe (which issues
-// at half rate on sm_100, so they bound the inner loop) and 8 fma.f32x2 on the
-// FMA pipe.  Lane l owns 64 consecutive input channels (8 words, half a group)
-// of each unit row.
+// Arithmetic.  Layout v1 puts elements 2t and 2t+1 of a word in nibble slots t
+// and t+4, i.e. at bits 4t and 4t+16: the two 16-bit halves of the word carry
+// a pair of consecutive elements.  One AND with 0x000F000F isolates elements
+// (0, 1) as the fp16 subnormal pair u 2^-24, one with 0x00F000F0 elements (2, 3)
+// as u 2^-20 (mantissa bits 4..7); the same two masks on w >> 8 give (4, 5) and
+// (6, 7).  Each fp16 pair meets the matching pair of activations, which are the
+// input's own fp16 pairs in natural order, in two mixed fp16 x fp16 -> fp32
+// FMAs (fma.rn.f32.f16): the products are exact in fp32 and the sums are fp32.
+// Per word: 1 shift and 4 ANDs on the ALU pipe (half rate on sm_100) and 8
+// mixed FMAs.  The u 2^-20 family is kept in accumulators of its own and scaled
+// by 2^-4 once per row.  The zero point is taken out once per row and lane:
+// sum (u - z) x = sum u x - z sum x, with 2^-24 sum x of the lane's 64 channels
+// staged beside them; 2^24 is folded into Delta.  Lane l owns 64 consecutive
+// input channels (8 words, half a group) of each unit row.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -51,10 +51,10 @@ constexpr int kUW = 256;                      // words per unit row (2048 channe
 constexpr int kUB = kR * kUW * 4;             // 4 KiB of codes per unit
 constexpr int kUG = kUW / 16;                 // 16 groups per unit row
 constexpr int kStage = kUB + 2 * kR * kUG * 2;  // + Delta and z tiles (4 x 16 fp16 each)
-constexpr int kSlice = 68;                    // floats per 64-channel lane slice (+4 pad)
+constexpr int kSlice = 36;                    // 4-byte words per 64-channel lane slice (33 used)
 constexpr int kXBatch = 4;                    // activation words a thread loads at once while staging
 constexpr int kMaxSmem = 227 * 1024;
-constexpr float kTwo40 = 1099511627776.0f;   // 2^40
+constexpr float kTwo24 = 16777216.0f;        // 2^24
 
 struct M1Args {
   const __half* x;
@@ -80,14 +80,10 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 }
 
 
-// Slot p of layout v1 holds element i = (p < 4 ? 2p : 2(p-4)+1) of its word.
-// Bit offset of slot p after the optional shift by 12: 4p (p <= 4), 4p - 12.
-__device__ __forceinline__ int slot_bit(int p) { return p <= 4 ? 4 * p : 4 * p - 12; }
-
 // Staged activations: channels are grouped in 64-channel lane slices kSlice
-// floats apart (the 16-byte pad makes the quarter-warp phases of a 128-bit read
-// hit distinct banks); inside a slice, block b = words 2b and 2b+1, and float
-// 16b + 2p + (j & 1) holds the element of word j in slot p.
+// 4-byte words apart (the 16-byte pad makes the quarter-warp phases of a
+// 128-bit read hit distinct banks); a slice holds its 8 words of fp16 x (16
+// bytes each) in the owning lane's read order, then 2^-24 times their sum.
 __device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
 
 
@@ -168,10 +164,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
   // x, y and anything earlier kernels produce are touched only after this
   griddep_wait();
 
-  // x'' = x * 2^(109 - b(slot)), fp32, in pair order.  Word c (8 channels) is
-  // word c & 7 of lane slice c >> 3: block (c >> 1) & 3, pair half c & 1;
-  // element 2t sits in slot t, element 2t + 1 in slot 4 + t.
-  // The pad float 64 of each slice holds 2^-40 times the sum of its 64 channels.
+  // Word c of x (8 channels) is word c & 7 of lane slice c >> 3.  The slice's
+  // lane (c >> 3) & 31 reads its second 16-byte half first when bit 2 of the
+  // lane index is set (see swap1 below), so the words are stored in that order.
+  // Word 32 of each slice holds 2^-24 times the sum of its 64 channels.
   // K / 8 is a multiple of 16, so the 8 words of a slice are 8 aligned lanes.
   // All of a thread's loads are issued before any is used, so the staging costs
   // one trip to L2 rather than one per word.
@@ -190,38 +186,38 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
       if (c - lane >= a.K / 8) break;  // uniform over the warp
       const bool valid = c < a.K / 8;
       const uint32_t hv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-      float* dst = xs + (c >> 3) * kSlice + 16 * ((c >> 1) & 3) + (c & 1);
+      // position of word c in its owning lane's read order
+      const int jj = ((c & 7) - 4 * ((c >> 5) & 1)) & 7;
+      float* slice = xs + (c >> 3) * kSlice;
       float sum = 0.0f;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 f = __half22float2(as_h2(hv[t]));
-        if (valid) {
-          dst[2 * t] = f.x * pow2f(109 - slot_bit(t));
-          dst[8 + 2 * t] = f.y * pow2f(109 - slot_bit(4 + t));
-        }
         sum += f.x + f.y;
       }
+      if (valid) *reinterpret_cast<uint4*>(slice + 4 * jj) = v[q];
       sum += __shfl_xor_sync(0xffffffffu, sum, 1);
       sum += __shfl_xor_sync(0xffffffffu, sum, 2);
       sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      if (valid && (c & 7) == 0) xs[(c >> 3) * kSlice + 64] = sum * pow2f(-40);
+      if (valid && (c & 7) == 0) slice[32] = sum * pow2f(-24);
     }
   }
   __syncthreads();
   // the rest of the ring
   for (int s = 1; s < S && jf < U; ++s) issue_next(s);
 
-  // Lanes with bit 2 set read the second half of their slice first (weights
-  // and activations alike) so that the 32-byte lane stride does not put two
-  // lanes of a quarter-warp phase on the same banks.
+  // Lanes with bit 2 set read the second 16-byte half of their 32 bytes of a
+  // weight row first, so that the 32-byte lane stride does not put two lanes of
+  // a quarter-warp phase on the same banks (their x slices are staged in the
+  // same order).
   const int swap1 = (lane >> 2) & 1;
   bool failed = false;
   int kc = warp % a.units_k;
   // this lane's staged activations for channel block xkc (reloaded only when the
   // warp's block changes; with 16 warps and K / 2048 dividing 16 it never does)
   int xkc = -1;
-  uint64_t xp[32];
-  float xsum = 0.0f;  // 2^-40 x the sum of this lane's 64 activations
+  uint32_t xh[32];     // x as fp16 pairs, the lane's 8 words in read order
+  float xsum = 0.0f;  // 2^-24 x the sum of this lane's 64 activations
   for (int j = warp, i = 0; j < U; j += kWarps, ++i) {
     const int s = i % S;
     const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
@@ -233,21 +229,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     if (ckc != xkc) {
       xkc = ckc;
       if (act) {
-        xsum = xs[(ckc * (kUW / 8) + lane) * kSlice + 64];
-        const ulonglong2* xb =
-            reinterpret_cast<const ulonglong2*>(xs + (ckc * (kUW / 8) + lane) * kSlice) + swap1 * 8;
+        const float* sl = xs + (ckc * (kUW / 8) + lane) * kSlice;
+        xsum = sl[32];
+        const uint4* xb = reinterpret_cast<const uint4*>(sl);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const ulonglong2 v = xb[c];
-          xp[2 * c] = v.x;
-          xp[2 * c + 1] = v.y;
-        }
-        xb += 8 - 16 * swap1;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const ulonglong2 v = xb[c];
-          xp[16 + 2 * c] = v.x;
-          xp[16 + 2 * c + 1] = v.y;
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = xb[k];
+          xh[4 * k] = v.x;
+          xh[4 * k + 1] = v.y;
+          xh[4 * k + 2] = v.z;
+          xh[4 * k + 3] = v.w;
         }
       }
     }
@@ -270,26 +261,24 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         const ulonglong2 wa = wq[r * (kUW / 4)];
         const ulonglong2 wb = wq[r * (kUW / 4) + 1 - 2 * swap1];
         const float zf = __half2float(tile[kR * kUG + r * kUG]);
-        const float df = __half2float(tile[r * kUG]) * kTwo40;
-        uint64_t pa = 0, pb = 0;
-        const uint64_t blk[4] = {wa.x, wa.y, wb.x, wb.y};
+        const float df = __half2float(tile[r * kUG]) * kTwo24;
+        // u 2^-24 (bits 0..3 of each 16-bit half) and u 2^-20 (bits 4..7) are
+        // fp16 subnormals; their products with x are exact in fp32
+        float e0 = 0.0f, e1 = 0.0f, o0 = 0.0f, o1 = 0.0f;
+        const uint32_t hw[8] = {static_cast<uint32_t>(wa.x), static_cast<uint32_t>(wa.x >> 32),
+                                static_cast<uint32_t>(wa.y), static_cast<uint32_t>(wa.y >> 32),
+                                static_cast<uint32_t>(wb.x), static_cast<uint32_t>(wb.x >> 32),
+                                static_cast<uint32_t>(wb.y), static_cast<uint32_t>(wb.y >> 32)};
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint64_t w = blk[b];
-          const uint64_t h = f2_pack(static_cast<uint32_t>(w) >> 12, static_cast<uint32_t>(w >> 32) >> 12);
-          const uint64_t* x8 = xp + 8 * b;
-          pa = f2_fma(w & 0x0000000F0000000Full, x8[0], pa);
-          pb = f2_fma(w & 0x000000F0000000F0ull, x8[1], pb);
-          pa = f2_fma(w & 0x00000F0000000F00ull, x8[2], pa);
-          pb = f2_fma(w & 0x0000F0000000F000ull, x8[3], pb);
-          pa = f2_fma(w & 0x000F0000000F0000ull, x8[4], pa);
-          pb = f2_fma(h & 0x00000F0000000F00ull, x8[5], pb);
-          pa = f2_fma(h & 0x0000F0000000F000ull, x8[6], pa);
-          pb = f2_fma(h & 0x000F0000000F0000ull, x8[7], pb);
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t w = hw[k], w8 = w >> 8;
+          fma2_f16_f32(w & 0x000F000Fu, xh[4 * k], e0, e1);
+          fma2_f16_f32(w & 0x00F000F0u, xh[4 * k + 1], o0, o1);
+          fma2_f16_f32(w8 & 0x000F000Fu, xh[4 * k + 2], e0, e1);
+          fma2_f16_f32(w8 & 0x00F000F0u, xh[4 * k + 3], o0, o1);
         }
-        const float2 fa = f2_unpack(pa), fb = f2_unpack(pb);
-        // sum (u - z) x = sum u x - z sum x, all scaled by 2^-40
-        acc[r] = df * fmaf(-zf, xsum, (fa.x + fb.x) + (fa.y + fb.y));
+        // sum (u - z) x = sum u x - z sum x, all scaled by 2^-24
+        acc[r] = df * fmaf(-zf, xsum, fmaf(o0 + o1, pow2f(-4), e0 + e1));
       }
     }
     // refill the stage with this warp's unit i + S (its reads above are done)
