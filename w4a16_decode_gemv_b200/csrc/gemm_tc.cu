@@ -538,10 +538,14 @@ __global__ void __maxnreg__(96)
 }
 
 // Sums the partial-sum slots of the row blocks no single CTA covered, in CTA
-// order (so y does not depend on timing), and writes y.  Block (rb, cy): the
-// 256 rows of row block rb, tokens 16 cy .. 16 cy + 15.
+// order (so y does not depend on timing), and writes y.  Block (rb, cy) covers
+// the 256 rows of row block rb and tokens 16 cy .. 16 cy + 15; thread (r, j)
+// takes row r and tokens 16 cy + 4 j .. + 3.  A thread issues the loads of up
+// to kFinBatch contributing CTAs before adding any of them, so the slots cost
+// one trip to L2 per batch rather than one per CTA.
+constexpr int kFinBatch = 8;
 template <int MP>
-__global__ void __launch_bounds__(kRows) gemm_tc_finalize(const TcArgs a, int grid_main) {
+__global__ void __launch_bounds__(kRows * 4) gemm_tc_finalize(const TcArgs a, int grid_main) {
   griddep_wait();
   const int rb = blockIdx.x;
   const int base = a.total_units / grid_main;
@@ -549,25 +553,34 @@ __global__ void __launch_bounds__(kRows) gemm_tc_finalize(const TcArgs a, int gr
   const int c0 = owner_cta(rb * a.Kg, base, rem);
   const int c1 = owner_cta(rb * a.Kg + a.Kg - 1, base, rem);
   if (c0 == c1) return;  // one CTA covered the row block and wrote y itself
-  const int r = threadIdx.x;
+  const int r = threadIdx.x, cg = blockIdx.y * 4 + threadIdx.y;
   const int n = rb * kRows + r;
-  if (n >= a.N) return;
-  for (int cg = blockIdx.y * 4; cg < blockIdx.y * 4 + 4 && cg < MP / 4; ++cg) {
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-      const int rbc = (c * base + min(c, rem)) / a.Kg;  // row block where c's range starts
-      const float4 v =
-          __ldcg(a.ws_part + static_cast<size_t>(c * 2 + (rb == rbc ? 0 : 1)) * (kRows * MP / 4) + cg * kRows + r);
-      s0 += v.x;
-      s1 += v.y;
-      s2 += v.z;
-      s3 += v.w;
-    }
-    const float sv[4] = {s0, s1, s2, s3};
+  if (n >= a.N || cg >= MP / 4) return;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  for (int cb = c0; cb <= c1; cb += kFinBatch) {
+    float4 v[kFinBatch];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (cg * 4 + j < a.M) a.y[static_cast<size_t>(cg * 4 + j) * a.N + n] = __float2half_rn(sv[j]);
+    for (int j = 0; j < kFinBatch; ++j) {
+      const int c = cb + j;
+      if (c <= c1) {
+        const int rbc = (c * base + min(c, rem)) / a.Kg;  // row block where c's range starts
+        v[j] = __ldcg(a.ws_part + static_cast<size_t>(c * 2 + (rb == rbc ? 0 : 1)) * (kRows * MP / 4) + cg * kRows + r);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kFinBatch; ++j) {
+      if (cb + j <= c1) {
+        s0 += v[j].x;
+        s1 += v[j].y;
+        s2 += v[j].z;
+        s3 += v[j].w;
+      }
+    }
   }
+  const float sv[4] = {s0, s1, s2, s3};
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (cg * 4 + j < a.M) a.y[static_cast<size_t>(cg * 4 + j) * a.N + n] = __float2half_rn(sv[j]);
 }
 
 int stages_for(int mp) {
@@ -605,7 +618,7 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   const int row_blocks = (a.N + kRows - 1) / kRows;
   cudaLaunchConfig_t fin = {};
   fin.gridDim = dim3(row_blocks, (MP / 4 + 3) / 4);
-  fin.blockDim = dim3(kRows);
+  fin.blockDim = dim3(kRows, 4);
   fin.stream = st;
   fin.attrs = attr;
   fin.numAttrs = pdl_enabled() ? 1 : 0;
