@@ -25,22 +25,25 @@
 // row-block-major and dealt to a persistent grid (one CTA per SM) in contiguous,
 // equal ranges.  A CTA accumulates its units of one row block in two 128 x MP
 // TMEM accumulators (double-buffered, so the next row block's MMAs overlap the
-// epilogue of the last).  A CTA that covers a whole row block writes y directly;
-// otherwise its fp32 partials are added into the workspace (vector reductions in
-// L2) and the last contributor of the row block converts them to fp16 and
-// zeroes the workspace.
+// read-out of the last).  A CTA that covers a whole row block writes y
+// directly; otherwise it writes its fp32 partial tile to one of its two slots
+// in the workspace (the row block its range starts in, and the one it ends
+// in), and gemm_tc_finalize, launched next on the stream, adds the slots of
+// each shared row block in CTA order: y does not depend on timing.
 //
-// Roles (16 warps):
-//   warp 0     one thread issues the tensor copies (TMA) of each unit into a ring
-//              of stages: the 256 x 16-word code tile (64-byte swizzle) and the
-//              two 64-input halves of the x tile (128-byte swizzle, rows past M
-//              zero-filled);
-//   warp 1     allocates TMEM; one thread issues tcgen05.mma (8 per 64-input half)
-//              and tcgen05.commit;
-//   warps 4-7  epilogue: tcgen05.ld of the accumulators, y or workspace;
-//   warps 8-15 dequantization: thread r owns weight row r of the block (warp
-//              8 + 4t + q holds tile t, TMEM lane quarter q) and writes its w_hat
-//              for 64 inputs at a time into one of the TMEM w_hat buffers.
+// Roles (18 warps):
+//   warps 0-15  dequantization and read-out: warp w holds tile t = (w >> 2) & 1
+//               (128 rows), TMEM lane quarter q = w & 3 and part p = w >> 3;
+//               lane i owns weight row t*128 + q*32 + i of the block, converts
+//               words 4p .. 4p + 3 of each 64-input half of a group into w_hat
+//               and writes them into one of the TMEM w_hat buffers; after a
+//               row block's MMAs it reads out its rows' accumulator columns;
+//   warp 16     one thread issues the tensor copies (TMA) of each unit into a
+//               ring of stages: the 256 x 16-word code tile (64-byte swizzle)
+//               and the two 64-input halves of the x tile (128-byte swizzle,
+//               rows past M zero-filled);
+//   warp 17     allocates TMEM; one thread issues tcgen05.mma (8 per 64-input
+//               half) and tcgen05.commit.
 // Dequantization of a code pair: (w >> 4t) & 0x000F000F | 0x64006400 (one LOP3)
 // reads as the fp16 pair 1024 + q; subtracting 1024 + z is exact and the
 // multiply by Delta rounds once (Lecture 13 guide, §TinyChat, slides 36-37;
