@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kAsWarps * 32) act_scale_kernel(const __half* 
 constexpr int kQpThreads = 256;
 constexpr int kQpHalfWarps = kQpThreads / 16;
 constexpr int kQpUnroll = 4;
+constexpr int kQpBlocksPerSm = 3;  // resident CTAs per SM the register budget allows
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
@@ -92,8 +93,13 @@ __device__ __forceinline__ float round_quotient(float w, float d, float inv_d) {
   return w > t ? k + 1.0f : k;  // d > 0
 }
 
+// 1.5 * 2^23: a float in [2^23, 2^24) has unit spacing, so adding this to a
+// value of magnitude below 2^22 rounds it to the nearest integer (ties to
+// even), and subtracting it again gives that integer exactly.
+constexpr float kRoundMagic = 12582912.0f;
+
 template <int BITS, int MODE, bool HAS_S>
-__global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half* __restrict__ W,
+__global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kernel(const __half* __restrict__ W,
                                                                    const __half* __restrict__ s, int N, int K,
                                                                    uint32_t* __restrict__ qweight,
                                                                    __half* __restrict__ scales,
@@ -103,25 +109,40 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half*
   const int Kg = K / kGroup;
   const int Kw = K / 8;
   const long long total = static_cast<long long>(N) * Kg;
-  const int hl = threadIdx.x & 15;
+  const int hl = threadIdx.x & 15, hw = threadIdx.x >> 4;
   const long long stride = static_cast<long long>(gridDim.x) * kQpHalfWarps;
-  long long g0 = static_cast<long long>(blockIdx.x) * kQpHalfWarps + (threadIdx.x >> 4);
+  long long g0 = static_cast<long long>(blockIdx.x) * kQpHalfWarps + hw;
+  // (row, group) of g0 and of the stride, kept in step with g0 without dividing again
+  int n0 = static_cast<int>(g0 / Kg), gi0 = static_cast<int>(g0 - static_cast<long long>(n0) * Kg);
+  const int sn = static_cast<int>(stride / Kg), sr = static_cast<int>(stride - static_cast<long long>(sn) * Kg);
+  auto step = [&](int& n, int& gi) {
+    n += sn;
+    gi += sr;
+    if (gi >= Kg) gi -= Kg, ++n;
+  };
 
-  for (; g0 - (threadIdx.x >> 4) % 2 < total; g0 += stride * kQpUnroll) {
+  // both half-warps of a warp run every iteration (the reductions shuffle over 32 lanes)
+  for (; g0 - (hw & 1) < total; g0 += stride * kQpUnroll) {
+    int nn[kQpUnroll], gg[kQpUnroll];
     uint4 wv[kQpUnroll];
     uint4 sv[kQpUnroll];
 #pragma unroll
     for (int u = 0; u < kQpUnroll; ++u) {
+      nn[u] = u ? nn[u - 1] : n0;
+      gg[u] = u ? gg[u - 1] : gi0;
+      if (u) step(nn[u], gg[u]);
       const long long g = g0 + u * stride;
       wv[u] = make_uint4(0, 0, 0, 0);
       sv[u] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // 1.0
       if (g < total) {
-        const long long n = g / Kg;
-        const int k = static_cast<int>(g - n * Kg) * kGroup + hl * 8;
-        wv[u] = ldg_stream(W + n * K + k);
+        const int k = gg[u] * kGroup + hl * 8;
+        wv[u] = ldg_stream(W + static_cast<size_t>(nn[u]) * K + k);
         if (HAS_S) sv[u] = __ldg(reinterpret_cast<const uint4*>(s + k));
       }
     }
+    n0 = nn[kQpUnroll - 1];
+    gi0 = gg[kQpUnroll - 1];
+    step(n0, gi0);
 #pragma unroll
     for (int u = 0; u < kQpUnroll; ++u) {
       const long long g = g0 + u * stride;
@@ -141,23 +162,34 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half*
       __half d;
       float zf;
       if (MODE == 0) {
-        __half2 hi = __hmax2(__hmax2(w2[0], w2[1]), __hmax2(w2[2], w2[3]));
-        __half2 lo = __hmin2(__hmin2(w2[0], w2[1]), __hmin2(w2[2], w2[3]));
-        // (max, min) of this lane's 8 values in one register
-        __half2 mm = __halves2half2(__hmax(__low2half(hi), __high2half(hi)), __hmin(__low2half(lo), __high2half(lo)));
+        // (max, -min) in one fp16 pair, so one max per level reduces both
+        const __half2 hi = __hmax2(__hmax2(w2[0], w2[1]), __hmax2(w2[2], w2[3]));
+        const __half2 nlo = __hmax2(__hmax2(__hneg2(w2[0]), __hneg2(w2[1])), __hmax2(__hneg2(w2[2]), __hneg2(w2[3])));
+        __half2 mm = __hmax2(__lows2half2(hi, nlo), __highs2half2(hi, nlo));
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) {
-          const __half2 other = as_h2(__shfl_xor_sync(0xffffffffu, as_u32(mm), o));
-          mm = __halves2half2(__hmax(__low2half(mm), __low2half(other)), __hmin(__high2half(mm), __high2half(other)));
+        for (int o = 8; o >= 1; o >>= 1) mm = __hmax2(mm, as_h2(__shfl_xor_sync(0xffffffffu, as_u32(mm), o)));
+        // a3: Delta = fp16((max - min) / (2^N - 1)), the exact quotient rounded
+        // once to fp16; a zero step becomes the unit range.  When max - min is
+        // exact in fp32 (its TwoSum error term is zero), the correctly rounded
+        // fp32 quotient rounded to fp16 is that value: a 24-bit intermediate is
+        // at least 2 p + 2 for the 11-bit fp16 significand, so the double
+        // rounding is innocuous.  Otherwise (exponents of max and min far
+        // apart) the difference and quotient are taken in fp64.
+        const float mx = __low2float(mm), nmn = __high2float(mm);  // nmn = -min
+        const float diff = mx + nmn;
+        const float bv = diff - mx;
+        const float err = (mx - (diff - bv)) + (nmn - bv);
+        if (err == 0.0f) {
+          d = __float2half_rn(__fdiv_rn(diff, static_cast<float>(kQmax)));
+        } else {
+          d = __double2half((static_cast<double>(mx) + static_cast<double>(nmn)) / static_cast<double>(kQmax));
         }
-        // a3: Delta = fp16(fp64(max - min) / (2^N - 1)); zero step -> unit range
-        const double mx = static_cast<double>(__low2float(mm));
-        const double mn = static_cast<double>(__high2float(mm));
-        d = __double2half((mx - mn) / static_cast<double>(kQmax));
-        if (__heq(d, __float2half(0.0f))) d = __double2half(1.0 / static_cast<double>(kQmax));
-        // z = clamp(Round(-min / Delta), 0, 2^N - 1) as a non-negative integer
-        const double zq = rint(-mn / static_cast<double>(__half2float(d)));
-        zf = static_cast<float>(static_cast<int>(fmin(fmax(zq, 0.0), static_cast<double>(kQmax))));
+        if (__heq(d, __float2half(0.0f))) d = __float2half_rn(__fdiv_rn(1.0f, static_cast<float>(kQmax)));
+        // z = clamp(Round(-min / Delta), 0, 2^N - 1) as a non-negative integer;
+        // the rounding decision is exact (round_quotient), and quotients beyond
+        // its range only reach the clamp
+        const float dz = __half2float(d);
+        zf = fminf(fmaxf(round_quotient(nmn, dz, __frcp_rn(dz)), 0.0f), static_cast<float>(kQmax)) + 0.0f;
       } else {
         __half2 a = __hmax2(__hmax2(__habs2(w2[0]), __habs2(w2[1])), __hmax2(__habs2(w2[2]), __habs2(w2[3])));
         __half am = __hmax(__low2half(a), __high2half(a));
@@ -167,29 +199,59 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(const __half*
               static_cast<unsigned short>(__shfl_xor_sync(0xffffffffu, static_cast<unsigned>(__half_as_ushort(am)), o)));
           am = __hmax(am, other);
         }
-        // a3: Delta = fp16(max|w'| / 2^(N-1)), z = 2^(N-1)
-        d = __double2half(static_cast<double>(__half2float(am)) / static_cast<double>(kHalfRange));
-        if (__heq(d, __float2half(0.0f))) d = __double2half(1.0 / static_cast<double>(kHalfRange));
+        // a3: Delta = fp16(max|w'| / 2^(N-1)) (a division by a power of two,
+        // exact in fp32, then one rounding), z = 2^(N-1)
+        d = __float2half_rn(__half2float(am) * (1.0f / static_cast<float>(kHalfRange)));
+        if (__heq(d, __float2half(0.0f))) d = __float2half_rn(1.0f / static_cast<float>(kHalfRange));
         zf = static_cast<float>(kHalfRange);
       }
       if (g >= total) continue;
-      // a4: u = clamp(Round(w' / Delta) + z, 0, 2^N - 1);  a5: pack into layout v1
+      // a4: u = clamp(Round(w' / Delta) + z, 0, 2^N - 1);  a5: pack into layout v1.
+      // Two values at a time (elements 2t, 2t + 1, bound for bits 4t and
+      // 16 + 4t).  q + z = w * inv_d + z is clamped to [-1/4, 2^N - 3/4] (which
+      // changes no clamped code) and rounded to an integer by the magic add.
+      // The product is within 2^-19 of w / d for the quotients that are not
+      // clamped (|w / d| < 2^5), so the integer is the exact Round unless q + z
+      // lies within 2^-16 of a half-integer; then the group is redone with
+      // round_quotient, which decides every case exactly.
       const float df = __half2float(d);
       const float inv_d = __frcp_rn(df);
-      uint32_t word = 0;
+      const uint64_t inv2 = f2_pack(inv_d, inv_d), z2 = f2_pack(zf, zf);
+      const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+      uint64_t u2[4];
+      bool near = false;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 wf = __half22float2(w2[t]);
-        const float u0 = fminf(fmaxf(round_quotient(wf.x, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax));
-        const float u1 = fminf(fmaxf(round_quotient(wf.y, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax));
-        word |= (static_cast<uint32_t>(u0) << (4 * t)) | (static_cast<uint32_t>(u1) << (16 + 4 * t));
+        const float2 qz = f2_unpack(f2_fma(f2_pack(wf.x, wf.y), inv2, z2));
+        const uint64_t c2 = f2_pack(fminf(fmaxf(qz.x, -0.25f), static_cast<float>(kQmax) + 0.25f),
+                                    fminf(fmaxf(qz.y, -0.25f), static_cast<float>(kQmax) + 0.25f));
+        u2[t] = f2_sub(f2_add(c2, magic2), magic2);
+        const float2 off = f2_unpack(f2_sub(c2, u2[t]));
+        near |= fabsf(off.x) >= 0.5f - 0x1p-16f || fabsf(off.y) >= 0.5f - 0x1p-16f;
       }
-      const long long n = g / Kg;
-      const int gi = static_cast<int>(g - n * Kg);
-      qweight[n * Kw + gi * 16 + hl] = word;
+      if (near) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 wf = __half22float2(w2[t]);
+          u2[t] = f2_pack(fminf(fmaxf(round_quotient(wf.x, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)),
+                          fminf(fmaxf(round_quotient(wf.y, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)));
+        }
+      }
+      // the two 16-bit halves of the word summed as integers in floats on a 2^23
+      // base (exact: below 2^16), so their low 16 bits are the packed nibbles
+      uint64_t acc = f2_pack(8388608.0f, 8388608.0f);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float sc = static_cast<float>(1 << (4 * t));
+        acc = f2_fma(u2[t], f2_pack(sc, sc), acc);
+      }
+      const float2 lh = f2_unpack(acc);
+      const uint32_t word = __byte_perm(__float_as_uint(lh.x), __float_as_uint(lh.y), 0x5410);
+      qweight[static_cast<size_t>(nn[u]) * Kw + gg[u] * 16 + hl] = word;
       if (hl == 0) {
-        scales[n * Kg + gi] = d;
-        zeros[n * Kg + gi] = __float2half_rn(zf);
+        scales[static_cast<size_t>(nn[u]) * Kg + gg[u]] = d;
+        zeros[static_cast<size_t>(nn[u]) * Kg + gg[u]] = __float2half_rn(zf);
       }
     }
   }
@@ -201,7 +263,7 @@ cudaError_t launch_qp(const __half* W, const __half* s, int N, int K, uint32_t* 
   const long long groups = static_cast<long long>(N) * (K / kGroup);
   const long long half_warps_needed = (groups + kQpUnroll - 1) / kQpUnroll;
   long long blocks = (half_warps_needed + kQpHalfWarps - 1) / kQpHalfWarps;
-  const long long cap = static_cast<long long>(device_sm_count()) * 8;
+  const long long cap = static_cast<long long>(device_sm_count()) * kQpBlocksPerSm;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   quantize_pack_kernel<BITS, MODE, HAS_S>
