@@ -549,6 +549,9 @@ __global__ void __maxnreg__(96)
 constexpr int kFinBatch = 8;
 template <int MP>
 __global__ void __launch_bounds__(kRows * 4) gemm_tc_finalize(const TcArgs a, int grid_main) {
+  // the next layer's main kernel may start its prologue and weight prefetch; it
+  // reads x (this kernel's y) only after its own griddepcontrol.wait
+  griddep_launch_dependents();
   griddep_wait();
   const int rb = blockIdx.x;
   const int base = a.total_units / grid_main;
