@@ -14,12 +14,13 @@
 // with A = w_hat (fp16) and B = x (fp16, K-major in shared memory), fp32
 // accumulators in tensor memory (TMEM lane = weight row, column = token).
 //
-// w_hat lives in tensor memory, not shared memory: the dequantizing thread of a
-// weight row writes its fp16 pairs straight into that row's TMEM lane
-// (tcgen05.st) and the MMA reads A from there.  Shared memory then only carries
-// the codes and x, so its bandwidth (which a shared-memory A tile of fp16 would
-// exhaust: 4x the bytes of the codes, written once and read once) is not the
-// bound, and four w_hat buffers fit beside the accumulators in the 512 columns.
+// w_hat lives in shared memory, in the K-major 128-byte-swizzled layout of an
+// MMA operand: the dequantizing thread of a weight row writes its fp16 pairs
+// straight into that row's line of a w_hat buffer, and the MMA reads A through
+// a shared-memory descriptor, as it reads x.  Tensor memory then holds only the
+// accumulators.  (An earlier version wrote w_hat into tensor memory with
+// tcgen05.st; on B200 those stores slowed the MMAs' reads of A from tensor
+// memory, and this version is faster at every M.)
 //
 // Work split.  Units are (row block of 256 rows, group of 128 inputs), ordered
 // row-block-major and dealt to a persistent grid (one CTA per SM) in contiguous,
@@ -36,8 +37,9 @@
 //               (128 rows), TMEM lane quarter q = w & 3 and part p = w >> 3;
 //               lane i owns weight row t*128 + q*32 + i of the block, converts
 //               words 4p .. 4p + 3 of each 64-input half of a group into w_hat
-//               and writes them into one of the TMEM w_hat buffers; after a
-//               row block's MMAs it reads out its rows' accumulator columns;
+//               and writes them into one of the shared-memory w_hat buffers;
+//               after a row block's MMAs it reads out its rows' accumulator
+//               columns;
 //   warp 16     one thread issues the tensor copies (TMA) of each unit into a
 //               ring of stages: the 256 x 16-word code tile (64-byte swizzle)
 //               and the two 64-input halves of the x tile (128-byte swizzle,
@@ -95,15 +97,15 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (128 rows x 16 inputs, fp16 pairs in 8
-// columns) is read from tensor memory.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem]^T: A (128 rows x 16 inputs) and B both
+// described by shared-memory matrix descriptors.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                            bool accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
       : "memory");
 }
 
@@ -111,19 +113,6 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t
 struct Word4 {
   uint32_t v[4];
 };
-
-// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (base + i).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const Word4& a, const Word4& b, const Word4& c,
-                                          const Word4& d) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16};" ::"r"(taddr),
-      "r"(a.v[0]), "r"(a.v[1]), "r"(a.v[2]), "r"(a.v[3]), "r"(b.v[0]), "r"(b.v[1]), "r"(b.v[2]), "r"(b.v[3]),
-      "r"(c.v[0]), "r"(c.v[1]), "r"(c.v[2]), "r"(c.v[3]), "r"(d.v[0]), "r"(d.v[1]), "r"(d.v[2]), "r"(d.v[3])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Arrives once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -185,14 +174,6 @@ __device__ __forceinline__ uint32_t lop3_nib(uint32_t w) {
   return r;
 }
 
-// A 16-bit load zero-extended into a 32-bit register, so that nothing reads the
-// destination (and waits for it) until the value is used.
-__device__ __forceinline__ uint32_t ld_nc_u16(const __half* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-
 // W consecutive fp16 values (W = 1, 2, 4 or 8, the address aligned to 2W bytes)
 // into the low halves of w[0..3], lowest address first.
 __device__ __forceinline__ void ld_nc_halves(const __half* p, int W, uint32_t (&w)[4]) {
@@ -211,6 +192,12 @@ __device__ __forceinline__ void ld_nc_halves(const __half* p, int W, uint32_t (&
 __device__ __forceinline__ uint32_t pick_half(const uint32_t (&w)[4], int idx) {
   const uint32_t v = (idx & 4) ? ((idx & 2) ? w[3] : w[2]) : ((idx & 2) ? w[1] : w[0]);
   return (idx & 1) ? (v >> 16) : (v & 0xFFFFu);
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const Word4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.v[0]), "r"(v.v[1]), "r"(v.v[2]),
+               "r"(v.v[3])
+               : "memory");
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -236,13 +223,18 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return p;
 }
 
-// Tensor-memory columns: [0, 4 MP) hold the accumulators (2 buffers x 2 tiles x
-// MP columns); from 4 MP on, as many w_hat buffers of 64 columns as fit (2 tiles
-// x 32 columns, one column = the fp16 pair of inputs 2c, 2c + 1 of one row):
-// 7 for MP = 16 down to 4 for MP = 64.
-constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxABufs = 7;
-__host__ __device__ constexpr int a_bufs(int mp) { return (512 - 4 * mp) / 64; }
+// Tensor memory holds only the accumulators: 2 buffers x 2 tiles x MP columns,
+// allocated as the next power of two of at least 32 columns.
+__host__ __device__ constexpr uint32_t tmem_cols(int mp) {
+  return 4 * mp <= 32 ? 32u : 4 * mp <= 64 ? 64u : 4 * mp <= 128 ? 128u : 256u;
+}
+// w_hat lives in shared memory: kABufs buffers, each one 64-input half of a
+// unit (2 tiles x 128 rows x 128 bytes, K-major with the 128-byte swizzle, the
+// layout the MMA's shared-memory descriptor reads).
+constexpr int kABufs = 4;
+constexpr int kMaxABufs = kABufs;
+constexpr int kTileBytes = 128 * 128;
+constexpr int kABufBytes = 2 * kTileBytes;
 
 // Unit u of the range partition: the CTA whose range holds it.
 __host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
@@ -256,19 +248,19 @@ __global__ void __maxnreg__(96)
   constexpr int kXHalf = MP * 128;                // one 64-input half of the x tile
   constexpr int kStageBytes = kCodeBytes + 2 * kXHalf;
   constexpr uint32_t kIdesc = idesc_f16(MP);
-  constexpr uint32_t kACol0 = 4 * MP;
-  constexpr int kABufs = a_bufs(MP);
-  static_assert(kACol0 + kABufs * 64 <= kTmemCols, "accumulators and w_hat buffers exceed tensor memory");
+  constexpr uint32_t kTmemCols = tmem_cols(MP);
   static_assert(kABufs >= 4, "a unit writes two w_hat buffers; four keep the MMAs one unit behind");
+  static_assert(kStageBytes % 1024 == 0, "w_hat buffers must stay 1024-byte aligned");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
   uint8_t* stages = smem;                        // S x kStageBytes: code tile, then x tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stages + S * kStageBytes);
+  uint8_t* abuf = stages + S * kStageBytes;      // kABufs x kABufBytes of w_hat
+  uint64_t* bars = reinterpret_cast<uint64_t*>(abuf + kABufs * kABufBytes);
   uint64_t* full = bars;                         // [S] codes and x landed
   uint64_t* rempty = bars + kMaxStages;          // [S] codes read and x consumed
-  uint64_t* wfull = bars + 2 * kMaxStages;       // [kABufs] w_hat half written to tensor memory
+  uint64_t* wfull = bars + 2 * kMaxStages;       // [kABufs] w_hat half written to shared memory
   uint64_t* wempty = wfull + kMaxABufs;          // [kABufs] w_hat half consumed by the MMAs
   uint64_t* afull = wempty + kMaxABufs;          // [2] accumulator complete
   uint64_t* aempty = afull + 2;                  // [2] accumulator read out
@@ -373,14 +365,14 @@ __global__ void __maxnreg__(96)
           // shares its scheduler with dequantizing warps, so few instructions
           // per MMA matter.
           const uint64_t bd0 = sw128_desc(xs + h * kXHalf);
-          const uint32_t at0 = tbase + kACol0 + static_cast<uint32_t>(b * 64);
+          const uint64_t ad0 = sw128_desc(abuf + b * kABufBytes);
           const uint32_t d0 = tbase + static_cast<uint32_t>(ab * 2 * MP);
           const bool acc0 = !(first && h == 0);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ts(d0 + t * MP, at0 + t * 32 + kk * 8, bd0 + 2 * kk, kIdesc, kk > 0 || acc0);
+              mma_f16_ss(d0 + t * MP, ad0 + t * (kTileBytes >> 4) + 2 * kk, bd0 + 2 * kk, kIdesc, kk > 0 || acc0);
           any = true;
           mma_commit(&wempty[b]);
           ++hb;
@@ -407,7 +399,11 @@ __global__ void __maxnreg__(96)
     const int t = (warp >> 2) & 1, q = warp & 3, p = warp >> 3;
     const int rloc = t * 128 + q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t acol = tbase + lane_addr + kACol0 + static_cast<uint32_t>(t * 32 + p * 16);
+    // this lane's w_hat row in a buffer: tile t, row q * 32 + lane, 128 bytes
+    // with the 16-byte chunk j at j ^ (row & 7)
+    const int arow = q * 32 + lane;
+    const uint32_t arow0 = smem_u32(abuf) + static_cast<uint32_t>(t * kTileBytes + arow * 128);
+    const uint32_t asw = static_cast<uint32_t>(arow & 7);
     const uint32_t st0 = smem_u32(stages);
     const uint32_t sw_ld = static_cast<uint32_t>((rloc >> 1) & 3);
     // Delta and z come a block of W groups at a time (W = 1, 2, 4 or 8 divides
@@ -504,11 +500,20 @@ __global__ void __maxnreg__(96)
         break;
       }
       tc_fence_after();
-      tmem_st16(acol + static_cast<uint32_t>(b0 * 64), dq_word(c0.x, zz, dd), dq_word(c0.y, zz, dd),
-                dq_word(c0.z, zz, dd), dq_word(c0.w, zz, dd));
-      tmem_st16(acol + static_cast<uint32_t>(b1 * 64), dq_word(c1.x, zz, dd), dq_word(c1.y, zz, dd),
-                dq_word(c1.z, zz, dd), dq_word(c1.w, zz, dd));
-      tmem_wait_st();
+      {
+        const uint32_t r0 = arow0 + static_cast<uint32_t>(b0 * kABufBytes);
+        const uint32_t r1 = arow0 + static_cast<uint32_t>(b1 * kABufBytes);
+        const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
+        const uint32_t cv[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t j = static_cast<uint32_t>(4 * p + i);  // word of the half = 16-byte chunk
+          sts128(r0 + (((j ^ asw) & 7u) << 4), dq_word(cw[i], zz, dd));
+          sts128(r1 + (((j ^ asw) & 7u) << 4), dq_word(cv[i], zz, dd));
+        }
+        // the MMAs read these rows through the async proxy
+        fence_proxy_async_smem();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -591,7 +596,7 @@ __global__ void __launch_bounds__(kRows * 4) gemm_tc_finalize(const TcArgs a, in
 
 int stages_for(int mp) {
   const int stage = kCodeBytes + 2 * mp * 128;
-  int s = (kMaxSmem - 1024 - kCtrlBytes) / stage;
+  int s = (kMaxSmem - 1024 - kCtrlBytes - kABufs * kABufBytes) / stage;
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -600,7 +605,7 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   TcArgs a = a0;
   a.stages = stages_for(MP);
   if (a.stages < 2) return cudaErrorNotSupported;
-  const int smem = 1024 + a.stages * (kCodeBytes + 2 * MP * 128) + kCtrlBytes;
+  const int smem = 1024 + a.stages * (kCodeBytes + 2 * MP * 128) + kABufs * kABufBytes + kCtrlBytes;
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
