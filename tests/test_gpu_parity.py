@@ -135,6 +135,10 @@ def _edge_groups():
     G.append(np.concatenate([[-0.625, 3.125], (np.arange(126) % 15 - 2) * 0.25 + 0.125]))
     G.append(np.concatenate([[-0.75, 3.0], (np.arange(126) % 14 - 3) * 0.25 + 0.125]))
     G.append(np.concatenate([[-2.0, 2.0], np.linspace(-2, 2, 126)]))
+    # max and min so far apart in magnitude that max - min is inexact in fp32
+    # (the step then comes from the fp64 path)
+    G.append(np.concatenate([[1000.0, -2.0 ** -20], rng.standard_normal(126) * 1e-3]))
+    G.append(np.concatenate([[2.0 ** -24, 1000.0], rng.uniform(2.0 ** -24, 1000.0, 126)]))
     return np.stack(G).astype(F16)
 
 
