@@ -71,8 +71,30 @@ def _check(status: int, name: str) -> None:
         raise W4A16Error(f"{name} failed with status {status}: {msg}")
 
 
-def _stream(device: torch.device) -> ctypes.c_void_p:
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+# torch's raw accessors for the current stream and device take a fraction of
+# the time of torch.cuda.current_stream / current_device (which build Python
+# objects); the public calls are the fallback.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_raw_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
+def _stream(device: torch.device) -> int:
+    """The cudaStream_t of the current stream of device, as an integer."""
+    if _raw_stream is not None:
+        return _raw_stream(device.index)
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _current_device() -> int:
+    return _raw_device() if _raw_device is not None else torch.cuda.current_device()
+
+
+def _call_on(device: torch.device, fn, *args) -> int:
+    """Runs fn(*args) with device current (the launches go to its streams)."""
+    if device.index == _current_device():
+        return fn(*args)
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
@@ -80,6 +102,9 @@ def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
 
 
 def _expect(t: torch.Tensor, dtype, shape, name: str) -> None:
+    # one combined test on the common path; the detailed checks name the fault
+    if isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.shape == shape and t.is_contiguous():
+        return
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise W4A16Error(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
@@ -157,7 +182,7 @@ def w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zer
                group: int = GROUP, out: torch.Tensor | None = None,
                workspace: torch.Tensor | None = None) -> torch.Tensor:
     """y fp16 [M, N] = x fp16 [M, K] @ dequant(qweight, scales, zeros)^T."""
-    lib = load_library()
+    lib = _lib if _lib is not None else load_library()
     if x.dim() != 2 or qweight.dim() != 2:
         raise W4A16Error("x must be [M, K] and qweight [N, K/8]")
     M, K = x.shape
@@ -168,13 +193,17 @@ def w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zer
     _expect(zeros, torch.float16, (N, K // group), "zeros")
     y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
     _expect(y, torch.float16, (M, N), "out")
-    need = gemm_workspace_size(M, N, K, group)
-    if need == 0:
-        raise W4A16Error(f"unsupported sizes M={M} N={N} K={K} group={group}")
-    ws = workspace_for(x.device, need) if workspace is None else workspace
-    with torch.cuda.device(x.device):
-        _check(lib.w4a16_gemm(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
-                              _ptr(ws), ws.numel() * ws.element_size(), _stream(x.device)), "w4a16_gemm")
+    if workspace is None:
+        need = gemm_workspace_size(M, N, K, group)
+        if need == 0:
+            raise W4A16Error(f"unsupported sizes M={M} N={N} K={K} group={group}")
+        ws = workspace_for(x.device, need)
+    else:
+        ws = workspace  # the library checks its size and alignment
+    dev = x.device
+    _check(_call_on(dev, lib.w4a16_gemm, x.data_ptr(), qweight.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+                    M, N, K, group, y.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(), _stream(dev)),
+           "w4a16_gemm")
     return y
 
 

@@ -1,5 +1,7 @@
 // C ABI of the w4a16 library: argument checks, error reporting, dispatch.
 // The operations themselves are specified in include/w4a16.h.
+#include <vector>
+#include <mutex>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -53,6 +55,31 @@ int device_sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+cudaError_t ensure_func_attr(const void* func, cudaFuncAttribute attr, int value) {
+  struct Entry {
+    const void* func;
+    int dev;
+    cudaFuncAttribute attr;
+    int value;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& en : done)
+      if (en.func == func && en.dev == dev && en.attr == attr && en.value == value) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(func, attr, value);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    done.push_back({func, dev, attr, value});
+  }
+  return e;
 }
 
 bool pdl_enabled() {

@@ -606,7 +606,8 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   a.stages = stages_for(MP);
   if (a.stages < 2) return cudaErrorNotSupported;
   const int smem = 1024 + a.stages * (kCodeBytes + 2 * MP * 128) + kABufs * kABufBytes + kCtrlBytes;
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_kernel<MP>),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -623,8 +624,8 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   // the partial sums of row blocks shared by several CTAs; asking for the same
   // shared-memory carveout as the main kernel spares the SMs a reconfiguration
   // between the two launches
-  e = cudaFuncSetAttribute(gemm_tc_finalize<MP>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
+  e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_finalize<MP>), cudaFuncAttributePreferredSharedMemoryCarveout,
+                       cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int row_blocks = (a.N + kRows - 1) / kRows;
   cudaLaunchConfig_t fin = {};

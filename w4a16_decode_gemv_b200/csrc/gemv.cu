@@ -363,7 +363,7 @@ int pick_stages(int x_bytes, int unit_bytes) {
 template <typename Kern>
 cudaError_t launch_kernel(Kern kern, const GemvArgs& a, int grid, int threads, int smem, cudaStream_t st,
                           bool pdl = false) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

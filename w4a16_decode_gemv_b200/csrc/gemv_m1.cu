@@ -383,21 +383,44 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   a.stages = stages;
   const int smem = smem_for(warps, stages, a.x_bytes, a.max_units);
 
-  // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256
-  CUtensorMap tmap;
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.Kw), static_cast<cuuint64_t>(p.N)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.Kw) * 4};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kUW), static_cast<cuuint32_t>(kR)};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256.
+  // The map depends only on the pointer and the shape, so the maps of the
+  // last few weights this thread launched on are kept (a decode step visits
+  // the same layers every token) and encoding is skipped for them.
+  struct CachedMap {
+    const uint32_t* ptr;
+    int n, kw;
+    CUtensorMap map;
+  };
+  constexpr int kMapCache = 64;
+  thread_local CachedMap cache[kMapCache] = {};
+  thread_local int cache_next = 0;
+  const CUtensorMap* tmap = nullptr;
+  for (int i = 0; i < kMapCache && !tmap; ++i)
+    if (cache[i].ptr == p.qweight && cache[i].n == p.N && cache[i].kw == a.Kw) tmap = &cache[i].map;
+  if (!tmap) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.Kw), static_cast<cuuint64_t>(p.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.Kw) * 4};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kUW), static_cast<cuuint32_t>(kR)};
+    const cuuint32_t estr[2] = {1, 1};
+    CachedMap& slot = cache[cache_next];
+    if (enc(&slot.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      slot.ptr = nullptr;
+      return cudaErrorInvalidValue;
+    }
+    slot.ptr = p.qweight;
+    slot.n = p.N;
+    slot.kw = a.Kw;
+    tmap = &slot.map;
+    cache_next = (cache_next + 1) % kMapCache;
+  }
 
   auto kern = warps == 16 ? gemv_m1_kernel<16> : gemv_m1_kernel<12>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -409,7 +432,7 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, a, tmap);
+  e = cudaLaunchKernelEx(&cfg, kern, a, *tmap);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -321,7 +321,8 @@ int max_units_for(int N, int K, int& grid) {
 
 template <int MT>
 cudaError_t launch_mt(const MtArgs& a, const CUtensorMap& tmap, int grid, int smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gemv_mt_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gemv_mt_kernel<MT>),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

@@ -20,6 +20,12 @@ void set_last_error(const char* msg);
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();
 
+// cudaFuncSetAttribute(func, attr, value), called once per kernel, device,
+// attribute and value: the attribute lives in the device's context, so later
+// launches need not set it again (it costs a driver call).  Not safe across a
+// cudaDeviceReset of the device, which discards the context's settings.
+cudaError_t ensure_func_attr(const void* func, cudaFuncAttribute attr, int value);
+
 // Whether the GEMV kernels are launched with programmatic dependent launch
 // (on unless the environment variable W4A16_NO_PDL is set to a non-empty value).
 bool pdl_enabled();
