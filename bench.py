@@ -444,6 +444,11 @@ def other_workloads(args, dev):
               "llama7b_decode": [(1, N, K) for _, N, K in inputs.LLAMA7B["layers"]],
               "llama65b_decode": [(1, N, K) for _, N, K in inputs.LLAMA65B["layers"]],
               "skinny_8192": [(M, 8192, 8192) for M in inputs.SKINNY_M]}
+    only = args.only
+    if only is not None:
+        # one workload alone (for profiling): a name, or skinny_8192:M for one M
+        name, _, m = only.partition(":")
+        shapes = {k: [e for e in v if not m or e[0] == int(m)] for k, v in shapes.items() if k == name}
     for name, lst in shapes.items():
         entries = []
         for M, N, K in lst:
@@ -459,6 +464,8 @@ def other_workloads(args, dev):
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries
+    if only is not None and only != "quantize_pack_11008x4096":
+        return res
     # quantize + pack of the 11008 x 4096 AWQ workload (4-bit asym and 3-bit sym)
     W, X, _ = inputs.quant_workload()
     Wd = torch.from_numpy(W).to(dev)
@@ -567,6 +574,9 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--skip-extras", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="run one of the other workloads only (gemv_4096x4096, llama7b_decode, llama65b_decode, "
+                         "skinny_8192 or skinny_8192:M, quantize_pack_11008x4096); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
