@@ -166,6 +166,20 @@ W4A16_API w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const 
 W4A16_API w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream);
 
 /*
+ * w4a16_wait_timeout_selftest -- diagnostics for the bounded waits behind
+ * W4A16_ERR_DEVICE.  Launches one small kernel on `stream` that waits on a
+ * shared-memory barrier nothing will ever complete, gives up after
+ * `limit_us` microseconds (1 .. 1000000), and records the timeout in the
+ * workspace's status word exactly as the GEMM kernels do.  A following
+ * w4a16_gemm_check on the same workspace then returns W4A16_ERR_DEVICE.
+ * Nothing faults or hangs: the wait is bounded by the device clock.
+ *   workspace  at least 16 bytes, 16-byte aligned (a w4a16_gemm workspace).
+ * Returns W4A16_ERR_ARG for a null workspace or a limit out of range,
+ * W4A16_ERR_CUDA if the launch fails.
+ */
+W4A16_API w4a16_status w4a16_wait_timeout_selftest(void* workspace, int limit_us, w4a16_stream_t stream);
+
+/*
  * w4a16_gemv_noalloc -- the split-K CUDA-core GEMV of w4a16_gemm (1 <= M <= 4)
  * for callers that cannot allocate device memory: inference servers that
  * reserve every buffer at start-up, plug-ins handed only the tensors they work

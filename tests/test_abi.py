@@ -107,6 +107,16 @@ def test_gemm_check_validation(lib):
     assert lib.w4a16_gemm_check(None, None) == ERR_ARG
 
 
+def test_wait_timeout_selftest_validation(lib):
+    """Argument checks happen before any launch (no GPU needed)."""
+    assert lib.w4a16_wait_timeout_selftest(None, 1000, None) == ERR_ARG
+    buf = ctypes.create_string_buffer(64)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    assert lib.w4a16_wait_timeout_selftest(ctypes.c_void_p(addr + 4), 1000, None) == ERR_ARG  # misaligned
+    assert lib.w4a16_wait_timeout_selftest(ctypes.c_void_p(addr), 0, None) == ERR_ARG
+    assert lib.w4a16_wait_timeout_selftest(ctypes.c_void_p(addr), 1000001, None) == ERR_ARG
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(w4.W4A16Error):

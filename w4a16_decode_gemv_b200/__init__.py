@@ -55,6 +55,8 @@ def load_library():
     lib.w4a16_gemv_noalloc_max_scratch.restype = sz
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
+    lib.w4a16_wait_timeout_selftest.argtypes = [vp, i, vp]
+    lib.w4a16_wait_timeout_selftest.restype = i
     lib.w4a16_last_error.argtypes = []
     lib.w4a16_last_error.restype = ctypes.c_char_p
     lib.w4a16_layout_version.argtypes = []
@@ -227,6 +229,17 @@ def w4a16_gemv_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Ten
         _check(lib.w4a16_gemv_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
                                       _stream(x.device)), "w4a16_gemv_noalloc")
     return y
+
+
+def wait_timeout_selftest(workspace: torch.Tensor, limit_us: int = 1000) -> None:
+    """Launches a kernel whose bounded barrier wait runs out after limit_us and
+    records the timeout in workspace's status word (see gemm_check)."""
+    lib = load_library()
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise W4A16Error("workspace must be a CUDA tensor")
+    with torch.cuda.device(workspace.device):
+        _check(lib.w4a16_wait_timeout_selftest(_ptr(workspace), limit_us, _stream(workspace.device)),
+               "w4a16_wait_timeout_selftest")
 
 
 def gemm_check(workspace: torch.Tensor) -> None:

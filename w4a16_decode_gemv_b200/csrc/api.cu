@@ -197,6 +197,18 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   return ok();
 }
 
+w4a16_status w4a16_wait_timeout_selftest(void* workspace, int limit_us, w4a16_stream_t stream) {
+  if (!workspace || !aligned16(workspace))
+    return fail(W4A16_ERR_ARG, "w4a16_wait_timeout_selftest: workspace must be non-null and 16-byte aligned");
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(W4A16_ERR_ARG, "w4a16_wait_timeout_selftest: limit_us=%d (1 .. 1000000)", limit_us);
+  const cudaError_t e = launch_wait_timeout_probe(static_cast<uint32_t*>(workspace),
+                                                  static_cast<uint64_t>(limit_us) * 1000ull,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_wait_timeout_selftest launch");
+  return ok();
+}
+
 w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream) {
   if (!workspace) return fail(W4A16_ERR_ARG, "w4a16_gemm_check: null workspace");
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -76,6 +76,9 @@ cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t 
 // partial-sum slots on the current device.
 size_t tc_partial_bytes(int M);
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+// One CTA waits on a shared-memory barrier that nothing completes, gives up
+// after limit_ns and sets kDevWaitTimeout in *status (the GEMM kernels' path).
+cudaError_t launch_wait_timeout_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
