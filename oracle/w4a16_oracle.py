@@ -49,6 +49,11 @@ Readings of points the pages leave open:
 8. Packed layout v1 (our own design, stated in include/w4a16.h): qweight is
    u32[N, K/8]; word (n, j) holds k = 8j + i, i = 0..7; nibble slot p (bits
    4p..4p+3) holds i = [0, 2, 4, 6, 1, 3, 5, 7][p].
+9. Search objective ([L13] slide 28): the norm is not named; the loss is the
+   mean squared output error, which has the same minimiser as the Frobenius
+   norm.  The divided activation is rounded to fp16 once, x' = fp16(x / s); the
+   quantized output is taken as the W4A16 GEMM delivers it, rounded to fp16;
+   the target W X is exact.  The grid of alphas is the caller's.
 
 Every function here is pinned by tests marked ``not gpu`` against closed
 forms, brute force, invariants the pages state, or special cases.
@@ -212,3 +217,36 @@ def gemm_rows(x, qweight, scales, zeros, rows, group: int = 128):
     rows = np.asarray(rows)
     w_hat = dequant(qweight[rows], scales[rows], zeros[rows], group)
     return gemm_ref(x, w_hat)
+
+
+# ---------------------------------------------------------------------------
+# search for the scaling strength  ([L13] slide 28; [YT]: a small grid search
+# on calibration data picks it)
+# ---------------------------------------------------------------------------
+def divide_activation(X: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """x'[t, k] = fp16(X[t, k] / s[k]): the activation that meets the scaled
+    weight, the 1/s folded into the previous op ([ML11] §11.3, [L13] slide 27)."""
+    X = np.asarray(X, dtype=F16).astype(F64)
+    return (X / np.asarray(s, dtype=F16).astype(F64)[None, :]).astype(F16)
+
+
+def awq_loss(W: np.ndarray, X: np.ndarray, alpha: float, group: int = 128, bits: int = 4, mode: int = ASYM) -> float:
+    """L(alpha) = mean over outputs of (Q(W s)(s^-1 X) - W X)^2 with s = s_X^alpha
+    ([L13] slide 28), for weights W[N, K] and calibration tokens X[T, K].
+
+    Q(W s)(s^-1 X) is the W4A16 product of the divided activation with the
+    packed, scaled weight, rounded to fp16 (reading 9); W X is exact.
+    """
+    s = act_scale(X, alpha)
+    q, sc, z = quantize_pack(W, s, group, bits, mode)
+    w_hat = dequant(q, sc, z, group)
+    y_q = (divide_activation(X, s).astype(F64) @ w_hat.T).astype(F16).astype(F64)
+    y = np.asarray(X, dtype=F16).astype(F64) @ np.asarray(W, dtype=F16).astype(F64).T
+    return float(np.mean((y_q - y) ** 2))
+
+
+def awq_search(W: np.ndarray, X: np.ndarray, alphas, group: int = 128, bits: int = 4, mode: int = ASYM):
+    """alpha* = argmin over the grid of L(alpha) ([L13] slide 28): (losses, index of the minimum)."""
+    losses = [awq_loss(W, X, float(a), group, bits, mode) for a in alphas]
+    return losses, int(np.argmin(losses))
+
