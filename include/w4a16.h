@@ -157,6 +157,53 @@ W4A16_API w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const 
                         void* workspace, size_t workspace_bytes, w4a16_stream_t stream);
 
 /*
+ * awq_search_workspace_size -- bytes of workspace that awq_search_alpha needs
+ * on the current device for these sizes; 0 for invalid sizes.
+ */
+W4A16_API size_t awq_search_workspace_size(int N, int K, int T, int n_alpha, int group);
+
+/*
+ * awq_search_alpha -- the AWQ scaling-strength search over a caller's grid.
+ *
+ *   for each alpha = alphas[a]:
+ *     s          = awq_act_scale(X, alpha)                   (fp16 [K])
+ *     qweight, scales, zeros = awq_quantize_pack(W, s, group, bits, mode)
+ *     x'         = fp16(X / s)                               (per element, one rounding)
+ *     y_q        = w4a16_gemm(x', qweight, scales, zeros)    (fp16 [T][N], chunks of <= 64 tokens)
+ *     losses[a]  = mean over the T x N outputs of (y_q - y)^2,   y = X W^T
+ *   *best = the first a with the smallest loss
+ *
+ * The objective is the AWQ one: the error of the layer's output with the
+ * scaled, quantized weight and the divided activation against the unquantized
+ * output, minimised over alpha by a grid search on calibration tokens
+ * ("MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading guide, §AWQ,
+ * slide 28; "Learning-ML-DL ch. 11", §11.4).  Every step for an alpha is the
+ * library's own entry point above, so the codes of the chosen alpha are the
+ * ones awq_quantize_pack produces for it.  y is formed once, in fp32 on the
+ * CUDA cores, from the exact fp16 products; each loss is an fp64 sum in a fixed
+ * order, so the losses repeat exactly from call to call whenever the GEMM
+ * outputs do (always when every chunk has 5 or more tokens; a chunk of 1 to 4
+ * tokens on the split-K GEMV may differ in the last bit of y).
+ *
+ *   W        fp16 [N][K], device.    X  fp16 [T][K] calibration tokens, device.
+ *   alphas   double [n_alpha], host, finite (the pages search [0, 1]).
+ *   losses   double [n_alpha], host (output).   best  int, host (output), or NULL.
+ *   N >= 1;  1 <= T <= 2^20;  K a multiple of group;  group == 128;  bits in {3, 4};
+ *   1 <= n_alpha <= 4096;  N*K, T*K and T*N below 2^31.
+ *   workspace  device memory of at least awq_search_workspace_size(N, K, T,
+ *              n_alpha, group) bytes, 16-byte aligned, any contents; it is
+ *              scratch (the call zero-fills what needs it).
+ * Unlike the other calls this one is synchronous: it enqueues the work on
+ * `stream`, waits for it and returns the losses.  W * s must stay finite in
+ * fp16 for every alpha of the grid (see awq_quantize_pack).  Returns
+ * W4A16_ERR_DEVICE if a GEMM kernel gave up waiting (losses then unspecified).
+ */
+W4A16_API w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T,
+                                        const double* alphas, int n_alpha, int group, int bits,
+                                        w4a16_mode mode, double* losses, int* best, void* workspace,
+                                        size_t workspace_bytes, w4a16_stream_t stream);
+
+/*
  * w4a16_gemm_check -- synchronizes `stream` and reads the workspace's device
  * status word.  Returns W4A16_ERR_DEVICE if any earlier w4a16_gemm with this
  * workspace gave up waiting for its weight tiles (bounded waits, about 2 s),

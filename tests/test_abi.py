@@ -124,3 +124,54 @@ def test_python_binding_rejects_cpu_tensors():
     with pytest.raises(w4.W4A16Error):
         w4.w4a16_gemm(torch.zeros((1, 128), dtype=torch.float16), torch.zeros((8, 16), dtype=torch.int32),
                       torch.zeros((8, 1), dtype=torch.float16), torch.zeros((8, 1), dtype=torch.float16))
+
+
+def test_search_workspace_size(lib):
+    ws = lib.awq_search_workspace_size
+    n = ws(11008, 4096, 512, 20, 128)
+    # at least the packed weight, the divided tokens, the fp16 and fp32 outputs
+    assert n >= 11008 * 4096 // 2 + 512 * 4096 * 2 + 512 * 11008 * (2 + 4)
+    assert ws(256, 1024, 100, 11, 128) > 0
+    assert ws(0, 1024, 100, 11, 128) == 0
+    assert ws(256, 1000, 100, 11, 128) == 0
+    assert ws(256, 1024, 0, 11, 128) == 0
+    assert ws(256, 1024, 100, 0, 128) == 0
+    assert ws(256, 1024, 100, 4097, 128) == 0
+    assert ws(256, 1024, 100, 11, 64) == 0
+    assert ws(1 << 20, 1 << 12, 1, 1, 128) == 0
+    assert ws(1, 128, (1 << 20) + 1, 1, 128) == 0
+
+
+def test_search_validation(lib):
+    """Every rejection happens before anything is enqueued (no GPU needed)."""
+    f = lib.awq_search_alpha
+    grid = (ctypes.c_double * 3)(0.0, 0.5, 1.0)
+    bad = (ctypes.c_double * 3)(0.0, float("nan"), 1.0)
+    losses = (ctypes.c_double * 3)()
+    best = ctypes.c_int(-1)
+    need = lib.awq_search_workspace_size(64, 256, 10, 3, 128)
+
+    def call(W=A, X=A, N=64, K=256, T=10, alphas=grid, n=3, group=128, bits=4, mode=0, out=losses, ws=B,
+             nbytes=need):
+        return f(W, X, N, K, T, alphas, n, group, bits, mode, out, ctypes.byref(best), ws, nbytes, None)
+
+    assert call(W=None) == ERR_ARG
+    assert call(alphas=None) == ERR_ARG
+    assert call(out=None) == ERR_ARG
+    assert call(ws=None) == ERR_ARG
+    assert call(T=0) == ERR_ARG
+    assert call(T=(1 << 20) + 1, K=128) == ERR_SHAPE
+    assert call(n=0) == ERR_ARG
+    assert call(n=5000) == ERR_ARG
+    assert call(alphas=bad) == ERR_ARG
+    assert "alphas[1]" in _err(lib)
+    assert call(mode=3) == ERR_ARG
+    assert call(group=64) == ERR_UNSUPPORTED
+    assert call(bits=8) == ERR_UNSUPPORTED
+    assert call(K=200) == ERR_SHAPE
+    assert call(N=1 << 20, K=1 << 12) == ERR_SHAPE
+    assert call(X=MIS) == ERR_ALIGN
+    assert call(ws=MIS) == ERR_ALIGN
+    assert call(nbytes=need - 1) == ERR_WORKSPACE
+    assert "workspace" in _err(lib)
+    assert best.value == -1

@@ -53,6 +53,10 @@ def load_library():
     lib.w4a16_gemv_noalloc.restype = i
     lib.w4a16_gemv_noalloc_max_scratch.argtypes = []
     lib.w4a16_gemv_noalloc_max_scratch.restype = sz
+    lib.awq_search_workspace_size.argtypes = [i, i, i, i, i]
+    lib.awq_search_workspace_size.restype = sz
+    lib.awq_search_alpha.argtypes = [vp, vp, i, i, i, vp, i, i, i, i, vp, vp, vp, sz, vp]
+    lib.awq_search_alpha.restype = i
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
     lib.w4a16_wait_timeout_selftest.argtypes = [vp, i, vp]
@@ -229,6 +233,48 @@ def w4a16_gemv_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Ten
         _check(lib.w4a16_gemv_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
                                       _stream(x.device)), "w4a16_gemv_noalloc")
     return y
+
+
+def search_workspace_size(N: int, K: int, T: int, n_alpha: int, group: int = GROUP) -> int:
+    return int(load_library().awq_search_workspace_size(N, K, T, n_alpha, group))
+
+
+def awq_search_alpha(W: torch.Tensor, X: torch.Tensor, alphas, group: int = GROUP, bits: int = 4,
+                     mode: int = ASYM, workspace: torch.Tensor | None = None):
+    """The AWQ alpha grid search for weights W fp16 [N, K] on calibration tokens X fp16 [T, K].
+
+    Returns (losses, best): the mean squared error of the W4A16 output against
+    X W^T for every alpha of the grid, and the index of the smallest.  The call
+    waits for the GPU.  ``workspace`` (uint8, any contents) may be given to
+    avoid the allocation of search_workspace_size bytes.
+    """
+    lib = load_library()
+    if W.dim() != 2 or X.dim() != 2:
+        raise W4A16Error("W must be [N, K] and X [T, K]")
+    N, K = W.shape
+    T = X.shape[0]
+    _expect(W, torch.float16, (N, K), "W")
+    _expect(X, torch.float16, (T, K), "X")
+    if X.device != W.device:
+        raise W4A16Error("W and X must be on the same device")
+    grid = [float(a) for a in alphas]
+    n = len(grid)
+    if workspace is None:
+        need = search_workspace_size(N, K, T, n, group)
+        if need == 0:
+            raise W4A16Error(f"unsupported sizes N={N} K={K} T={T} n_alpha={n} group={group}")
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    elif not isinstance(workspace, torch.Tensor) or workspace.device != W.device:
+        raise W4A16Error("workspace must be a tensor on W's device")
+    a_buf = (ctypes.c_double * max(n, 1))(*grid)
+    losses = (ctypes.c_double * max(n, 1))()
+    best = ctypes.c_int(-1)
+    with torch.cuda.device(W.device):
+        _check(lib.awq_search_alpha(_ptr(W), _ptr(X), N, K, T, a_buf, n, group, bits, mode, losses,
+                                    ctypes.byref(best), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(W.device)),
+               "awq_search_alpha")
+    return [losses[i] for i in range(n)], best.value
 
 
 def wait_timeout_selftest(workspace: torch.Tensor, limit_us: int = 1000) -> None:

@@ -119,6 +119,56 @@ Workspace carve_workspace(void* base, int M, int N, int K) {
   return w;
 }
 
+// The kernel w4a16_gemm runs for an M x N x K problem: M = 1 on whole rows when
+// the activation fits the kernel's staging, M = 2..4 on whole rows or split-K,
+// M = 5..64 on the tensor cores.
+cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
+  if (p.M == 1 && gemv_m1_supports(p.N, p.K)) return launch_gemv_m1(p, ws.status, st);
+  if (gemv_mt_supports(p.M, p.N, p.K)) return launch_gemv_mt(p, ws.status, st);
+  if (p.M <= kMaxGemvM && gemv_supports(p.M, p.K)) return launch_gemv(p, ws, st);
+  return launch_gemm_tc(p, ws, st);
+}
+
+// Workspace of awq_search_alpha: every region starts on a 256-byte boundary.
+// The quantized outputs are kept per GEMM chunk of up to kMaxM tokens, each
+// chunk's [rows][N] block starting on a 16-byte boundary as w4a16_gemm needs.
+struct SearchLayout {
+  int chunk_rows;            // tokens per GEMM chunk: min(T, kMaxM)
+  long long chunk_stride;    // elements between chunks of yq
+  size_t gemm, qweight, scales, zeros, s, xd, yq, yref, partial, sums, total;
+};
+
+static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+static SearchLayout search_layout(int N, int K, int T, int n_alpha) {
+  SearchLayout L;
+  L.chunk_rows = T < kMaxM ? T : kMaxM;
+  L.chunk_stride = (static_cast<long long>(L.chunk_rows) * N + 7) / 8 * 8;
+  const size_t chunks = (static_cast<size_t>(T) + L.chunk_rows - 1) / L.chunk_rows;
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  const size_t groups = static_cast<size_t>(N) * (K / kGroup);
+  L.gemm = take(workspace_bytes(L.chunk_rows, N, K));
+  L.qweight = take(static_cast<size_t>(N) * (K / 8) * 4);
+  L.scales = take(groups * 2);
+  L.zeros = take(groups * 2);
+  L.s = take(static_cast<size_t>(K) * 2);
+  L.xd = take(static_cast<size_t>(T) * K * 2);
+  L.yq = take(chunks * static_cast<size_t>(L.chunk_stride) * 2);
+  L.yref = take(static_cast<size_t>(T) * N * 4);
+  L.partial = take(static_cast<size_t>(n_alpha) * search_error_blocks() * 8);
+  L.sums = take(static_cast<size_t>(n_alpha) * 8);
+  L.total = off;
+  return L;
+}
+
+constexpr int kMaxAlphas = 4096;
+constexpr int kMaxSearchTokens = 1 << 20;  // the target GEMM's grid holds T / 64 in its y dimension
+
 }  // namespace w4a16
 
 using namespace w4a16;
@@ -180,20 +230,100 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   if (!aligned16(workspace)) return fail(W4A16_ERR_ALIGN, "w4a16_gemm: workspace must be 16-byte aligned");
   GemmProblem p{static_cast<const __half*>(x), qweight, static_cast<const __half*>(scales),
                 static_cast<const __half*>(zeros), static_cast<__half*>(y), M, N, K};
-  const Workspace ws = carve_workspace(workspace, M, N, K);
-  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (M == 1 && gemv_m1_supports(N, K)) {
-    e = launch_gemv_m1(p, ws.status, st);
-  } else if (gemv_mt_supports(M, N, K)) {
-    e = launch_gemv_mt(p, ws.status, st);
-  } else if (M <= kMaxGemvM && gemv_supports(M, K)) {
-    e = launch_gemv(p, ws, st);
-  } else {
-    e = launch_gemm_tc(p, ws, st);
-  }
+  const cudaError_t e = dispatch_gemm(p, carve_workspace(workspace, M, N, K), reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: M=%d K=%d not supported yet", M, K);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm launch");
+  return ok();
+}
+
+size_t awq_search_workspace_size(int N, int K, int T, int n_alpha, int group) {
+  if (N < 1 || K < 1 || T < 1 || T > kMaxSearchTokens || n_alpha < 1 || n_alpha > kMaxAlphas || group != kGroup ||
+      K % group)
+    return 0;
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(T) * K >= kMaxElems ||
+      static_cast<long long>(T) * N >= kMaxElems)
+    return 0;
+  return search_layout(N, K, T, n_alpha).total;
+}
+
+w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T, const double* alphas, int n_alpha,
+                              int group, int bits, w4a16_mode mode, double* losses, int* best, void* workspace,
+                              size_t workspace_bytes_, w4a16_stream_t stream) {
+  if (!W || !X || !alphas || !losses || !workspace) return fail(W4A16_ERR_ARG, "awq_search_alpha: null pointer");
+  if (N < 1 || K < 1 || T < 1) return fail(W4A16_ERR_ARG, "awq_search_alpha: N=%d K=%d T=%d must be >= 1", N, K, T);
+  if (T > kMaxSearchTokens) return fail(W4A16_ERR_SHAPE, "awq_search_alpha: T=%d (at most %d)", T, kMaxSearchTokens);
+  if (n_alpha < 1 || n_alpha > kMaxAlphas)
+    return fail(W4A16_ERR_ARG, "awq_search_alpha: n_alpha=%d (1 .. %d)", n_alpha, kMaxAlphas);
+  for (int a = 0; a < n_alpha; ++a)
+    if (!std::isfinite(alphas[a])) return fail(W4A16_ERR_ARG, "awq_search_alpha: alphas[%d] is not finite", a);
+  if (mode != W4A16_ASYM && mode != W4A16_SYM) return fail(W4A16_ERR_ARG, "awq_search_alpha: bad mode %d", mode);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "awq_search_alpha: group=%d (only 128)", group);
+  if (bits != 3 && bits != 4) return fail(W4A16_ERR_UNSUPPORTED, "awq_search_alpha: bits=%d (3 or 4)", bits);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "awq_search_alpha: K=%d not a multiple of group=%d", K, group);
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(T) * K >= kMaxElems ||
+      static_cast<long long>(T) * N >= kMaxElems)
+    return fail(W4A16_ERR_SHAPE, "awq_search_alpha: N*K, T*K or T*N too large");
+  if (!aligned16(W) || !aligned16(X) || !aligned16(workspace))
+    return fail(W4A16_ERR_ALIGN, "awq_search_alpha: W, X and workspace must be 16-byte aligned");
+  const SearchLayout L = search_layout(N, K, T, n_alpha);
+  if (workspace_bytes_ < L.total)
+    return fail(W4A16_ERR_WORKSPACE, "awq_search_alpha: workspace of %zu bytes needed, %zu given", L.total,
+                workspace_bytes_);
+
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const __half* Wh = static_cast<const __half*>(W);
+  const __half* Xh = static_cast<const __half*>(X);
+  uint32_t* qweight = reinterpret_cast<uint32_t*>(base + L.qweight);
+  __half* scales = reinterpret_cast<__half*>(base + L.scales);
+  __half* zeros = reinterpret_cast<__half*>(base + L.zeros);
+  __half* s = reinterpret_cast<__half*>(base + L.s);
+  __half* xd = reinterpret_cast<__half*>(base + L.xd);
+  __half* yq = reinterpret_cast<__half*>(base + L.yq);
+  float* yref = reinterpret_cast<float*>(base + L.yref);
+  double* partial = reinterpret_cast<double*>(base + L.partial);
+  double* sums = reinterpret_cast<double*>(base + L.sums);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int blocks = search_error_blocks();
+
+  // The GEMM workspace must start zeroed; its status word doubles as the search's.
+  cudaError_t e = cudaMemsetAsync(base + L.gemm, 0, workspace_bytes(L.chunk_rows, N, K), st);
+  if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: clear workspace");
+  e = launch_reference_gemm(Xh, Wh, T, N, K, yref, st);
+  if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: reference product");
+  for (int a = 0; a < n_alpha && e == cudaSuccess; ++a) {
+    e = launch_act_scale(Xh, T, K, alphas[a], s, st);
+    if (e == cudaSuccess)
+      e = launch_quantize_pack(Wh, s, N, K, bits, static_cast<int>(mode), qweight, scales, zeros, st);
+    if (e == cudaSuccess) e = launch_divide_activation(Xh, s, T, K, xd, st);
+    for (int t0 = 0, c = 0; t0 < T && e == cudaSuccess; t0 += L.chunk_rows, ++c) {
+      const int m = T - t0 < L.chunk_rows ? T - t0 : L.chunk_rows;
+      const GemmProblem p{xd + static_cast<size_t>(t0) * K, qweight, scales, zeros, yq + c * L.chunk_stride,
+                          m, N, K};
+      e = dispatch_gemm(p, carve_workspace(base + L.gemm, m, N, K), st);
+    }
+    if (e == cudaSuccess)
+      e = launch_squared_error(yq, yref, T, N, L.chunk_rows, L.chunk_stride,
+                               partial + static_cast<size_t>(a) * blocks, st);
+  }
+  if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "awq_search_alpha: K=%d not supported", K);
+  if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha launch");
+  e = launch_sum_partials(partial, n_alpha, sums, st);
+  if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: loss sums");
+  uint32_t flag = 0;
+  e = cudaMemcpyAsync(losses, sums, static_cast<size_t>(n_alpha) * 8, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, base + L.gemm, sizeof(flag), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: read losses");
+  if (flag != kDevOk)
+    return fail(W4A16_ERR_DEVICE, "awq_search_alpha: a GEMM kernel gave up waiting for its weight tiles (status %u)",
+                flag);
+  const double count = static_cast<double>(T) * N;
+  int arg = 0;
+  for (int a = 0; a < n_alpha; ++a) {
+    losses[a] /= count;
+    if (losses[a] < losses[arg]) arg = a;
+  }
+  if (best) *best = arg;
   return ok();
 }
 

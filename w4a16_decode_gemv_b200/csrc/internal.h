@@ -80,6 +80,21 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
 // after limit_ns and sets kDevWaitTimeout in *status (the GEMM kernels' path).
 cudaError_t launch_wait_timeout_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
+// The kernel w4a16_gemm dispatches to for p (api.cu).
+cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+
+// Kernels of the AWQ alpha search (awq_search.cu).  Y = X W^T in fp32 (X [T][K],
+// W [N][K] fp16); Xd = fp16(X / s); per-block fp64 partial sums of (Yq - Y)^2,
+// search_error_blocks() of them, with Yq in GEMM-sized chunks of chunk_rows
+// tokens at chunk_stride elements apart; sums[a] = the n_alpha groups of
+// partials added in block order.
+int search_error_blocks();
+cudaError_t launch_reference_gemm(const __half* X, const __half* W, int T, int N, int K, float* Y, cudaStream_t st);
+cudaError_t launch_divide_activation(const __half* X, const __half* s, int T, int K, __half* Xd, cudaStream_t st);
+cudaError_t launch_squared_error(const __half* Yq, const float* Y, int T, int N, int chunk_rows, long long chunk_stride,
+                                 double* partial, cudaStream_t st);
+cudaError_t launch_sum_partials(const double* partial, int n_alpha, double* sums, cudaStream_t st);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
