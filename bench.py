@@ -209,6 +209,44 @@ def profiled_traffic(kernel_key):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def search_workload(Wd, Xd, dev, n_alpha=20, reps=3):
+    """The alpha grid search of the 11008 x 4096 layer on its 512 calibration tokens.
+
+    A search of 1 and of n_alpha grid points is timed with CUDA events (the
+    call is synchronous); their difference gives the time per grid point, the
+    rest is the target product W X and the set-up, done once per search.
+    """
+    import torch
+
+    import w4a16_decode_gemv_b200 as w4
+    N, K = Wd.shape
+    T = Xd.shape[0]
+    grid = [i / (n_alpha - 1) for i in range(n_alpha)]
+    ws = torch.empty(w4.search_workspace_size(N, K, T, n_alpha), dtype=torch.uint8, device=dev)
+
+    def timed(alphas):
+        best_ms, out = None, None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            out = w4.awq_search_alpha(Wd, Xd, alphas, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best_ms = ms if best_ms is None else min(best_ms, ms)
+        return best_ms, out
+
+    timed(grid[:1])  # warm-up (library load, first launches)
+    ms1, _ = timed(grid[:1])
+    msn, (losses, best) = timed(grid)
+    per = (msn - ms1) / (n_alpha - 1)
+    return {"N": N, "K": K, "T": T, "n_alpha": n_alpha, "ms_per_search": round(msn, 3),
+            "ms_per_alpha": round(per, 4), "ms_once_per_search": round(ms1 - per, 3),
+            "best_alpha": round(grid[best], 4), "losses_min_max": [min(losses), max(losses)],
+            "timing": f"CUDA events around the synchronous call, best of {reps}"}
+
+
 def run_ours(args, dist):
     import torch
 
@@ -440,10 +478,24 @@ def other_workloads(args, dev):
         w4.gemm_check(ws_)
         return ms * 1e3 / c
 
+    def cublas_us(M, N, K):
+        # the dense fp16 product the W4A16 path replaces (torch.matmul -> cuBLAS), for the crossover
+        Ws = [torch.randn((N, K), device=dev, generator=gen).half() for _ in range(2)]
+        x = torch.randn((M, K), device=dev, generator=gen).half()
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+
+        def fn():
+            for Wf in Ws:
+                torch.matmul(x, Wf.t(), out=y)
+        ms = time_graph(fn, reps=20)
+        del Ws
+        return ms * 1e3 / 2
+
     shapes = {"gemv_4096x4096": [(1, 4096, 4096)],
               "llama7b_decode": [(1, N, K) for _, N, K in inputs.LLAMA7B["layers"]],
               "llama65b_decode": [(1, N, K) for _, N, K in inputs.LLAMA65B["layers"]],
-              "skinny_8192": [(M, 8192, 8192) for M in inputs.SKINNY_M]}
+              "skinny_8192": [(M, 8192, 8192) for M in inputs.SKINNY_M],
+              "prefill_8192": [(M, 8192, 8192) for M in (128, 200, 512)]}
     only = args.only
     if only is not None:
         # one workload alone (for profiling): a name, or skinny_8192:M for one M
@@ -458,18 +510,25 @@ def other_workloads(args, dev):
                 e = {"M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(b / us / 1e3, 1),
                      "hbm_frac": round(b / us / 1e3 / hbm_peak, 4), "tflops": round(2 * M * N * K / us / 1e6, 2)}
                 if M > 4:
-                    e["path"] = "tcgen05 tensor cores"
+                    e["path"] = "tcgen05 tensor cores" + (f", {-(-M // 128)} chunks of <= 128 tokens" if M > 128 else "")
                     e["tensor_frac"] = round(2 * M * N * K / us / 1e6 / tc_peak, 4)
+                if M >= 16:
+                    e["cublas_fp16_us"] = round(cublas_us(M, N, K), 3)
                 entries.append(e)
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries
+    if only is not None and only not in ("quantize_pack_11008x4096", "awq_search_11008x4096"):
+        return res
+    W, X, _ = inputs.quant_workload()
+    Wd = torch.from_numpy(W).to(dev)
+    Xd = torch.from_numpy(X).to(dev)
+    if only is None or only == "awq_search_11008x4096":
+        res["awq_search_11008x4096"] = search_workload(Wd, Xd, dev)
     if only is not None and only != "quantize_pack_11008x4096":
         return res
     # quantize + pack of the 11008 x 4096 AWQ workload (4-bit asym and 3-bit sym)
-    W, X, _ = inputs.quant_workload()
-    Wd = torch.from_numpy(W).to(dev)
-    s = w4.awq_act_scale(torch.from_numpy(X).to(dev), 0.5)
+    s = w4.awq_act_scale(Xd, 0.5)
     Wc = [Wd] + [Wd.clone() for _ in range(3)]   # 4 x 90 MB > L2
     outs = [(torch.empty((11008, 512), dtype=torch.int32, device=dev),
              torch.empty((11008, 32), dtype=torch.float16, device=dev),
@@ -576,7 +635,8 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run one of the other workloads only (gemv_4096x4096, llama7b_decode, llama65b_decode, "
-                         "skinny_8192 or skinny_8192:M, quantize_pack_11008x4096); for profiling")
+                         "skinny_8192 or skinny_8192:M, prefill_8192 or prefill_8192:M, quantize_pack_11008x4096, "
+                         "awq_search_11008x4096); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -121,8 +121,9 @@ W4A16_API w4a16_status awq_quantize_pack(const void* W, const void* s, int N, in
  * Returns 0 for invalid sizes.  The workspace holds a device status word,
  * per-row-block arrival counters and fp32 split-K partial sums (M x N for
  * M <= 4); for M >= 5 it adds, after room for the M = 4 partial sums, two
- * 256 x round_up(M, 16) fp32 slots per streaming multiprocessor of the current
- * device for the tensor-core path's partial sums.
+ * 256 x MP fp32 slots per streaming multiprocessor of the current device for
+ * the tensor-core path's partial sums (MP = M rounded up to 16 up to 64, then
+ * 96 or 128).  For M > 128 it is the size for M = 128.
  */
 W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
 
@@ -132,17 +133,18 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  *   y[m][n] = fp16( sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k] )
  *
  * with fp32 accumulation.  M = 1..4 runs on the CUDA cores (M = 1: whole rows
- * per SM, no partial sums; M = 2..4: split-K); M = 5..64 runs on the tensor
- * cores (tcgen05), with w_hat = Delta * (u - z) rounded once to fp16 before the
- * MMA (so |w_hat| must stay below 65504).  x is the activation already divided
- * by the AWQ scale s.
+ * per SM, no partial sums; M = 2..4: whole rows or split-K); M = 5..128 runs on
+ * the tensor cores (tcgen05), with w_hat = Delta * (u - z) rounded once to fp16
+ * before the MMA (so |w_hat| must stay below 65504).  Larger M (prefill) runs
+ * as consecutive chunks of 128 tokens, each chunk as above, on the same
+ * workspace.  x is the activation already divided by the AWQ scale s.
  * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
  * y_ref the exact product with the dequantized weight.  The order of the
  * split-K additions may vary between calls, so y may differ in the last bit.
  *
  *   x        fp16 [M][K], device.     y  fp16 [M][N], device (output).
  *   qweight, scales, zeros as produced by awq_quantize_pack (layout v1).
- *   1 <= M <= 64;  N >= 1;  K a multiple of group;  group == 128.
+ *   M, N >= 1;  K a multiple of group;  group == 128;  N*K, M*K, M*N below 2^31.
  *   workspace  device memory of at least w4a16_gemm_workspace_size(M, N, K, group)
  *              bytes, 16-byte aligned, ZERO-FILLED before its first use.  Every
  *              call that completes leaves the part that must start at zero (the
@@ -169,7 +171,7 @@ W4A16_API size_t awq_search_workspace_size(int N, int K, int T, int n_alpha, int
  *     s          = awq_act_scale(X, alpha)                   (fp16 [K])
  *     qweight, scales, zeros = awq_quantize_pack(W, s, group, bits, mode)
  *     x'         = fp16(X / s)                               (per element, one rounding)
- *     y_q        = w4a16_gemm(x', qweight, scales, zeros)    (fp16 [T][N], chunks of <= 64 tokens)
+ *     y_q        = w4a16_gemm(x', qweight, scales, zeros)    (fp16 [T][N])
  *     losses[a]  = mean over the T x N outputs of (y_q - y)^2,   y = X W^T
  *   *best = the first a with the smallest loss
  *
@@ -182,8 +184,8 @@ W4A16_API size_t awq_search_workspace_size(int N, int K, int T, int n_alpha, int
  * ones awq_quantize_pack produces for it.  y is formed once, in fp32 on the
  * CUDA cores, from the exact fp16 products; each loss is an fp64 sum in a fixed
  * order, so the losses repeat exactly from call to call whenever the GEMM
- * outputs do (always when every chunk has 5 or more tokens; a chunk of 1 to 4
- * tokens on the split-K GEMV may differ in the last bit of y).
+ * outputs do (always unless a final chunk of 1 to 4 tokens runs on the split-K
+ * GEMV, whose y may differ in the last bit).
  *
  *   W        fp16 [N][K], device.    X  fp16 [T][K] calibration tokens, device.
  *   alphas   double [n_alpha], host, finite (the pages search [0, 1]).

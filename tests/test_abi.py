@@ -82,7 +82,9 @@ def test_workspace_size(lib):
     assert ws(1, 8192, 8192, 128) > 8192 * 4
     assert ws(4, 100, 256, 128) >= 4 * 100 * 4
     assert ws(0, 8, 128, 128) == 0
-    assert ws(65, 8, 128, 128) == 0
+    # M above one launch's 128 tokens runs in chunks on the M = 128 workspace
+    assert ws(200, 8, 128, 128) == ws(128, 8, 128, 128) > ws(64, 8, 128, 128)
+    assert ws(1 << 20, 4096, 4096, 128) == 0
     assert ws(1, 8, 100, 128) == 0
     assert ws(1, 8, 128, 64) == 0
 
@@ -94,7 +96,7 @@ def test_gemm_validation(lib):
     assert g(A, A, A, A, 0, 64, 256, 128, A, B, need, None) == ERR_ARG
     assert g(A, A, A, A, 1, 64, 256, 64, A, B, need, None) == ERR_UNSUPPORTED
     assert g(A, A, A, A, 1, 64, 200, 128, A, B, need, None) == ERR_SHAPE
-    assert g(A, A, A, A, 65, 64, 256, 128, A, B, need, None) == ERR_UNSUPPORTED
+    assert g(A, A, A, A, 1 << 24, 64, 256, 128, A, B, need, None) == ERR_SHAPE
     assert g(MIS, A, A, A, 1, 64, 256, 128, A, B, need, None) == ERR_ALIGN
     assert g(A, A, A, A, 1, 64, 256, 128, MIS, B, need, None) == ERR_ALIGN
     assert g(A, A, A, A, 1, 64, 256, 128, A, None, need, None) == ERR_WORKSPACE

@@ -4,9 +4,9 @@ L(alpha) = mean over outputs of (Q(W s)(s^-1 X) - W X)^2, s = s_X^alpha, and
 alpha* = argmin over the grid ("MIT 6.5940 Fall 2024 Lecture 13: LLM
 Deployment" reading guide, §AWQ, slide 28).  The codes behind every loss are
 bit-exact to the oracle's (the quantizer's own tests pin that); the losses
-differ only through the W4A16 GEMM's fp32 accumulation (and, for chunks of 5
-or more tokens, the fp16 rounding of w_hat before the MMA) and through the
-fp32 target.  Those errors are far below the quantization error and not
+differ only through the W4A16 GEMM's fp32 accumulation (and, on the tensor
+cores, the fp16 rounding of w_hat before the MMA) and through the fp32
+target.  Those errors are far below the quantization error and not
 correlated with it, so each loss must agree to RTOL relative; the GEMM's
 stated worst-case bound would allow much more, but it is not what decides
 alpha.  Where the two searches pick different grid points, the oracle's loss
@@ -48,9 +48,9 @@ def compare(losses, best, ref_losses, ref_best):
 
 
 @pytest.mark.parametrize("N,K,T,bits,mode", [
-    (256, 1024, 100, 4, oracle.ASYM),   # two GEMM chunks: 64 tokens on the tensor cores, then 36
-    (129, 512, 130, 4, oracle.ASYM),    # odd N (padded chunk stride), chunks 64 + 64 + 2 (a GEMV tail)
-    (200, 512, 64, 3, oracle.SYM),      # the 3-bit symmetric codes, one chunk
+    (256, 1024, 100, 4, oracle.ASYM),   # one GEMM launch with a 128-token tile
+    (129, 512, 130, 4, oracle.ASYM),    # odd N, chunks of 128 + 2 tokens (a GEMV tail)
+    (200, 512, 300, 3, oracle.SYM),     # the 3-bit symmetric codes, chunks of 128 + 128 + 44
     (300, 256, 3, 4, oracle.ASYM),      # a few tokens: the CUDA-core GEMV only
     (64, 128, 1, 4, oracle.ASYM),       # one token, one group
 ])

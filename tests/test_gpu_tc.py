@@ -1,4 +1,5 @@
-"""Parity of the tensor-core skinny GEMM (M = 5..64) with the CPU oracle.
+"""Parity of the tensor-core GEMM (M = 5..128 per launch, larger M in chunks of
+128 tokens) with the CPU oracle.
 
 Every case goes through the C ABI (``w4a16_gemm``).  The output must satisfy,
 per element, |y - y_ref| <= 2e-3 * B + 1e-3 with B = sum_k |x * w_hat| and
@@ -68,6 +69,43 @@ def case(dev, M, N, K, seed, bits=4, mode=oracle.ASYM, workspace=None):
 ])
 def test_tc_small_shapes(dev, M, N, K):
     case(dev, M, N, K, seed=M * 7919 + N)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (65, 300, 1024),      # MP = 96, ragged row block
+    (96, 513, 2048),
+    (100, 256, 1152),     # MP = 128, odd groups per row
+    (128, 1000, 4096),
+    (128, 64, 8192),      # many CTAs share one row block
+])
+def test_tc_wide_token_tiles(dev, M, N, K):
+    case(dev, M, N, K, seed=M * 7919 + N)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (129, 300, 1024),     # 128 + 1: the tail runs on the M = 1 GEMV
+    (130, 256, 2048),     # 128 + 2: the tail on the whole-row GEMV for M = 2..4
+    (200, 513, 1152),     # 128 + 72, odd groups per row
+    (300, 256, 4096),     # 128 + 128 + 44
+    (512, 384, 2048),     # four full chunks
+])
+def test_tc_large_m_chunks(dev, M, N, K):
+    case(dev, M, N, K, seed=M * 7919 + N)
+
+
+def test_tc_prefill_workload_sampled_rows(dev):
+    """M = 512 tokens on the 8192 x 8192 layer; 128 sampled rows checked for every token."""
+    (layer,) = inputs.layer_set(inputs.SKINNY)
+    rng = np.random.default_rng(512)
+    x = inputs.activations(rng, 512, layer.K, layer.outliers)
+    qg, sg, zg = w4.awq_quantize_pack(to_dev(layer.W, dev))
+    y = w4.w4a16_gemm(to_dev(x, dev), qg, sg, zg)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([rng.choice(layer.N, 124, replace=False), [0, 255, 256, layer.N - 1]]))
+    qw = qg.cpu().numpy().view(np.uint32)[rows]
+    y_ref, B = oracle.gemm_ref(x, oracle.dequant(qw, sg.cpu().numpy()[rows], zg.cpu().numpy()[rows]))
+    err = np.abs(y.cpu().numpy()[:, rows].astype(np.float64) - y_ref)
+    assert np.all(err <= RTOL * B + ATOL)
 
 
 def test_tc_whole_row_blocks_written_directly(dev):

@@ -119,22 +119,36 @@ Workspace carve_workspace(void* base, int M, int N, int K) {
   return w;
 }
 
-// The kernel w4a16_gemm runs for an M x N x K problem: M = 1 on whole rows when
+// The kernels for an M x N x K problem with M <= kMaxM: M = 1 on whole rows when
 // the activation fits the kernel's staging, M = 2..4 on whole rows or split-K,
-// M = 5..64 on the tensor cores.
-cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
+// M = 5..128 on the tensor cores.
+static cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
   if (p.M == 1 && gemv_m1_supports(p.N, p.K)) return launch_gemv_m1(p, ws.status, st);
   if (gemv_mt_supports(p.M, p.N, p.K)) return launch_gemv_mt(p, ws.status, st);
   if (p.M <= kMaxGemvM && gemv_supports(p.M, p.K)) return launch_gemv(p, ws, st);
   return launch_gemm_tc(p, ws, st);
 }
 
+cudaError_t gemm_chunks(const GemmProblem& p, void* workspace, cudaStream_t st) {
+  // Chunk c starts kMaxM * c tokens in: its x and y offsets are multiples of
+  // 256 bytes per input and per output channel, so both stay 16-byte aligned.
+  // Stream order keeps the chunks' uses of the workspace apart (a chunk's
+  // partial sums are written only after its griddepcontrol.wait, which waits
+  // for the previous chunk's finalize to complete).
+  for (int t0 = 0; t0 < p.M; t0 += kMaxM) {
+    GemmProblem c = p;
+    c.M = p.M - t0 < kMaxM ? p.M - t0 : kMaxM;
+    c.x = p.x + static_cast<size_t>(t0) * p.K;
+    c.y = p.y + static_cast<size_t>(t0) * p.N;
+    const cudaError_t e = dispatch_gemm(c, carve_workspace(workspace, c.M, p.N, p.K), st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 // Workspace of awq_search_alpha: every region starts on a 256-byte boundary.
-// The quantized outputs are kept per GEMM chunk of up to kMaxM tokens, each
-// chunk's [rows][N] block starting on a 16-byte boundary as w4a16_gemm needs.
 struct SearchLayout {
-  int chunk_rows;            // tokens per GEMM chunk: min(T, kMaxM)
-  long long chunk_stride;    // elements between chunks of yq
+  int gemm_rows;  // tokens of the GEMM workspace: min(T, kMaxM)
   size_t gemm, qweight, scales, zeros, s, xd, yq, yref, partial, sums, total;
 };
 
@@ -142,9 +156,7 @@ static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 static SearchLayout search_layout(int N, int K, int T, int n_alpha) {
   SearchLayout L;
-  L.chunk_rows = T < kMaxM ? T : kMaxM;
-  L.chunk_stride = (static_cast<long long>(L.chunk_rows) * N + 7) / 8 * 8;
-  const size_t chunks = (static_cast<size_t>(T) + L.chunk_rows - 1) / L.chunk_rows;
+  L.gemm_rows = T < kMaxM ? T : kMaxM;
   size_t off = 0;
   auto take = [&off](size_t bytes) {
     const size_t at = off;
@@ -152,13 +164,13 @@ static SearchLayout search_layout(int N, int K, int T, int n_alpha) {
     return at;
   };
   const size_t groups = static_cast<size_t>(N) * (K / kGroup);
-  L.gemm = take(workspace_bytes(L.chunk_rows, N, K));
+  L.gemm = take(workspace_bytes(L.gemm_rows, N, K));
   L.qweight = take(static_cast<size_t>(N) * (K / 8) * 4);
   L.scales = take(groups * 2);
   L.zeros = take(groups * 2);
   L.s = take(static_cast<size_t>(K) * 2);
   L.xd = take(static_cast<size_t>(T) * K * 2);
-  L.yq = take(chunks * static_cast<size_t>(L.chunk_stride) * 2);
+  L.yq = take(static_cast<size_t>(T) * N * 2);
   L.yref = take(static_cast<size_t>(T) * N * 4);
   L.partial = take(static_cast<size_t>(n_alpha) * search_error_blocks() * 8);
   L.sums = take(static_cast<size_t>(n_alpha) * 8);
@@ -210,8 +222,11 @@ w4a16_status awq_quantize_pack(const void* W, const void* s, int N, int K, int g
 }
 
 size_t w4a16_gemm_workspace_size(int M, int N, int K, int group) {
-  if (M < 1 || M > kMaxM || N < 1 || K < 1 || group != kGroup || K % group) return 0;
-  return workspace_bytes(M, N, K);
+  if (M < 1 || N < 1 || K < 1 || group != kGroup || K % group) return 0;
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(M) * K >= kMaxElems ||
+      static_cast<long long>(M) * N >= kMaxElems)
+    return 0;
+  return workspace_bytes(M < kMaxM ? M : kMaxM, N, K);
 }
 
 w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scales, const void* zeros, int M, int N,
@@ -220,17 +235,18 @@ w4a16_status w4a16_gemm(const void* x, const uint32_t* qweight, const void* scal
   if (M < 1 || N < 1 || K < 1) return fail(W4A16_ERR_ARG, "w4a16_gemm: M=%d N=%d K=%d must be >= 1", M, N, K);
   if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: group=%d (only 128)", group);
   if (K % group) return fail(W4A16_ERR_SHAPE, "w4a16_gemm: K=%d not a multiple of group=%d", K, group);
-  if (M > kMaxM) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: M=%d (at most %d)", M, kMaxM);
-  if (static_cast<long long>(N) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "w4a16_gemm: N*K too large");
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(M) * K >= kMaxElems ||
+      static_cast<long long>(M) * N >= kMaxElems)
+    return fail(W4A16_ERR_SHAPE, "w4a16_gemm: N*K, M*K or M*N too large");
   if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
     return fail(W4A16_ERR_ALIGN, "w4a16_gemm: pointers must be 16-byte aligned");
-  const size_t need = workspace_bytes(M, N, K);
+  const size_t need = workspace_bytes(M < kMaxM ? M : kMaxM, N, K);
   if (!workspace || workspace_bytes_ < need)
     return fail(W4A16_ERR_WORKSPACE, "w4a16_gemm: workspace of %zu bytes needed, %zu given", need, workspace_bytes_);
   if (!aligned16(workspace)) return fail(W4A16_ERR_ALIGN, "w4a16_gemm: workspace must be 16-byte aligned");
   GemmProblem p{static_cast<const __half*>(x), qweight, static_cast<const __half*>(scales),
                 static_cast<const __half*>(zeros), static_cast<__half*>(y), M, N, K};
-  const cudaError_t e = dispatch_gemm(p, carve_workspace(workspace, M, N, K), reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e = gemm_chunks(p, workspace, reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "w4a16_gemm: M=%d K=%d not supported yet", M, K);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm launch");
   return ok();
@@ -286,7 +302,7 @@ w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T,
   const int blocks = search_error_blocks();
 
   // The GEMM workspace must start zeroed; its status word doubles as the search's.
-  cudaError_t e = cudaMemsetAsync(base + L.gemm, 0, workspace_bytes(L.chunk_rows, N, K), st);
+  cudaError_t e = cudaMemsetAsync(base + L.gemm, 0, workspace_bytes(L.gemm_rows, N, K), st);
   if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: clear workspace");
   e = launch_reference_gemm(Xh, Wh, T, N, K, yref, st);
   if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha: reference product");
@@ -295,15 +311,9 @@ w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T,
     if (e == cudaSuccess)
       e = launch_quantize_pack(Wh, s, N, K, bits, static_cast<int>(mode), qweight, scales, zeros, st);
     if (e == cudaSuccess) e = launch_divide_activation(Xh, s, T, K, xd, st);
-    for (int t0 = 0, c = 0; t0 < T && e == cudaSuccess; t0 += L.chunk_rows, ++c) {
-      const int m = T - t0 < L.chunk_rows ? T - t0 : L.chunk_rows;
-      const GemmProblem p{xd + static_cast<size_t>(t0) * K, qweight, scales, zeros, yq + c * L.chunk_stride,
-                          m, N, K};
-      e = dispatch_gemm(p, carve_workspace(base + L.gemm, m, N, K), st);
-    }
+    if (e == cudaSuccess) e = gemm_chunks(GemmProblem{xd, qweight, scales, zeros, yq, T, N, K}, base + L.gemm, st);
     if (e == cudaSuccess)
-      e = launch_squared_error(yq, yref, T, N, L.chunk_rows, L.chunk_stride,
-                               partial + static_cast<size_t>(a) * blocks, st);
+      e = launch_squared_error(yq, yref, static_cast<long long>(T) * N, partial + static_cast<size_t>(a) * blocks, st);
   }
   if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "awq_search_alpha: K=%d not supported", K);
   if (e != cudaSuccess) return cuda_fail(e, "awq_search_alpha launch");

@@ -80,23 +80,15 @@ __global__ void __launch_bounds__(256) divide_activation_kernel(const __half* __
 }
 
 // ---- squared error, per-block fp64 partials ---------------------------------------
-// Yq holds the quantized outputs in chunks of chunk_rows tokens, chunk c at
-// element c * chunk_stride (each chunk is one GEMM's [rows][N] output, aligned
-// for it); Y is the dense [T][N] target.  Block b adds (Yq - Y)^2 over the
-// elements i = b * 256 + tid + j * stride of Y in j order, then over its
-// threads in a fixed tree; sum_partials_kernel adds the blocks in order, so the
-// loss is the same on every run.
+// Block b adds (Yq - Y)^2 over elements b * 256 + tid + j * stride in j order,
+// then over its threads in a fixed tree; sum_partials_kernel adds the blocks in
+// order, so the loss is the same on every run.
 __global__ void __launch_bounds__(256) squared_error_kernel(const __half* __restrict__ Yq, const float* __restrict__ Y,
-                                                            int T, int N, int chunk_rows, long long chunk_stride,
-                                                            double* __restrict__ partial) {
+                                                            long long total, double* __restrict__ partial) {
   __shared__ double red[256];
-  const long long total = static_cast<long long>(T) * N;
-  const long long chunk_elems = static_cast<long long>(chunk_rows) * N;
   double acc = 0.0;
   for (long long i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
-    const long long c = i / chunk_elems;
-    const double d = static_cast<double>(__half2float(Yq[c * chunk_stride + (i - c * chunk_elems)])) -
-                     static_cast<double>(Y[i]);
+    const double d = static_cast<double>(__half2float(Yq[i])) - static_cast<double>(Y[i]);
     acc = fma(d, d, acc);
   }
   red[threadIdx.x] = acc;
@@ -136,9 +128,8 @@ cudaError_t launch_divide_activation(const __half* X, const __half* s, int T, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_squared_error(const __half* Yq, const float* Y, int T, int N, int chunk_rows, long long chunk_stride,
-                                 double* partial, cudaStream_t st) {
-  squared_error_kernel<<<search_error_blocks(), 256, 0, st>>>(Yq, Y, T, N, chunk_rows, chunk_stride, partial);
+cudaError_t launch_squared_error(const __half* Yq, const float* Y, long long total, double* partial, cudaStream_t st) {
+  squared_error_kernel<<<search_error_blocks(), 256, 0, st>>>(Yq, Y, total, partial);
   return cudaGetLastError();
 }
 

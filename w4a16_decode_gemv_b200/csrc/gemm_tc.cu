@@ -1,4 +1,5 @@
-// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05) for M = 5..64.
+// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05) for M = 5..128
+// (larger M runs as chunks of 128 tokens, one launch pair per chunk).
 //
 //   y[m][n] = sum_k x[m][k] * w_hat[n][k],   w_hat = Delta[n][g] * (u[n][k] - z[n][g])
 //
@@ -10,7 +11,8 @@
 // the dequantization and the MMAs under that time.
 //
 // Swap-AB.  The weight rows are the MMA's M dimension (128 rows per MMA) and the
-// tokens its N dimension (MP = M rounded up to 16): D[n][m] = sum_k A[n][k] B[m][k]
+// tokens its N dimension (the token tile MP: M rounded up to 16 up to 64, then
+// 96 or 128): D[n][m] = sum_k A[n][k] B[m][k]
 // with A = w_hat (fp16) and B = x (fp16, K-major in shared memory), fp32
 // accumulators in tensor memory (TMEM lane = weight row, column = token).
 //
@@ -226,7 +228,7 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
 // Tensor memory holds only the accumulators: 2 buffers x 2 tiles x MP columns,
 // allocated as the next power of two of at least 32 columns.
 __host__ __device__ constexpr uint32_t tmem_cols(int mp) {
-  return 4 * mp <= 32 ? 32u : 4 * mp <= 64 ? 64u : 4 * mp <= 128 ? 128u : 256u;
+  return 4 * mp <= 32 ? 32u : 4 * mp <= 64 ? 64u : 4 * mp <= 128 ? 128u : 4 * mp <= 256 ? 256u : 512u;
 }
 // w_hat lives in shared memory: kABufs buffers, each one 64-input half of a
 // unit (2 tiles x 128 rows x 128 bytes, K-major with the 128-byte swizzle, the
@@ -639,16 +641,22 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   return cudaGetLastError();
 }
 
+// The token tile of a launch: M rounded up to 16 up to 64, then 96 or 128.
+int tc_tile(int M) {
+  const int mp = (M + 15) / 16 * 16;
+  return mp <= 64 ? mp : (mp <= 96 ? 96 : 128);
+}
+
 }  // namespace
 
 size_t tc_partial_bytes(int M) {
-  const size_t mp = (static_cast<size_t>(M) + 15) / 16 * 16;
+  const size_t mp = static_cast<size_t>(tc_tile(M));
   return 2 * static_cast<size_t>(device_sm_count()) * kRows * mp * 4;
 }
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
   if (p.M < 1 || p.M > kMaxM || !ws.part) return cudaErrorNotSupported;
-  const int mp = (p.M + 15) / 16 * 16;
+  const int mp = tc_tile(p.M);
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
 
@@ -696,7 +704,9 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
     case 16: return launch_mp<16>(a, tq, tx, grid, st);
     case 32: return launch_mp<32>(a, tq, tx, grid, st);
     case 48: return launch_mp<48>(a, tq, tx, grid, st);
-    default: return launch_mp<64>(a, tq, tx, grid, st);
+    case 64: return launch_mp<64>(a, tq, tx, grid, st);
+    case 96: return launch_mp<96>(a, tq, tx, grid, st);
+    default: return launch_mp<128>(a, tq, tx, grid, st);
   }
 }
 

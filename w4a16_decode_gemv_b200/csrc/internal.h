@@ -12,7 +12,7 @@ namespace w4a16 {
 
 constexpr int kGroup = 128;        // group size along K (the only one supported)
 constexpr int kMaxGemvM = 4;       // largest M the CUDA-core GEMV handles
-constexpr int kMaxM = 64;          // largest M of w4a16_gemm
+constexpr int kMaxM = 128;         // largest M of one launch sequence; larger M runs in chunks of it
 
 // Replaces the calling thread's message returned by w4a16_last_error().
 void set_last_error(const char* msg);
@@ -38,7 +38,7 @@ cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K,
 // Workspace: [status word | padding to 16 B] [row-block counters, padded to
 // 16 B] [fp32 partial sums M x N of the CUDA-core GEMV, M <= 4] and, for
 // M >= 5, after room for 4 x N GEMV partials: the tensor-core path's
-// partial-sum slots (2 per CTA of 256 x MP fp32, MP = M rounded up to 16).
+// partial-sum slots (2 per CTA of 256 x MP fp32, MP the launch's token tile).
 // The counters and GEMV partials must be zero when a kernel starts and are
 // left zero; the slots are scratch, written before they are read.
 struct Workspace {
@@ -72,27 +72,27 @@ cudaError_t launch_gemv_mt(const GemmProblem& p, uint32_t* status, cudaStream_t 
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 
-// The tensor-core skinny GEMM (gemm_tc.cu), M = 5..64, and the bytes of its
-// partial-sum slots on the current device.
+// The tensor-core GEMM (gemm_tc.cu), M = 5..128 per launch, and the bytes of
+// its partial-sum slots on the current device.
 size_t tc_partial_bytes(int M);
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 // One CTA waits on a shared-memory barrier that nothing completes, gives up
 // after limit_ns and sets kDevWaitTimeout in *status (the GEMM kernels' path).
 cudaError_t launch_wait_timeout_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
-// The kernel w4a16_gemm dispatches to for p (api.cu).
-cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
+// The kernels w4a16_gemm runs for p (api.cu): one launch sequence per chunk of
+// at most kMaxM tokens, all on the workspace at `workspace` (sized for
+// min(M, kMaxM) tokens).
+cudaError_t gemm_chunks(const GemmProblem& p, void* workspace, cudaStream_t st);
 
 // Kernels of the AWQ alpha search (awq_search.cu).  Y = X W^T in fp32 (X [T][K],
-// W [N][K] fp16); Xd = fp16(X / s); per-block fp64 partial sums of (Yq - Y)^2,
-// search_error_blocks() of them, with Yq in GEMM-sized chunks of chunk_rows
-// tokens at chunk_stride elements apart; sums[a] = the n_alpha groups of
-// partials added in block order.
+// W [N][K] fp16); Xd = fp16(X / s); per-block fp64 partial sums of (Yq - Y)^2
+// over `total` elements, search_error_blocks() of them; sums[a] = the n_alpha
+// groups of partials added in block order.
 int search_error_blocks();
 cudaError_t launch_reference_gemm(const __half* X, const __half* W, int T, int N, int K, float* Y, cudaStream_t st);
 cudaError_t launch_divide_activation(const __half* X, const __half* s, int T, int K, __half* Xd, cudaStream_t st);
-cudaError_t launch_squared_error(const __half* Yq, const float* Y, int T, int N, int chunk_rows, long long chunk_stride,
-                                 double* partial, cudaStream_t st);
+cudaError_t launch_squared_error(const __half* Yq, const float* Y, long long total, double* partial, cudaStream_t st);
 cudaError_t launch_sum_partials(const double* partial, int n_alpha, double* sums, cudaStream_t st);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
