@@ -105,6 +105,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's ordinary shared-memory reads of a ring stage before the
+// tensor copy (async proxy) that will next overwrite the stage.  Every thread
+// that read the stage runs it before the hand-off (__syncwarp or an mbarrier
+// arrival) that lets the copy be issued; without it, on B200 a refilled stage
+// was seen to change under reads still in flight.
+__device__ __forceinline__ void release_stage_reads() { fence_proxy_async_smem(); }
+
 // ---- fp16 nibble unpacking ---------------------------------------------------
 // (w & mask) | 0x64006400: a nibble q placed in the low mantissa bits of the
 // fp16 exponent-10 binade reads as 1024 + q (bits 0..3) or 1024 + 16 q (bits 4..7).

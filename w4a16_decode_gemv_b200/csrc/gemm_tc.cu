@@ -485,6 +485,7 @@ __global__ void __maxnreg__(96)
       const uint32_t row = st0 + static_cast<uint32_t>(s * kStageBytes + rloc * 64);
       const uint4 c0 = lds128(row + ((static_cast<uint32_t>(p) ^ sw_ld) << 4));
       const uint4 c1 = lds128(row + ((static_cast<uint32_t>(2 + p) ^ sw_ld) << 4));
+      release_stage_reads();
       __syncwarp();
       if (lane == 0) mbar_arrive(&rempty[s]);  // codes are in registers
       const uint32_t dv = pick_half(dc, g & (W - 1)), zv = pick_half(zc, g & (W - 1));

@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         acc[r] = df * fmaf(-zf, xsum, fmaf(o0 + o1, pow2f(-4), e0 + e1));
       }
     }
-    // refill the stage with this warp's unit i + S (its reads above are done)
+    // refill the stage with this warp's unit i + S once every lane's reads are done
+    release_stage_reads();
     __syncwarp();
     if (jf < U) issue_next(s);
     // reduce the unit's 4 row partials over the lanes

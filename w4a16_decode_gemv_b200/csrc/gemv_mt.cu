@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_mt_kernel(const MtArgs a, co
         }
       }
     }
+    release_stage_reads();
     __syncwarp();
     if (jf < U) issue_next(s);
     // totals of the unit's kR x MP partials over the lanes; lane q < kR * MP
