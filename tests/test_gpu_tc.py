@@ -147,9 +147,28 @@ def test_tc_workspace_shared_across_paths(dev):
 
 
 def test_tc_repeated_calls_identical(dev):
-    """Calls repeat on the same inputs; partial sums may add in another order, so each is checked."""
+    """Calls repeat on the same inputs and agree with the oracle every time."""
     args, ref = case(dev, 64, 512, 8192, seed=7)
     y1 = w4.w4a16_gemm(*args).cpu().numpy()
     y2 = w4.w4a16_gemm(*args).cpu().numpy()
     check(y1, *ref)
     check(y2, *ref)
+
+
+@pytest.mark.parametrize("M", [16, 128, 300])
+def test_tc_bit_identical_across_calls(dev, M):
+    """The partial sums of shared row blocks are added in CTA order, so y must not
+    change by a single bit from call to call.  At 8192 x 8192 every CTA streams
+    about 14 units through its rings, which exposes a ring stage overwritten
+    while it is still being read (the tolerance of the parity tests can hide it)."""
+    (layer,) = inputs.layer_set(inputs.SKINNY)
+    rng = np.random.default_rng(M)
+    qg, sg, zg = w4.awq_quantize_pack(to_dev(layer.W, dev))
+    x = to_dev(inputs.activations(rng, M, layer.K, layer.outliers), dev)
+    ws = torch.zeros(w4.gemm_workspace_size(M, layer.N, layer.K), dtype=torch.uint8, device=dev)
+    y0 = w4.w4a16_gemm(x, qg, sg, zg, workspace=ws).clone()
+    diff = torch.zeros((), dtype=torch.int64, device=dev)
+    for _ in range(20):
+        diff += (w4.w4a16_gemm(x, qg, sg, zg, workspace=ws) != y0).sum()
+    w4.gemm_check(ws)
+    assert int(diff) == 0
