@@ -22,14 +22,26 @@ Pages cited (by title and section):
   lecture slide 10: zero-point scale from (max - min) / (2^8 - 1), a rounded
   zero point, clipping to the code range, dequant = (q - zp) * step, and a
   zero range replaced by 1.  §"back to the question": batch-1 decode is a GEMV
-  and memory-bound.
+  and memory-bound.  §L20 "GPTQ": the layer objective ||WX - W_hat X||^2;
+  quantize one column block at a time and push each column's rounding error
+  onto the columns not yet quantized; the four steps (G = Cholesky((2XX^T +
+  lambda I)^-1)^T computed first; quantize one column; divide its error by
+  G's diagonal element; update the rest of the block, then everything right
+  of the block at once); a fixed column order (slide 18); the Cholesky factor
+  precomputed instead of updating H^-1 (slide 20); the AutoGPTQ example uses
+  4 bits and group size 128.
 * [Lab4] "MIT 6.5940 Lab 4 + Lab 5" reading guide (quidproquo.cc).  §Lab 4
   setup: calibration statistic = mean |X| per input channel over 512-token
   blocks; pseudo quantization (quantize, then dequantize at once); 3-bit,
   group 128.
 * [ML11] "Learning-ML-DL ch. 11: Quantization for LLMs"
   (hoangvt2501.github.io).  §11.3: Y = (X diag(s)^-1)(W diag(s))^T;
-  §11.4: AWQ's s = s_X^alpha with s_X the mean channel magnitude.
+  §11.4: AWQ's s = s_X^alpha with s_X the mean channel magnitude; GPTQ's
+  Hessian H = 2XX^T of the output error per weight row, the OBS correction
+  of the later columns after quantizing column q, damping by a fraction of
+  the mean diagonal of H, the upper Cholesky factor of H^-1, and the
+  qualitative result that GPTQ raises the weight error but lowers the output
+  error.
 
 Readings of points the pages leave open:
 
@@ -54,6 +66,25 @@ Readings of points the pages leave open:
    norm.  The divided activation is rounded to fp16 once, x' = fp16(x / s); the
    quantized output is taken as the W4A16 GEMM delivers it, rounded to fp16;
    the target W X is exact.  The grid of alphas is the caller's.
+10. GPTQ Hessian: H = 2 X^T X over calibration tokens X[T, K] (the pages'
+   2 X X^T with tokens as columns), plus lambda I with lambda = 0.01 *
+   mean(diag(2 X^T X)) ([ML11] §11.4 damps by a fraction of the mean
+   diagonal; 0.01 is its default; [CMU] L20 writes lambda I without a value).
+11. GPTQ blocks are the quantization groups (128 columns), swept left to
+   right.  Delta and z of a group come from the group's weights as they stand
+   when the sweep reaches its first column (the rounding errors of earlier
+   groups already pushed into them), by the RTN formulas of readings 1-5
+   applied to those float64 values: Delta = fp16(fp64(fp64(max - min) /
+   (2^N - 1))).  GPTQ here takes no AWQ scale (s = 1).
+12. GPTQ arithmetic order (float64, each product and each sum rounded once):
+   for column i of a block, u = clamp(Round(w / Delta) + z), q = (u - z) Delta,
+   e = (w - q) / G[i, i]; every later column j of the block becomes
+   w_j - e G[i, j].  After the block, every column j right of it becomes
+   w_j - A_j with A_j = sum of e_i G[i, j] over the block's columns i, added
+   in column order starting from 0.
+13. G = Cholesky(H^-1)^T is the upper-triangular factor with H^-1 = G^T G and
+   a positive diagonal ([CMU] L20 step 1); it is computed by numpy's Cholesky
+   of numpy's inverse.
 
 Every function here is pinned by tests marked ``not gpu`` against closed
 forms, brute force, invariants the pages state, or special cases.
@@ -250,3 +281,71 @@ def awq_search(W: np.ndarray, X: np.ndarray, alphas, group: int = 128, bits: int
     losses = [awq_loss(W, X, float(a), group, bits, mode) for a in alphas]
     return losses, int(np.argmin(losses))
 
+
+# ---------------------------------------------------------------------------
+# GPTQ: error-compensating column sweep  ([CMU] §L20 "GPTQ"; [ML11] §11.4)
+# ---------------------------------------------------------------------------
+GPTQ_DAMP = 0.01
+
+
+def gptq_hessian(X: np.ndarray, damp: float = GPTQ_DAMP) -> np.ndarray:
+    """H = 2 X^T X + lambda I for calibration tokens X[T, K], lambda = damp * mean
+    of the diagonal of 2 X^T X (reading 10).  H is K x K, independent of T."""
+    Xf = np.asarray(X, dtype=F16).astype(F64)
+    H = 2.0 * (Xf.T @ Xf)
+    lam = damp * float(np.mean(np.diag(H)))
+    return H + lam * np.eye(H.shape[0])
+
+
+def gptq_factor(H: np.ndarray) -> np.ndarray:
+    """G = Cholesky(H^-1)^T: upper triangular, H^-1 = G^T G (reading 13)."""
+    return np.linalg.cholesky(np.linalg.inv(np.asarray(H, dtype=F64))).T
+
+
+def gptq_sweep(W: np.ndarray, G: np.ndarray, group: int = 128, bits: int = 4, mode: int = ASYM):
+    """The column sweep of [CMU] §L20 in the order of readings 11-12.
+
+    Returns (u uint8[N, K], Delta fp16[N, K/group], z fp16[N, K/group], wq
+    float64[N, K]), where wq[:, i] is column i as it stood when it was
+    quantized (the value its code rounds).
+    """
+    Wc = np.asarray(W, dtype=F16).astype(F64).copy()
+    G = np.asarray(G, dtype=F64)
+    N, K = Wc.shape
+    qmax = 2 ** bits - 1
+    u = np.zeros((N, K), dtype=np.uint8)
+    wq = np.zeros((N, K), dtype=F64)
+    deltas = np.zeros((N, K // group), dtype=F16)
+    zeros = np.zeros((N, K // group), dtype=F16)
+    for gi, b0 in enumerate(range(0, K, group)):
+        b1 = b0 + group
+        # group parameters from the block as the sweep finds it (reading 11)
+        d16, z16 = group_params(Wc[:, b0:b1], bits, mode, group)
+        deltas[:, gi], zeros[:, gi] = d16[:, 0], z16[:, 0]
+        d, z = d16[:, 0].astype(F64), z16[:, 0].astype(F64)
+        errs = np.zeros((N, group), dtype=F64)
+        for i in range(b0, b1):
+            w = Wc[:, i].copy()
+            wq[:, i] = w
+            ui = np.clip(np.rint(w / d) + z, 0, qmax)
+            u[:, i] = ui.astype(np.uint8)
+            e = (w - (ui - z) * d) / G[i, i]
+            errs[:, i - b0] = e
+            # the rest of the block, one column's correction at a time
+            Wc[:, i + 1:b1] = Wc[:, i + 1:b1] - e[:, None] * G[i, i + 1:b1][None, :]
+        # everything right of the block at once: the block's corrections summed in column order
+        if b1 < K:
+            acc = np.zeros((N, K - b1), dtype=F64)
+            for i in range(b0, b1):
+                acc = acc + errs[:, i - b0][:, None] * G[i, b1:][None, :]
+            Wc[:, b1:] = Wc[:, b1:] - acc
+    return u, deltas, zeros, wq
+
+
+def gptq_quantize(W: np.ndarray, X: np.ndarray, group: int = 128, bits: int = 4, mode: int = ASYM,
+                  damp: float = GPTQ_DAMP):
+    """GPTQ end to end: (qweight u32[N, K/8] in layout v1, scales fp16, zeros fp16),
+    the same format awq_quantize_pack produces, for the same GEMV."""
+    G = gptq_factor(gptq_hessian(X, damp))
+    u, d, z, _ = gptq_sweep(W, G, group, bits, mode)
+    return pack_v1(u), d, z

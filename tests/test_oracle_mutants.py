@@ -1,5 +1,6 @@
 """Plant plausible mistakes in a copy of the oracle and check that the pins in
-test_oracle.py catch every one of them.  CPU only; the real oracle is untouched."""
+test_oracle.py (quantizer, packing, GEMM) and test_oracle_gptq.py (GPTQ)
+catch every one of them.  CPU only; the real oracle is untouched."""
 import os
 import shutil
 import subprocess
@@ -31,12 +32,30 @@ MUTANTS = {
     "dequant_drops_zero": ("return (u - z) * d", "return u * d"),
     "zero_range_rule": ("delta[delta == 0] = F16(1.0 / qmax)", "delta[delta == 0] = F16(1.0)"),
     "bound_not_absolute": ("bound = np.abs(x64) @ np.abs(w_hat).T", "bound = np.abs(x64 @ w_hat.T)"),
+    # GPTQ: caught by tests/test_oracle_gptq.py
+    "gptq_lower_factor": ("return np.linalg.cholesky(np.linalg.inv(np.asarray(H, dtype=F64))).T",
+                          "return np.linalg.cholesky(np.linalg.inv(np.asarray(H, dtype=F64)))", "gptq"),
+    "gptq_no_diagonal_division": ("e = (w - (ui - z) * d) / G[i, i]", "e = (w - (ui - z) * d)", "gptq"),
+    "gptq_error_sign": ("Wc[:, i + 1:b1] = Wc[:, i + 1:b1] - e[:, None] * G[i, i + 1:b1][None, :]",
+                        "Wc[:, i + 1:b1] = Wc[:, i + 1:b1] + e[:, None] * G[i, i + 1:b1][None, :]", "gptq"),
+    "gptq_no_trailing_update": ("Wc[:, b1:] = Wc[:, b1:] - acc", "Wc[:, b1:] = Wc[:, b1:]", "gptq"),
+    "gptq_trailing_row_shift": ("acc = acc + errs[:, i - b0][:, None] * G[i, b1:][None, :]",
+                                "acc = acc + errs[:, i - b0][:, None] * G[max(i - 1, 0), b1:][None, :]", "gptq"),
+    "gptq_no_damping": ("return H + lam * np.eye(H.shape[0])", "return H", "gptq"),
+    "gptq_hessian_without_2": ("H = 2.0 * (Xf.T @ Xf)", "H = Xf.T @ Xf", "gptq"),
+    "gptq_stats_from_original": ("d16, z16 = group_params(Wc[:, b0:b1], bits, mode, group)",
+                                 "d16, z16 = group_params(np.asarray(W, dtype=F16)[:, b0:b1], bits, mode, group)",
+                                 "gptq"),
+    "gptq_code_from_original": ("w = Wc[:, i].copy()", "w = np.asarray(W, dtype=F16)[:, i].astype(F64)", "gptq"),
 }
+
+PIN_FILES = {None: "tests/test_oracle.py", "gptq": "tests/test_oracle_gptq.py"}
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
-    before, after = MUTANTS[name]
+    before, after, *which = MUTANTS[name]
+    pins = PIN_FILES[which[0] if which else None]
     src = open(os.path.join(ROOT, "oracle", "w4a16_oracle.py")).read()
     assert before in src, "mutation site moved; update the mutant"
     shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle")
@@ -44,6 +63,6 @@ def test_pins_catch_mutant(name, tmp_path):
                     ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
     (tmp_path / "oracle" / "w4a16_oracle.py").write_text(src.replace(before, after))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_oracle.py"], cwd=tmp_path, capture_output=True, text=True,
+                        pins], cwd=tmp_path, capture_output=True, text=True,
                        timeout=300)
     assert r.returncode != 0, f"mutant {name} survived:\n{r.stdout[-2000:]}"
