@@ -206,6 +206,57 @@ W4A16_API w4a16_status awq_search_alpha(const void* W, const void* X, int N, int
                                         size_t workspace_bytes, w4a16_stream_t stream);
 
 /*
+ * gptq_hessian -- the damped Hessian of GPTQ's layer objective.
+ *
+ *   H = 2 X^T X + lambda I,   lambda = damp * (sum_i (2 X^T X)[i][i]) / K
+ *
+ * ("CMU 11-868 LLM Systems: Model Quantization" reading guide, §L20 "GPTQ",
+ * step 1: (2 X X^T + lambda I) with tokens as the columns of X; "Learning-ML-DL
+ * ch. 11", §11.4: damping by a fraction of the mean diagonal, 0.01 in its
+ * example.)  Entries are fp64 sums of the exact fp16 products in token order.
+ *
+ *   X  fp16 [T][K] calibration tokens, device.   H  fp64 [K][K], device (output).
+ *   T, K >= 1;  K <= 32768;  T*K below 2^31;  damp finite and >= 0.
+ */
+W4A16_API w4a16_status gptq_hessian(const void* X, int T, int K, double damp, double* H,
+                                    w4a16_stream_t stream);
+
+/* gptq_sweep_workspace_size -- bytes of workspace gptq_sweep needs; 0 for invalid sizes. */
+W4A16_API size_t gptq_sweep_workspace_size(int N, int K, int group);
+
+/*
+ * gptq_sweep -- GPTQ's error-compensating column sweep, emitting layout v1.
+ *
+ * Columns are quantized left to right in blocks of `group` columns, one block
+ * per quantization group (§L20 "GPTQ": one column block at a time, a fixed
+ * order; the error of each column, divided by G's diagonal element, updates
+ * the rest of the block, then every column right of the block at once):
+ *   at a block's first column: Delta, z from the block as it stands, by the
+ *     formulas of awq_quantize_pack (ASYM: fp16((max - min) / (2^bits - 1)) and
+ *     clamp(Round(-min / Delta)); SYM: fp16(max|w| / 2^(bits-1)) and 2^(bits-1));
+ *   column i: u = clamp(Round(w / Delta) + z, 0, 2^bits - 1),
+ *             e = (w - (u - z) Delta) / G[i][i];
+ *   later columns j of the block: w_j -= e G[i][j];
+ *   after the block, columns j right of it: w_j -= sum over the block's
+ *     columns i, in order, of e_i G[i][j].
+ * All arithmetic is fp64, one rounding per operation in that order, so the
+ * result is identical on every call and bit-exact to that definition.
+ *
+ *   W        fp16 [N][K], device.
+ *   G        fp64 [K][K], device: the upper-triangular factor with
+ *            H^-1 = G^T G (G = Cholesky(H^-1)^T, §L20 step 1), positive diagonal.
+ *   qweight  uint32 [N][K/8], scales, zeros  fp16 [N][K/group] (outputs, the
+ *            format of awq_quantize_pack, for w4a16_gemm).
+ *   N >= 1;  K a multiple of group, at most 32768;  group == 128;  bits in {3, 4}.
+ *   workspace  at least gptq_sweep_workspace_size(N, K, group) bytes, any
+ *              contents (an fp64 copy of W, the codes and one block of errors).
+ * Asynchronous on `stream`.  Computing G from H is the caller's for now.
+ */
+W4A16_API w4a16_status gptq_sweep(const void* W, const double* G, int N, int K, int group, int bits,
+                                  w4a16_mode mode, uint32_t* qweight, void* scales, void* zeros,
+                                  void* workspace, size_t workspace_bytes, w4a16_stream_t stream);
+
+/*
  * w4a16_gemm_check -- synchronizes `stream` and reads the workspace's device
  * status word.  Returns W4A16_ERR_DEVICE if any earlier w4a16_gemm with this
  * workspace gave up waiting for its weight tiles (bounded waits, about 2 s),

@@ -177,3 +177,27 @@ def test_search_validation(lib):
     assert call(nbytes=need - 1) == ERR_WORKSPACE
     assert "workspace" in _err(lib)
     assert best.value == -1
+
+
+def test_gptq_validation(lib):
+    """Every rejection happens before anything is enqueued (no GPU needed)."""
+    h = lib.gptq_hessian
+    assert h(None, 10, 128, 0.01, A, None) == ERR_ARG
+    assert h(A, 0, 128, 0.01, A, None) == ERR_ARG
+    assert h(A, 10, 128, -1.0, A, None) == ERR_ARG
+    assert h(A, 10, 128, float("nan"), A, None) == ERR_ARG
+    assert h(A, 10, 32768 + 128, 0.01, A, None) == ERR_SHAPE
+    assert h(MIS, 10, 128, 0.01, A, None) == ERR_ALIGN
+    ws = lib.gptq_sweep_workspace_size
+    assert ws(100, 256, 128) >= 100 * 256 * 9
+    assert ws(100, 200, 128) == 0 and ws(100, 256, 64) == 0 and ws(0, 256, 128) == 0
+    assert ws(1, 32768 + 128, 128) == 0
+    f = lib.gptq_sweep
+    need = ws(64, 256, 128)
+    assert f(None, A, 64, 256, 128, 4, 0, A, A, A, B, need, None) == ERR_ARG
+    assert f(A, A, 64, 256, 128, 4, 5, A, A, A, B, need, None) == ERR_ARG
+    assert f(A, A, 64, 256, 64, 4, 0, A, A, A, B, need, None) == ERR_UNSUPPORTED
+    assert f(A, A, 64, 256, 128, 2, 0, A, A, A, B, need, None) == ERR_UNSUPPORTED
+    assert f(A, A, 64, 200, 128, 4, 0, A, A, A, B, need, None) == ERR_SHAPE
+    assert f(A, MIS, 64, 256, 128, 4, 0, A, A, A, B, need, None) == ERR_ALIGN
+    assert f(A, A, 64, 256, 128, 4, 0, A, A, A, B, need - 1, None) == ERR_WORKSPACE

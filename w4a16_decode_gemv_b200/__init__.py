@@ -57,6 +57,12 @@ def load_library():
     lib.awq_search_workspace_size.restype = sz
     lib.awq_search_alpha.argtypes = [vp, vp, i, i, i, vp, i, i, i, i, vp, vp, vp, sz, vp]
     lib.awq_search_alpha.restype = i
+    lib.gptq_hessian.argtypes = [vp, i, i, d, vp, vp]
+    lib.gptq_hessian.restype = i
+    lib.gptq_sweep_workspace_size.argtypes = [i, i, i]
+    lib.gptq_sweep_workspace_size.restype = sz
+    lib.gptq_sweep.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
+    lib.gptq_sweep.restype = i
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
     lib.w4a16_wait_timeout_selftest.argtypes = [vp, i, vp]
@@ -275,6 +281,55 @@ def awq_search_alpha(W: torch.Tensor, X: torch.Tensor, alphas, group: int = GROU
                                     workspace.numel() * workspace.element_size(), _stream(W.device)),
                "awq_search_alpha")
     return [losses[i] for i in range(n)], best.value
+
+
+def gptq_hessian(X: torch.Tensor, damp: float = 0.01, out: torch.Tensor | None = None) -> torch.Tensor:
+    """H fp64 [K, K] = 2 X^T X + damp * mean(diag(2 X^T X)) I for calibration tokens X fp16 [T, K]."""
+    lib = load_library()
+    if X.dim() != 2:
+        raise W4A16Error("X must be 2-D [T, K]")
+    T, K = X.shape
+    _expect(X, torch.float16, (T, K), "X")
+    H = torch.empty((K, K), dtype=torch.float64, device=X.device) if out is None else out
+    _expect(H, torch.float64, (K, K), "out")
+    with torch.cuda.device(X.device):
+        _check(lib.gptq_hessian(_ptr(X), T, K, float(damp), _ptr(H), _stream(X.device)), "gptq_hessian")
+    return H
+
+
+def gptq_sweep(W: torch.Tensor, G: torch.Tensor, group: int = GROUP, bits: int = 4, mode: int = ASYM,
+               workspace: torch.Tensor | None = None, out=None):
+    """GPTQ's column sweep of W fp16 [N, K] with the upper Cholesky factor G fp64 [K, K] of H^-1.
+
+    Returns (qweight int32 [N, K/8] in layout v1, scales fp16, zeros fp16), as awq_quantize_pack.
+    """
+    lib = load_library()
+    if W.dim() != 2:
+        raise W4A16Error("W must be 2-D [N, K]")
+    N, K = W.shape
+    _expect(W, torch.float16, (N, K), "W")
+    _expect(G, torch.float64, (K, K), "G")
+    if group <= 0 or K % group:
+        raise W4A16Error(f"K={K} must be a multiple of group={group}")
+    if out is None:
+        qweight = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+        scales = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+        zeros = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+    else:
+        qweight, scales, zeros = out
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(scales, torch.float16, (N, K // group), "scales")
+    _expect(zeros, torch.float16, (N, K // group), "zeros")
+    if workspace is None:
+        need = int(lib.gptq_sweep_workspace_size(N, K, group))
+        if need == 0:
+            raise W4A16Error(f"unsupported sizes N={N} K={K} group={group}")
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib.gptq_sweep(_ptr(W), _ptr(G), N, K, group, bits, mode, _ptr(qweight), _ptr(scales), _ptr(zeros),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(W.device)),
+               "gptq_sweep")
+    return qweight, scales, zeros
 
 
 def wait_timeout_selftest(workspace: torch.Tensor, limit_us: int = 1000) -> None:

@@ -337,6 +337,49 @@ w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T,
   return ok();
 }
 
+w4a16_status gptq_hessian(const void* X, int T, int K, double damp, double* H, w4a16_stream_t stream) {
+  if (!X || !H) return fail(W4A16_ERR_ARG, "gptq_hessian: null pointer");
+  if (T < 1 || K < 1) return fail(W4A16_ERR_ARG, "gptq_hessian: T=%d K=%d must be >= 1", T, K);
+  if (!std::isfinite(damp) || damp < 0) return fail(W4A16_ERR_ARG, "gptq_hessian: damp must be finite and >= 0");
+  if (K > kMaxGptqK) return fail(W4A16_ERR_SHAPE, "gptq_hessian: K=%d (at most %d)", K, kMaxGptqK);
+  if (static_cast<long long>(T) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "gptq_hessian: T*K too large");
+  if (!aligned16(X) || !aligned16(H)) return fail(W4A16_ERR_ALIGN, "gptq_hessian: pointers must be 16-byte aligned");
+  const cudaError_t e = launch_gptq_hessian(static_cast<const __half*>(X), T, K, damp, H,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gptq_hessian launch");
+  return ok();
+}
+
+size_t gptq_sweep_workspace_size(int N, int K, int group) {
+  if (N < 1 || K < 1 || group != kGroup || K % group || K > kMaxGptqK) return 0;
+  if (static_cast<long long>(N) * K >= kMaxElems) return 0;
+  return gptq_sweep_workspace_bytes(N, K);
+}
+
+w4a16_status gptq_sweep(const void* W, const double* G, int N, int K, int group, int bits, w4a16_mode mode,
+                        uint32_t* qweight, void* scales, void* zeros, void* workspace, size_t workspace_bytes_,
+                        w4a16_stream_t stream) {
+  if (!W || !G || !qweight || !scales || !zeros || !workspace) return fail(W4A16_ERR_ARG, "gptq_sweep: null pointer");
+  if (N < 1 || K < 1) return fail(W4A16_ERR_ARG, "gptq_sweep: N=%d K=%d must be >= 1", N, K);
+  if (mode != W4A16_ASYM && mode != W4A16_SYM) return fail(W4A16_ERR_ARG, "gptq_sweep: bad mode %d", mode);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "gptq_sweep: group=%d (only 128)", group);
+  if (bits != 3 && bits != 4) return fail(W4A16_ERR_UNSUPPORTED, "gptq_sweep: bits=%d (3 or 4)", bits);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "gptq_sweep: K=%d not a multiple of group=%d", K, group);
+  if (K > kMaxGptqK) return fail(W4A16_ERR_SHAPE, "gptq_sweep: K=%d (at most %d)", K, kMaxGptqK);
+  if (static_cast<long long>(N) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "gptq_sweep: N*K too large");
+  if (!aligned16(W) || !aligned16(G) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      !aligned16(workspace))
+    return fail(W4A16_ERR_ALIGN, "gptq_sweep: pointers must be 16-byte aligned");
+  const size_t need = gptq_sweep_workspace_bytes(N, K);
+  if (workspace_bytes_ < need)
+    return fail(W4A16_ERR_WORKSPACE, "gptq_sweep: workspace of %zu bytes needed, %zu given", need, workspace_bytes_);
+  const cudaError_t e = launch_gptq_sweep(static_cast<const __half*>(W), G, N, K, bits, static_cast<int>(mode),
+                                          qweight, static_cast<__half*>(scales), static_cast<__half*>(zeros),
+                                          workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gptq_sweep launch");
+  return ok();
+}
+
 w4a16_status w4a16_wait_timeout_selftest(void* workspace, int limit_us, w4a16_stream_t stream) {
   if (!workspace || !aligned16(workspace))
     return fail(W4A16_ERR_ARG, "w4a16_wait_timeout_selftest: workspace must be non-null and 16-byte aligned");

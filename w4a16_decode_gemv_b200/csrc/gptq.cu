@@ -1,0 +1,277 @@
+// GPTQ on the GPU: the damped Hessian and the error-compensating column sweep.
+//
+// "CMU 11-868 LLM Systems: Model Quantization" reading guide, §L20 "GPTQ":
+// quantize one column block at a time; after each column, push its rounding
+// error, divided by the diagonal element of G = Cholesky((2 X X^T + lambda I)^-1)^T,
+// onto the rest of the block, and after the block onto every column right of
+// it; the columns go in a fixed order.  "Learning-ML-DL ch. 11", §11.4: H = 2 X X^T
+// is the Hessian of the output error of each weight row, damped by a fraction
+// of its mean diagonal.
+//
+// Everything is float64 with one rounding per product, sum, difference and
+// quotient (the _rn intrinsics), in this order:
+//   group (block of 128 columns) parameters from the block as the sweep
+//   reaches it: Delta = fp16((max - min) / (2^N - 1)), z = clamp(rint(-min / Delta));
+//   column i: u = clamp(rint(w / Delta) + z), e = (w - (u - z) Delta) / G[i][i],
+//   later columns j of the block: w_j - e G[i][j];
+//   after the block, columns j right of it: w_j - (sum over the block's i, in
+//   order, of e_i G[i][j]).
+// Given the same G, the codes, steps and zero points are therefore the same
+// bits whatever the launch shape.  Rows are independent: a warp sweeps a row
+// block by block, and the update right of the block is a separate kernel.
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+namespace {
+
+// ---- H = 2 X^T X (+ lambda I, added by gptq_damp_kernel) -----------------------
+// 64 x 64 tiles of H, 4 x 4 per thread, tokens in chunks of 16 staged in shared
+// memory.  The fp16 products are exact in fp64; each entry adds them in token order.
+constexpr int kHTile = 64;
+constexpr int kHChunk = 16;
+
+__global__ void __launch_bounds__(256) gptq_hessian_kernel(const __half* __restrict__ X, int T, int K,
+                                                           double* __restrict__ H) {
+  __shared__ double xa[kHChunk][kHTile];
+  __shared__ double xb[kHChunk][kHTile];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int i0 = blockIdx.y * kHTile, j0 = blockIdx.x * kHTile;
+  double acc[4][4] = {};
+  for (int t0 = 0; t0 < T; t0 += kHChunk) {
+    for (int e = threadIdx.x; e < kHChunk * kHTile; e += 256) {
+      const int c = e % kHTile, t = e / kHTile;
+      const bool in_t = t0 + t < T;
+      xa[t][c] = (in_t && i0 + c < K) ? static_cast<double>(__half2float(X[static_cast<size_t>(t0 + t) * K + i0 + c])) : 0.0;
+      xb[t][c] = (in_t && j0 + c < K) ? static_cast<double>(__half2float(X[static_cast<size_t>(t0 + t) * K + j0 + c])) : 0.0;
+    }
+    __syncthreads();
+    for (int t = 0; t < kHChunk; ++t) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = __dadd_rn(acc[a][b], __dmul_rn(xa[t][ty * 4 + a], xb[t][tx * 4 + b]));
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty * 4 + a;
+    if (i >= K) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + tx * 4 + b;
+      if (j < K) H[static_cast<size_t>(i) * K + j] = 2.0 * acc[a][b];
+    }
+  }
+}
+
+// lambda = damp * (mean of the diagonal), the diagonal added in index order by one thread.
+__global__ void gptq_damp_kernel(double* __restrict__ H, int K, double damp) {
+  __shared__ double lam;
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < K; ++i) s = __dadd_rn(s, H[static_cast<size_t>(i) * K + i]);
+    lam = __dmul_rn(damp, __ddiv_rn(s, static_cast<double>(K)));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    double* d = H + static_cast<size_t>(i) * K + i;
+    *d = __dadd_rn(*d, lam);
+  }
+}
+
+// ---- the sweep of one block of 128 columns ---------------------------------------
+// A warp per row; lane l holds columns b0 + l + 32 m, m = 0..3.  The warp writes
+// the row's codes (bytes), the block's errors e and the group's Delta and z.
+constexpr int kGroupCols = 128;
+constexpr int kSweepRows = 8;  // warps (rows) per CTA
+
+struct SweepArgs {
+  const __half* W;      // [N][K] fp16, read for the first block
+  double* Wc;           // [N][K] working copy (columns right of the current block)
+  const double* G;      // [K][K] upper-triangular factor
+  uint8_t* codes;       // [N][K]
+  double* errs;         // [N][128] the current block's e
+  __half* scales;       // [N][K/128]
+  __half* zeros;
+  int N, K, bits, mode;
+};
+
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_min(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__global__ void __launch_bounds__(32 * kSweepRows) gptq_block_kernel(const SweepArgs a, int b0) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kSweepRows + (threadIdx.x >> 5);
+  if (r >= a.N) return;  // a whole warp leaves together
+  const size_t row = static_cast<size_t>(r) * a.K;
+  double w[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int j = b0 + lane + 32 * m;
+    w[m] = b0 == 0 ? static_cast<double>(__half2float(a.W[row + j])) : a.Wc[row + j];
+  }
+  // group parameters from the block as it stands (max and min are exact)
+  const double qmax = static_cast<double>((1 << a.bits) - 1);
+  double d, z;
+  if (a.mode == 0) {
+    const double mx = warp_max(fmax(fmax(w[0], w[1]), fmax(w[2], w[3])));
+    const double mn = warp_min(fmin(fmin(w[0], w[1]), fmin(w[2], w[3])));
+    __half dh = __double2half(__ddiv_rn(__dsub_rn(mx, mn), qmax));
+    if (__half2float(dh) == 0.0f) dh = __double2half(__ddiv_rn(1.0, qmax));
+    d = static_cast<double>(__half2float(dh));
+    z = fmin(fmax(rint(__ddiv_rn(-mn, d)), 0.0), qmax) + 0.0;
+  } else {
+    const double amax = warp_max(fmax(fmax(fabs(w[0]), fabs(w[1])), fmax(fabs(w[2]), fabs(w[3]))));
+    const double half = static_cast<double>(1 << (a.bits - 1));
+    __half dh = __double2half(__ddiv_rn(amax, half));
+    if (__half2float(dh) == 0.0f) dh = __double2half(__ddiv_rn(1.0, half));
+    d = static_cast<double>(__half2float(dh));
+    z = half;
+  }
+  if (lane == 0) {
+    const size_t g = static_cast<size_t>(r) * (a.K / kGroupCols) + b0 / kGroupCols;
+    a.scales[g] = __double2half(d);
+    a.zeros[g] = __double2half(z);
+  }
+  // the columns of the block, left to right
+  for (int i = 0; i < kGroupCols; ++i) {
+    const int owner = i & 31, slot = i >> 5;
+    const double wi = __shfl_sync(0xffffffffu, slot == 0 ? w[0] : slot == 1 ? w[1] : slot == 2 ? w[2] : w[3], owner);
+    const double u = fmin(fmax(__dadd_rn(rint(__ddiv_rn(wi, d)), z), 0.0), qmax);
+    const double gii = __ldg(a.G + static_cast<size_t>(b0 + i) * a.K + b0 + i);
+    const double e = __ddiv_rn(__dsub_rn(wi, __dmul_rn(__dsub_rn(u, z), d)), gii);
+    if (lane == owner) {
+      a.codes[row + b0 + i] = static_cast<uint8_t>(u);
+      a.errs[static_cast<size_t>(r) * kGroupCols + i] = e;
+    }
+    const double* gi = a.G + static_cast<size_t>(b0 + i) * a.K + b0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = lane + 32 * m;  // column within the block
+      if (c > i) w[m] = __dsub_rn(w[m], __dmul_rn(e, __ldg(gi + c)));
+    }
+  }
+}
+
+// ---- the block's corrections to every column right of it ------------------------
+// Wc[r][j] -= sum_i e[r][i] G[b0 + i][j], i = 0..127 added in order.  64 x 64
+// tiles of (rows, columns), 4 x 4 per thread; e and G staged 16 columns of the
+// block at a time.  For the first block, the columns come from W itself.
+constexpr int kUTile = 64;
+constexpr int kUChunk = 16;
+
+__global__ void __launch_bounds__(256) gptq_update_kernel(const SweepArgs a, int b0) {
+  __shared__ double es[kUChunk][kUTile];  // [i][row]
+  __shared__ double gs[kUChunk][kUTile];  // [i][column]
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int r0 = blockIdx.x * kUTile;
+  const int b1 = b0 + kGroupCols;
+  const int j0 = b1 + blockIdx.y * kUTile;
+  double acc[4][4] = {};
+  for (int i0 = 0; i0 < kGroupCols; i0 += kUChunk) {
+    for (int e = threadIdx.x; e < kUChunk * kUTile; e += 256) {
+      const int c = e % kUTile, i = e / kUTile;
+      es[i][c] = r0 + c < a.N ? a.errs[static_cast<size_t>(r0 + c) * kGroupCols + i0 + i] : 0.0;
+      gs[i][c] = j0 + c < a.K ? a.G[static_cast<size_t>(b0 + i0 + i) * a.K + j0 + c] : 0.0;
+    }
+    __syncthreads();
+    for (int i = 0; i < kUChunk; ++i) {
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = __dadd_rn(acc[p][q], __dmul_rn(es[i][ty * 4 + p], gs[i][tx * 4 + q]));
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int r = r0 + ty * 4 + p;
+    if (r >= a.N) continue;
+    const size_t row = static_cast<size_t>(r) * a.K;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + tx * 4 + q;
+      if (j >= a.K) continue;
+      const double w = b0 == 0 ? static_cast<double>(__half2float(a.W[row + j])) : a.Wc[row + j];
+      a.Wc[row + j] = __dsub_rn(w, acc[p][q]);
+    }
+  }
+}
+
+// ---- codes -> layout v1 ------------------------------------------------------------
+// Word (n, j) holds inputs 8j + i; nibble slot p holds i = {0, 2, 4, 6, 1, 3, 5, 7}[p].
+__global__ void gptq_pack_kernel(const uint8_t* __restrict__ codes, long long words, uint32_t* __restrict__ qweight) {
+  for (long long wi = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; wi < words;
+       wi += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint8_t* c = codes + wi * 8;
+    qweight[wi] = static_cast<uint32_t>(c[0]) | (static_cast<uint32_t>(c[2]) << 4) | (static_cast<uint32_t>(c[4]) << 8) |
+                  (static_cast<uint32_t>(c[6]) << 12) | (static_cast<uint32_t>(c[1]) << 16) |
+                  (static_cast<uint32_t>(c[3]) << 20) | (static_cast<uint32_t>(c[5]) << 24) |
+                  (static_cast<uint32_t>(c[7]) << 28);
+  }
+}
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace
+
+cudaError_t launch_gptq_hessian(const __half* X, int T, int K, double damp, double* H, cudaStream_t st) {
+  const dim3 grid((K + kHTile - 1) / kHTile, (K + kHTile - 1) / kHTile);
+  gptq_hessian_kernel<<<grid, 256, 0, st>>>(X, T, K, H);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gptq_damp_kernel<<<1, 256, 0, st>>>(H, K, damp);
+  return cudaGetLastError();
+}
+
+size_t gptq_sweep_workspace_bytes(int N, int K) {
+  return align256(static_cast<size_t>(N) * K * 8) + align256(static_cast<size_t>(N) * K) +
+         align256(static_cast<size_t>(N) * kGroupCols * 8);
+}
+
+cudaError_t launch_gptq_sweep(const __half* W, const double* G, int N, int K, int bits, int mode, uint32_t* qweight,
+                              __half* scales, __half* zeros, void* workspace, cudaStream_t st) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SweepArgs a;
+  a.W = W;
+  a.G = G;
+  a.Wc = reinterpret_cast<double*>(ws);
+  a.codes = ws + align256(static_cast<size_t>(N) * K * 8);
+  a.errs = reinterpret_cast<double*>(a.codes + align256(static_cast<size_t>(N) * K));
+  a.scales = scales;
+  a.zeros = zeros;
+  a.N = N;
+  a.K = K;
+  a.bits = bits;
+  a.mode = mode;
+  const int sweep_grid = (N + kSweepRows - 1) / kSweepRows;
+  for (int b0 = 0; b0 < K; b0 += kGroupCols) {
+    gptq_block_kernel<<<sweep_grid, 32 * kSweepRows, 0, st>>>(a, b0);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int right = K - (b0 + kGroupCols);
+    if (right > 0) {
+      const dim3 grid((N + kUTile - 1) / kUTile, (right + kUTile - 1) / kUTile);
+      gptq_update_kernel<<<grid, 256, 0, st>>>(a, b0);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+  }
+  const long long words = static_cast<long long>(N) * (K / 8);
+  const long long blocks = (words + 255) / 256;
+  const int pgrid = static_cast<int>(blocks < 8 * device_sm_count() ? blocks : 8 * device_sm_count());
+  gptq_pack_kernel<<<pgrid, 256, 0, st>>>(a.codes, words, qweight);
+  return cudaGetLastError();
+}
+
+}  // namespace w4a16

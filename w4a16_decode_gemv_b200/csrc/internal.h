@@ -95,6 +95,16 @@ cudaError_t launch_divide_activation(const __half* X, const __half* s, int T, in
 cudaError_t launch_squared_error(const __half* Yq, const float* Y, long long total, double* partial, cudaStream_t st);
 cudaError_t launch_sum_partials(const double* partial, int n_alpha, double* sums, cudaStream_t st);
 
+// GPTQ (gptq.cu): H = 2 X^T X + damp * mean(diag) I in fp64 [K][K]; the column
+// sweep with a given upper-triangular factor G, writing layout-v1 codes, Delta
+// and z; the sweep's workspace: the fp64 working copy of W, the codes and one
+// block of errors.
+constexpr int kMaxGptqK = 32768;
+cudaError_t launch_gptq_hessian(const __half* X, int T, int K, double damp, double* H, cudaStream_t st);
+size_t gptq_sweep_workspace_bytes(int N, int K);
+cudaError_t launch_gptq_sweep(const __half* W, const double* G, int N, int K, int bits, int mode, uint32_t* qweight,
+                              __half* scales, __half* zeros, void* workspace, cudaStream_t st);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
