@@ -1,6 +1,7 @@
 """Plant plausible mistakes in a copy of the oracle and check that the pins in
-test_oracle.py (quantizer, packing, GEMM) and test_oracle_gptq.py (GPTQ)
-catch every one of them.  CPU only; the real oracle is untouched."""
+test_oracle.py (quantizer, packing, GEMM), test_oracle_gptq.py (GPTQ) and
+test_oracle_search.py (the alpha search) catch every one of them.  CPU only;
+the real oracle is untouched."""
 import os
 import shutil
 import subprocess
@@ -47,9 +48,22 @@ MUTANTS = {
                                  "d16, z16 = group_params(np.asarray(W, dtype=F16)[:, b0:b1], bits, mode, group)",
                                  "gptq"),
     "gptq_code_from_original": ("w = Wc[:, i].copy()", "w = np.asarray(W, dtype=F16)[:, i].astype(F64)", "gptq"),
+    # alpha search: caught by tests/test_oracle_search.py
+    "search_multiplies_activation": ("return (X / np.asarray(s, dtype=F16).astype(F64)[None, :]).astype(F16)",
+                                     "return (X * np.asarray(s, dtype=F16).astype(F64)[None, :]).astype(F16)",
+                                     "search"),
+    "search_output_not_rounded": ("y_q = (divide_activation(X, s).astype(F64) @ w_hat.T).astype(F16).astype(F64)",
+                                  "y_q = divide_activation(X, s).astype(F64) @ w_hat.T", "search"),
+    "search_target_divided": ("y = np.asarray(X, dtype=F16).astype(F64) @ np.asarray(W, dtype=F16).astype(F64).T",
+                              "y = divide_activation(X, s).astype(F64) @ np.asarray(W, dtype=F16).astype(F64).T",
+                              "search"),
+    "search_argmax": ("return losses, int(np.argmin(losses))", "return losses, int(np.argmax(losses))", "search"),
+    "search_sum_not_mean": ("return float(np.mean((y_q - y) ** 2))", "return float(np.sum((y_q - y) ** 2))",
+                            "search"),
+    "search_alpha_ignored": ("s = act_scale(X, alpha)", "s = act_scale(X, 0.5)", "search"),
 }
 
-PIN_FILES = {None: "tests/test_oracle.py", "gptq": "tests/test_oracle_gptq.py"}
+PIN_FILES = {None: "tests/test_oracle.py", "gptq": "tests/test_oracle_gptq.py", "search": "tests/test_oracle_search.py"}
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
