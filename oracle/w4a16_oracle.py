@@ -34,6 +34,12 @@ Pages cited (by title and section):
   setup: calibration statistic = mean |X| per input channel over 512-token
   blocks; pseudo quantization (quantize, then dequantize at once); 3-bit,
   group 128.
+* [L13] §QServe (slides 47-57; also the lecture summary of the same guide):
+  the W4A8 setting -- 4-bit per-group weights, 8-bit per-token activations,
+  INT8 tensor cores with the float conversion delayed to the end of the
+  accumulation -- and progressive quantization, whose dequantization
+  multiplies by the group scale before subtracting the zero point so that the
+  register-level (packed byte) arithmetic cannot overflow.
 * [ML11] "Learning-ML-DL ch. 11: Quantization for LLMs"
   (hoangvt2501.github.io).  §11.3: Y = (X diag(s)^-1)(W diag(s))^T;
   §11.4: AWQ's s = s_X^alpha with s_X the mean channel magnitude; GPTQ's
@@ -85,6 +91,29 @@ Readings of points the pages leave open:
 13. G = Cholesky(H^-1)^T is the upper-triangular factor with H^-1 = G^T G and
    a positive diagonal ([CMU] L20 step 1); it is computed by numpy's Cholesky
    of numpy's inverse.
+14. W4A8 level 1 (per output channel, symmetric INT8): s1 = fp16(max|W| / 119),
+   w8 = clamp(Round(W / s1), -119, 119); a zero row takes s1 = fp16(1/119).
+   119 is the largest R with R + ceil(2R / 15) / 2 <= 127: the level-2 values
+   of a range within [-R, R] then dequantize inside int8 (see 15).  The pages
+   ask only that the dequantization not overflow.
+15. W4A8 level 2 (per group of 128 along K, asymmetric INT4 with integer
+   step), over the group's range widened to include 0 (mn = min(min w8, 0),
+   mx = max(max w8, 0)): s2 = max(1, ceil((mx - mn) / 15)) <= 16,
+   z2 = Round(-mn / s2) (in [0, 15] without clamping), u = clamp(Round(w8 / s2)
+   + z2, 0, 15).  Without the widening, a group far from zero (all values near
+   -119, say) would take a small step and a clamped zero point and dequantize
+   far from its values; with it every value lands within half a step.
+   stored as layout-v1 codes, s2 (uint8) and the scaled zero zs = z2 * s2
+   (uint8 <= 240).  Progressive dequantization: w8_hat = u * s2 - zs, where
+   u * s2 <= 240 fits an unsigned byte, so four codes packed in a 32-bit word
+   are scaled by one integer multiply and the zero removed by a bytewise
+   subtraction.
+16. W4A8 activations (per token, symmetric INT8): s_x = fp16(max|x| / 127),
+   x8 = clamp(Round(x / s_x), -127, 127); a zero row takes s_x = fp16(1/127).
+   The quotient of two fp16 values never lies within 2^-19 (relative) of a
+   half-integer unless it is one, so an fp32 quotient rounds to the same x8.
+17. W4A8 output: acc = sum_k x8 * w8_hat exactly (int64 here; it fits int32
+   for K < 133,000), y = fp16(acc * s_x * s1) with the product exact (fp64).
 
 Every function here is pinned by tests marked ``not gpu`` against closed
 forms, brute force, invariants the pages state, or special cases.
@@ -349,3 +378,57 @@ def gptq_quantize(W: np.ndarray, X: np.ndarray, group: int = 128, bits: int = 4,
     G = gptq_factor(gptq_hessian(X, damp))
     u, d, z, _ = gptq_sweep(W, G, group, bits, mode)
     return pack_v1(u), d, z
+
+
+# ---------------------------------------------------------------------------
+# W4A8 with progressive group quantization  ([L13] §QServe; readings 14-17)
+# ---------------------------------------------------------------------------
+W4A8_L1 = 119   # level-1 range (reading 14)
+W4A8_ACT = 127  # activation range (reading 16)
+
+
+def w4a8_level2_params(w8: np.ndarray, group: int = 128):
+    """Integer step s2 and zero point z2 of each group of int8 values (reading 15)."""
+    N, K = w8.shape
+    g = np.asarray(w8, dtype=np.int64).reshape(N, K // group, group)
+    mx, mn = np.maximum(g.max(axis=-1), 0), np.minimum(g.min(axis=-1), 0)
+    s2 = np.maximum(1, -((mn - mx) // 15))            # ceil((mx - mn) / 15) in integers
+    z2 = np.clip(np.rint(-mn / s2), 0, 15).astype(np.int64)  # exact rationals of small integers, ties to even
+    return s2, z2
+
+
+def w4a8_quantize_weight(W: np.ndarray, group: int = 128):
+    """(qweight u32[N, K/8] layout v1, s1 fp16[N], s2 uint8[N, K/group], zs uint8[N, K/group])."""
+    W64 = np.asarray(W, dtype=F16).astype(F64)
+    N, K = W64.shape
+    amax = np.abs(W64).max(axis=1)
+    s1 = (amax / W4A8_L1).astype(F16)
+    s1[s1 == 0] = F16(1.0 / W4A8_L1)
+    w8 = np.clip(np.rint(W64 / s1.astype(F64)[:, None]), -W4A8_L1, W4A8_L1).astype(np.int64)
+    s2, z2 = w4a8_level2_params(w8, group)
+    g = w8.reshape(N, K // group, group)
+    u = np.clip(np.rint(g / s2[..., None]) + z2[..., None], 0, 15).astype(np.uint8).reshape(N, K)
+    return pack_v1(u), s1, s2.astype(np.uint8), (z2 * s2).astype(np.uint8)
+
+
+def w4a8_dequant_int8(qweight: np.ndarray, s2: np.ndarray, zs: np.ndarray, group: int = 128) -> np.ndarray:
+    """w8_hat = u * s2 - zs as int64 [N, K] (the progressive order of reading 15)."""
+    u = unpack_v1(qweight).astype(np.int64)
+    return u * np.repeat(s2.astype(np.int64), group, axis=1) - np.repeat(zs.astype(np.int64), group, axis=1)
+
+
+def w4a8_quantize_act(x: np.ndarray):
+    """(x8 int8 [M, K], s_x fp16 [M]) per token (reading 16)."""
+    x64 = np.asarray(x, dtype=F16).astype(F64)
+    sx = (np.abs(x64).max(axis=1) / W4A8_ACT).astype(F16)
+    sx[sx == 0] = F16(1.0 / W4A8_ACT)
+    x8 = np.clip(np.rint(x64 / sx.astype(F64)[:, None]), -W4A8_ACT, W4A8_ACT).astype(np.int8)
+    return x8, sx
+
+
+def w4a8_gemm(x8, sx, qweight, s1, s2, zs, group: int = 128):
+    """(y fp16 [M, N], acc int64 [M, N]): acc = x8 . w8_hat^T exactly, y = fp16(acc s_x s1) (reading 17)."""
+    acc = np.asarray(x8, dtype=np.int64) @ w4a8_dequant_int8(qweight, s2, zs, group).T
+    y = (acc.astype(F64) * np.asarray(sx, dtype=F16).astype(F64)[:, None]
+         * np.asarray(s1, dtype=F16).astype(F64)[None, :]).astype(F16)
+    return y, acc

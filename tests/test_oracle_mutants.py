@@ -1,6 +1,7 @@
 """Plant plausible mistakes in a copy of the oracle and check that the pins in
-test_oracle.py (quantizer, packing, GEMM), test_oracle_gptq.py (GPTQ) and
-test_oracle_search.py (the alpha search) catch every one of them.  CPU only;
+test_oracle.py (quantizer, packing, GEMM), test_oracle_gptq.py (GPTQ),
+test_oracle_search.py (the alpha search) and test_oracle_w4a8.py (W4A8) catch
+every one of them.  CPU only;
 the real oracle is untouched."""
 import os
 import shutil
@@ -61,9 +62,19 @@ MUTANTS = {
     "search_sum_not_mean": ("return float(np.mean((y_q - y) ** 2))", "return float(np.sum((y_q - y) ** 2))",
                             "search"),
     "search_alpha_ignored": ("s = act_scale(X, alpha)", "s = act_scale(X, 0.5)", "search"),
+    # W4A8: caught by tests/test_oracle_w4a8.py
+    "w4a8_level1_range_127": ("W4A8_L1 = 119", "W4A8_L1 = 127", "w4a8"),
+    "w4a8_floor_step": ("s2 = np.maximum(1, -((mn - mx) // 15))", "s2 = np.maximum(1, (mx - mn) // 15)", "w4a8"),
+    "w4a8_unscaled_zero": ("(z2 * s2).astype(np.uint8)", "z2.astype(np.uint8)", "w4a8"),
+    "w4a8_range_without_zero": ("mx, mn = np.maximum(g.max(axis=-1), 0), np.minimum(g.min(axis=-1), 0)",
+                                "mx, mn = g.max(axis=-1), g.min(axis=-1)", "w4a8"),
+    "w4a8_activation_range_128": ("W4A8_ACT = 127", "W4A8_ACT = 128", "w4a8"),
+    "w4a8_output_without_s1": ("* np.asarray(s1, dtype=F16).astype(F64)[None, :]).astype(F16)",
+                               ").astype(F16)", "w4a8"),
 }
 
-PIN_FILES = {None: "tests/test_oracle.py", "gptq": "tests/test_oracle_gptq.py", "search": "tests/test_oracle_search.py"}
+PIN_FILES = {None: "tests/test_oracle.py", "gptq": "tests/test_oracle_gptq.py", "search": "tests/test_oracle_search.py",
+             "w4a8": "tests/test_oracle_w4a8.py"}
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
