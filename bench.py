@@ -247,6 +247,45 @@ def search_workload(Wd, Xd, dev, n_alpha=20, reps=3):
             "timing": f"CUDA events around the synchronous call, best of {reps}"}
 
 
+def gptq_workload(Wd, Xd, dev, reps=3):
+    """GPTQ's GPU steps on the 11008 x 4096 layer and its 512 calibration tokens: the
+    damped Hessian (gptq_hessian) and the column sweep (gptq_sweep).  The factor G is
+    the caller's step for now; here torch.linalg computes it, outside the timed calls."""
+    import torch
+
+    import w4a16_decode_gemv_b200 as w4
+    N, K = Wd.shape
+    T = Xd.shape[0]
+    H = w4.gptq_hessian(Xd)
+    G = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H)), upper=True).contiguous()
+    ws = torch.empty(int(w4.load_library().gptq_sweep_workspace_size(N, K, 128)), dtype=torch.uint8, device=dev)
+    out = (torch.empty((N, K // 8), dtype=torch.int32, device=dev),
+           torch.empty((N, K // 128), dtype=torch.float16, device=dev),
+           torch.empty((N, K // 128), dtype=torch.float16, device=dev))
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    h_ms = timed(lambda: w4.gptq_hessian(Xd, out=H))
+    s_ms = timed(lambda: w4.gptq_sweep(Wd, G, workspace=ws, out=out))
+    sweep_flop = N * K * K  # the updates right of each block: N K^2 / 2 multiply-add pairs
+    return {"N": N, "K": K, "T": T, "hessian_ms": round(h_ms, 4), "sweep_ms": round(s_ms, 3),
+            "sweep_fp64_tflops": round(sweep_flop / (s_ms * 1e-3) / 1e12, 2),
+            "hessian_fp64_tflops": round(2 * T * K * K / (h_ms * 1e-3) / 1e12, 2),
+            "timing": f"CUDA events, best of {reps}; the factor G from torch.linalg, not timed"}
+
+
 def run_ours(args, dist):
     import torch
 
@@ -518,13 +557,18 @@ def other_workloads(args, dev):
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries
-    if only is not None and only not in ("quantize_pack_11008x4096", "awq_search_11008x4096"):
+    if only is not None and only not in ("quantize_pack_11008x4096", "awq_search_11008x4096", "gptq_11008x4096"):
         return res
     W, X, _ = inputs.quant_workload()
     Wd = torch.from_numpy(W).to(dev)
     Xd = torch.from_numpy(X).to(dev)
     if only is None or only == "awq_search_11008x4096":
         res["awq_search_11008x4096"] = search_workload(Wd, Xd, dev)
+    if only is None or only == "gptq_11008x4096":
+        try:
+            res["gptq_11008x4096"] = gptq_workload(Wd, Xd, dev)
+        except Exception as e:  # report, never hide
+            res["gptq_11008x4096"] = {"error": str(e)[:300]}
     if only is not None and only != "quantize_pack_11008x4096":
         return res
     # quantize + pack of the 11008 x 4096 AWQ workload (4-bit asym and 3-bit sym)
@@ -636,7 +680,7 @@ def main():
     ap.add_argument("--only", default=None,
                     help="run one of the other workloads only (gemv_4096x4096, llama7b_decode, llama65b_decode, "
                          "skinny_8192 or skinny_8192:M, prefill_8192 or prefill_8192:M, quantize_pack_11008x4096, "
-                         "awq_search_11008x4096); for profiling")
+                         "awq_search_11008x4096, gptq_11008x4096); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
