@@ -250,11 +250,48 @@ W4A16_API size_t gptq_sweep_workspace_size(int N, int K, int group);
  *   N >= 1;  K a multiple of group, at most 32768;  group == 128;  bits in {3, 4}.
  *   workspace  at least gptq_sweep_workspace_size(N, K, group) bytes, any
  *              contents (an fp64 copy of W, the codes and one block of errors).
- * Asynchronous on `stream`.  Computing G from H is the caller's for now.
+ * Asynchronous on `stream`.  G comes from gptq_factor (or the caller).
  */
 W4A16_API w4a16_status gptq_sweep(const void* W, const double* G, int N, int K, int group, int bits,
                                   w4a16_mode mode, uint32_t* qweight, void* scales, void* zeros,
                                   void* workspace, size_t workspace_bytes, w4a16_stream_t stream);
+
+/* gptq_factor_workspace_size -- bytes of workspace gptq_factor needs (2 K^2 fp64); 0 for invalid K. */
+W4A16_API size_t gptq_factor_workspace_size(int K);
+
+/*
+ * gptq_factor -- G = Cholesky(H^-1)^T, the upper-triangular factor with
+ * H^-1 = G^T G and a positive diagonal ([CMU] §L20 "GPTQ", step 1).
+ *
+ * With P the reversal of the index order, P H P = L L^T (Cholesky, left-looking,
+ * fp64), and G = P L^-1 P (triangular inverse by forward substitution, fp64):
+ * U = P L P is upper triangular with H = U U^T, so G = U^-1 satisfies
+ * G^T G = H^-1 and, being upper triangular with a positive diagonal, is that
+ * factor.  The sums run over warp lanes: G agrees with other implementations
+ * to rounding (about 1e-12 relative at K = 4096), not bit for bit.  The call
+ * enqueues 2K + 2 kernel launches (offline use).
+ *
+ *   H  fp64 [K][K] symmetric positive definite, device (gptq_hessian's output).
+ *   G  fp64 [K][K], device (output; the lower triangle is written as zeros).
+ *   1 <= K <= 32768;  workspace  gptq_factor_workspace_size(K) bytes, any contents.
+ */
+W4A16_API w4a16_status gptq_factor(const double* H, int K, double* G, void* workspace,
+                                   size_t workspace_bytes, w4a16_stream_t stream);
+
+/* gptq_quantize_workspace_size -- bytes of workspace gptq_quantize needs; 0 for invalid sizes. */
+W4A16_API size_t gptq_quantize_workspace_size(int N, int K, int group);
+
+/*
+ * gptq_quantize -- GPTQ end to end: gptq_hessian(X, damp), gptq_factor, then
+ * gptq_sweep(W, G), all on `stream`, into qweight / scales / zeros (layout v1,
+ * the format w4a16_gemm reads).  Arguments as for those calls; T is the number
+ * of calibration tokens in X (fp16 [T][K]).  The workspace (any contents) holds
+ * H, G and the scratch of the factor and of the sweep.
+ */
+W4A16_API w4a16_status gptq_quantize(const void* W, const void* X, int N, int K, int T, double damp,
+                                     int group, int bits, w4a16_mode mode, uint32_t* qweight,
+                                     void* scales, void* zeros, void* workspace,
+                                     size_t workspace_bytes, w4a16_stream_t stream);
 
 /*
  * w4a16_gemm_check -- synchronizes `stream` and reads the workspace's device

@@ -201,3 +201,33 @@ def test_gptq_validation(lib):
     assert f(A, A, 64, 200, 128, 4, 0, A, A, A, B, need, None) == ERR_SHAPE
     assert f(A, MIS, 64, 256, 128, 4, 0, A, A, A, B, need, None) == ERR_ALIGN
     assert f(A, A, 64, 256, 128, 4, 0, A, A, A, B, need - 1, None) == ERR_WORKSPACE
+
+
+def test_gptq_factor_and_quantize_validation(lib):
+    """Every rejection happens before anything is enqueued (no GPU needed)."""
+    fws = lib.gptq_factor_workspace_size
+    assert fws(4096) >= 2 * 4096 * 4096 * 8 and fws(0) == 0 and fws(32768 + 1) == 0
+    f = lib.gptq_factor
+    assert f(None, 256, A, B, fws(256), None) == ERR_ARG
+    assert f(A, 0, A, B, fws(256), None) == ERR_ARG
+    assert f(A, 40000, A, B, 1 << 40, None) == ERR_SHAPE
+    assert f(MIS, 256, A, B, fws(256), None) == ERR_ALIGN
+    assert f(A, 256, A, B, fws(256) - 1, None) == ERR_WORKSPACE
+    qws = lib.gptq_quantize_workspace_size
+    assert qws(64, 256, 128) > fws(256) + lib.gptq_sweep_workspace_size(64, 256, 128)
+    assert qws(64, 200, 128) == 0 and qws(64, 256, 64) == 0
+    q = lib.gptq_quantize
+    need = qws(64, 256, 128)
+
+    def call(W=A, X=A, N=64, K=256, T=10, damp=0.01, group=128, bits=4, mode=0, ws=B, nbytes=need):
+        return q(W, X, N, K, T, damp, group, bits, mode, A, A, A, ws, nbytes, None)
+
+    assert call(X=None) == ERR_ARG
+    assert call(T=0) == ERR_ARG
+    assert call(damp=float("inf")) == ERR_ARG
+    assert call(mode=2) == ERR_ARG
+    assert call(group=32) == ERR_UNSUPPORTED
+    assert call(bits=5) == ERR_UNSUPPORTED
+    assert call(K=200) == ERR_SHAPE
+    assert call(X=MIS) == ERR_ALIGN
+    assert call(nbytes=need - 1) == ERR_WORKSPACE

@@ -63,6 +63,14 @@ def load_library():
     lib.gptq_sweep_workspace_size.restype = sz
     lib.gptq_sweep.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
     lib.gptq_sweep.restype = i
+    lib.gptq_factor_workspace_size.argtypes = [i]
+    lib.gptq_factor_workspace_size.restype = sz
+    lib.gptq_factor.argtypes = [vp, i, vp, vp, sz, vp]
+    lib.gptq_factor.restype = i
+    lib.gptq_quantize_workspace_size.argtypes = [i, i, i]
+    lib.gptq_quantize_workspace_size.restype = sz
+    lib.gptq_quantize.argtypes = [vp, vp, i, i, i, d, i, i, i, vp, vp, vp, vp, sz, vp]
+    lib.gptq_quantize.restype = i
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
     lib.w4a16_wait_timeout_selftest.argtypes = [vp, i, vp]
@@ -329,6 +337,61 @@ def gptq_sweep(W: torch.Tensor, G: torch.Tensor, group: int = GROUP, bits: int =
         _check(lib.gptq_sweep(_ptr(W), _ptr(G), N, K, group, bits, mode, _ptr(qweight), _ptr(scales), _ptr(zeros),
                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(W.device)),
                "gptq_sweep")
+    return qweight, scales, zeros
+
+
+def gptq_factor(H: torch.Tensor, workspace: torch.Tensor | None = None,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """G fp64 [K, K] = Cholesky(H^-1)^T for a symmetric positive definite H fp64 [K, K]."""
+    lib = load_library()
+    if H.dim() != 2 or H.shape[0] != H.shape[1]:
+        raise W4A16Error("H must be square [K, K]")
+    K = H.shape[0]
+    _expect(H, torch.float64, (K, K), "H")
+    G = torch.empty((K, K), dtype=torch.float64, device=H.device) if out is None else out
+    _expect(G, torch.float64, (K, K), "out")
+    if workspace is None:
+        need = int(lib.gptq_factor_workspace_size(K))
+        if need == 0:
+            raise W4A16Error(f"unsupported size K={K}")
+        workspace = torch.empty(need, dtype=torch.uint8, device=H.device)
+    with torch.cuda.device(H.device):
+        _check(lib.gptq_factor(_ptr(H), K, _ptr(G), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(H.device)), "gptq_factor")
+    return G
+
+
+def gptq_quantize(W: torch.Tensor, X: torch.Tensor, damp: float = 0.01, group: int = GROUP, bits: int = 4,
+                  mode: int = ASYM, workspace: torch.Tensor | None = None, out=None):
+    """GPTQ of W fp16 [N, K] with calibration tokens X fp16 [T, K]: the Hessian, its factor
+    and the column sweep on the GPU.  Returns (qweight int32 [N, K/8] layout v1, scales, zeros)."""
+    lib = load_library()
+    if W.dim() != 2 or X.dim() != 2:
+        raise W4A16Error("W must be [N, K] and X [T, K]")
+    N, K = W.shape
+    T = X.shape[0]
+    _expect(W, torch.float16, (N, K), "W")
+    _expect(X, torch.float16, (T, K), "X")
+    if group <= 0 or K % group:
+        raise W4A16Error(f"K={K} must be a multiple of group={group}")
+    if out is None:
+        qweight = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+        scales = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+        zeros = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+    else:
+        qweight, scales, zeros = out
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(scales, torch.float16, (N, K // group), "scales")
+    _expect(zeros, torch.float16, (N, K // group), "zeros")
+    if workspace is None:
+        need = int(lib.gptq_quantize_workspace_size(N, K, group))
+        if need == 0:
+            raise W4A16Error(f"unsupported sizes N={N} K={K} group={group}")
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib.gptq_quantize(_ptr(W), _ptr(X), N, K, T, float(damp), group, bits, mode, _ptr(qweight),
+                                 _ptr(scales), _ptr(zeros), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(W.device)), "gptq_quantize")
     return qweight, scales, zeros
 
 

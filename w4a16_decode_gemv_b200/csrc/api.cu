@@ -380,6 +380,70 @@ w4a16_status gptq_sweep(const void* W, const double* G, int N, int K, int group,
   return ok();
 }
 
+size_t gptq_factor_workspace_size(int K) {
+  if (K < 1 || K > kMaxGptqK) return 0;
+  return gptq_factor_workspace_bytes(K);
+}
+
+w4a16_status gptq_factor(const double* H, int K, double* G, void* workspace, size_t workspace_bytes_,
+                         w4a16_stream_t stream) {
+  if (!H || !G || !workspace) return fail(W4A16_ERR_ARG, "gptq_factor: null pointer");
+  if (K < 1) return fail(W4A16_ERR_ARG, "gptq_factor: K=%d must be >= 1", K);
+  if (K > kMaxGptqK) return fail(W4A16_ERR_SHAPE, "gptq_factor: K=%d (at most %d)", K, kMaxGptqK);
+  if (!aligned16(H) || !aligned16(G) || !aligned16(workspace))
+    return fail(W4A16_ERR_ALIGN, "gptq_factor: pointers must be 16-byte aligned");
+  const size_t need = gptq_factor_workspace_bytes(K);
+  if (workspace_bytes_ < need)
+    return fail(W4A16_ERR_WORKSPACE, "gptq_factor: workspace of %zu bytes needed, %zu given", need, workspace_bytes_);
+  const cudaError_t e = launch_gptq_factor(H, K, G, workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gptq_factor launch");
+  return ok();
+}
+
+// gptq_quantize's workspace: H, G, the factor's scratch, the sweep's, each 256-byte aligned.
+static size_t gptq_matrix_bytes(int K) { return (static_cast<size_t>(K) * K * 8 + 255) / 256 * 256; }
+
+size_t gptq_quantize_workspace_size(int N, int K, int group) {
+  if (gptq_sweep_workspace_size(N, K, group) == 0) return 0;
+  return 2 * gptq_matrix_bytes(K) + gptq_factor_workspace_bytes(K) + gptq_sweep_workspace_bytes(N, K);
+}
+
+w4a16_status gptq_quantize(const void* W, const void* X, int N, int K, int T, double damp, int group, int bits,
+                           w4a16_mode mode, uint32_t* qweight, void* scales, void* zeros, void* workspace,
+                           size_t workspace_bytes_, w4a16_stream_t stream) {
+  if (!W || !X || !qweight || !scales || !zeros || !workspace)
+    return fail(W4A16_ERR_ARG, "gptq_quantize: null pointer");
+  if (N < 1 || K < 1 || T < 1) return fail(W4A16_ERR_ARG, "gptq_quantize: N=%d K=%d T=%d must be >= 1", N, K, T);
+  if (!std::isfinite(damp) || damp < 0) return fail(W4A16_ERR_ARG, "gptq_quantize: damp must be finite and >= 0");
+  if (mode != W4A16_ASYM && mode != W4A16_SYM) return fail(W4A16_ERR_ARG, "gptq_quantize: bad mode %d", mode);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "gptq_quantize: group=%d (only 128)", group);
+  if (bits != 3 && bits != 4) return fail(W4A16_ERR_UNSUPPORTED, "gptq_quantize: bits=%d (3 or 4)", bits);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "gptq_quantize: K=%d not a multiple of group=%d", K, group);
+  if (K > kMaxGptqK) return fail(W4A16_ERR_SHAPE, "gptq_quantize: K=%d (at most %d)", K, kMaxGptqK);
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(T) * K >= kMaxElems)
+    return fail(W4A16_ERR_SHAPE, "gptq_quantize: N*K or T*K too large");
+  if (!aligned16(W) || !aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      !aligned16(workspace))
+    return fail(W4A16_ERR_ALIGN, "gptq_quantize: pointers must be 16-byte aligned");
+  const size_t need = gptq_quantize_workspace_size(N, K, group);
+  if (workspace_bytes_ < need)
+    return fail(W4A16_ERR_WORKSPACE, "gptq_quantize: workspace of %zu bytes needed, %zu given", need,
+                workspace_bytes_);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  double* H = reinterpret_cast<double*>(base);
+  double* G = reinterpret_cast<double*>(base + gptq_matrix_bytes(K));
+  void* fws = base + 2 * gptq_matrix_bytes(K);
+  void* sws = base + 2 * gptq_matrix_bytes(K) + gptq_factor_workspace_bytes(K);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_gptq_hessian(static_cast<const __half*>(X), T, K, damp, H, st);
+  if (e == cudaSuccess) e = launch_gptq_factor(H, K, G, fws, st);
+  if (e == cudaSuccess)
+    e = launch_gptq_sweep(static_cast<const __half*>(W), G, N, K, bits, static_cast<int>(mode), qweight,
+                          static_cast<__half*>(scales), static_cast<__half*>(zeros), sws, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gptq_quantize launch");
+  return ok();
+}
+
 w4a16_status w4a16_wait_timeout_selftest(void* workspace, int limit_us, w4a16_stream_t stream) {
   if (!workspace || !aligned16(workspace))
     return fail(W4A16_ERR_ARG, "w4a16_wait_timeout_selftest: workspace must be non-null and 16-byte aligned");

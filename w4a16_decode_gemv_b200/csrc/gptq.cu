@@ -221,9 +221,91 @@ __global__ void gptq_pack_kernel(const uint8_t* __restrict__ codes, long long wo
   }
 }
 
+// ---- the factor G = Cholesky(H^-1)^T ---------------------------------------------
+// With P the reversal of the index order, P H P = L L^T (Cholesky), U = P L P is
+// upper triangular with H = U U^T, and G = U^-1 = P L^-1 P is upper triangular
+// with a positive diagonal and G^T G = H^-1: by the uniqueness of the Cholesky
+// factorization it is the factor of [CMU] §L20 step 1.  fp64 throughout; the
+// sums run over warp lanes, so G matches numpy's to rounding (about 1e-12
+// relative at K = 4096), not bit for bit.
+
+// A[i][j] = H[K-1-i][K-1-j] on and below the diagonal, 0 above.
+__global__ void gptq_reverse_kernel(const double* __restrict__ H, int K, double* __restrict__ A) {
+  const long long n = static_cast<long long>(K) * K;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(e / K), j = static_cast<int>(e % K);
+    A[e] = j <= i ? H[static_cast<long long>(K - 1 - i) * K + (K - 1 - j)] : 0.0;
+  }
+}
+
+// Column j of L in place, left-looking, one warp per row: first the diagonal
+// (diag = true), L[j][j] = sqrt(A[j][j] - sum_k L[j][k]^2); then the rows below,
+// L[i][j] = (A[i][j] - sum_k L[i][k] L[j][k]) / L[j][j].
+__global__ void gptq_chol_col_kernel(double* __restrict__ L, int K, int j, bool diag) {
+  const int lane = threadIdx.x & 31;
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int i = diag ? j : j + 1 + w;
+  if (i >= K || (diag && w > 0)) return;
+  const double* li = L + static_cast<long long>(i) * K;
+  const double* lj = L + static_cast<long long>(j) * K;
+  double s = 0.0;
+  for (int k = lane; k < j; k += 32) s = fma(li[k], lj[k], s);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    double* d = L + static_cast<long long>(i) * K + j;
+    if (diag) *d = sqrt(*d - s);
+    else *d = (*d - s) / lj[j];
+  }
+}
+
+// Column c of X = L^-1 by forward substitution (one warp per column):
+// X[c][c] = 1 / L[c][c], X[i][c] = -(sum_{k=c}^{i-1} L[i][k] X[k][c]) / L[i][i];
+// written reversed into G: G[K-1-i][K-1-c] = X[i][c] (0 for i < c).
+__global__ void gptq_trinv_kernel(const double* __restrict__ L, int K, double* __restrict__ G,
+                                  double* __restrict__ scratch) {
+  const int lane = threadIdx.x & 31;
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (c >= K) return;
+  double* x = scratch + static_cast<long long>(c) * K;
+  if (lane == 0) x[c] = 1.0 / L[static_cast<long long>(c) * K + c];
+  __syncwarp();
+  for (int i = c + 1; i < K; ++i) {
+    const double* li = L + static_cast<long long>(i) * K;
+    double s = 0.0;
+    for (int k = c + lane; k < i; k += 32) s = fma(li[k], x[k], s);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) x[i] = -s / li[i];
+    __syncwarp();
+  }
+  for (int i = c + lane; i < K; i += 32) G[static_cast<long long>(K - 1 - i) * K + (K - 1 - c)] = x[i];
+  for (int i = lane; i < c; i += 32) G[static_cast<long long>(K - 1 - i) * K + (K - 1 - c)] = 0.0;
+}
+
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
+
+size_t gptq_factor_workspace_bytes(int K) { return 2 * align256(static_cast<size_t>(K) * K * 8); }
+
+cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspace, cudaStream_t st) {
+  double* L = static_cast<double*>(workspace);
+  double* scratch = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + align256(static_cast<size_t>(K) * K * 8));
+  gptq_reverse_kernel<<<4 * device_sm_count(), 256, 0, st>>>(H, K, L);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int j = 0; j < K; ++j) {
+    gptq_chol_col_kernel<<<1, 32, 0, st>>>(L, K, j, true);
+    const int rows = K - 1 - j;
+    if (rows > 0) gptq_chol_col_kernel<<<(rows + 7) / 8, 256, 0, st>>>(L, K, j, false);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  gptq_trinv_kernel<<<(K + 7) / 8, 256, 0, st>>>(L, K, G, scratch);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gptq_hessian(const __half* X, int T, int K, double damp, double* H, cudaStream_t st) {
   const dim3 grid((K + kHTile - 1) / kHTile, (K + kHTile - 1) / kHTile);

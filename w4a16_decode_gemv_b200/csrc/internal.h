@@ -102,6 +102,8 @@ cudaError_t launch_sum_partials(const double* partial, int n_alpha, double* sums
 constexpr int kMaxGptqK = 32768;
 cudaError_t launch_gptq_hessian(const __half* X, int T, int K, double damp, double* H, cudaStream_t st);
 size_t gptq_sweep_workspace_bytes(int N, int K);
+size_t gptq_factor_workspace_bytes(int K);
+cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspace, cudaStream_t st);
 cudaError_t launch_gptq_sweep(const __half* W, const double* G, int N, int K, int bits, int mode, uint32_t* qweight,
                               __half* scales, __half* zeros, void* workspace, cudaStream_t st);
 
