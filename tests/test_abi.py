@@ -231,3 +231,21 @@ def test_gptq_factor_and_quantize_validation(lib):
     assert call(K=200) == ERR_SHAPE
     assert call(X=MIS) == ERR_ALIGN
     assert call(nbytes=need - 1) == ERR_WORKSPACE
+
+
+def test_python_binding_rejects_cpu_tensors_for_search_and_gptq():
+    """No CPU fallback: every binding refuses host tensors before calling the library."""
+    import torch
+    W = torch.zeros((8, 128), dtype=torch.float16)
+    X = torch.zeros((4, 128), dtype=torch.float16)
+    H = torch.eye(128, dtype=torch.float64)
+    with pytest.raises(w4.W4A16Error):
+        w4.awq_search_alpha(W, X, [0.0, 0.5])
+    with pytest.raises(w4.W4A16Error):
+        w4.gptq_hessian(X)
+    with pytest.raises(w4.W4A16Error):
+        w4.gptq_sweep(W, H)
+    with pytest.raises(w4.W4A16Error):
+        w4.gptq_factor(H)
+    with pytest.raises(w4.W4A16Error):
+        w4.gptq_quantize(W, X)
