@@ -140,9 +140,9 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  * workspace.  x is the activation already divided by the AWQ scale s.
  * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
  * y_ref the exact product with the dequantized weight.  y is the same on every
- * call, bit for bit, except on the split-K CUDA-core GEMV (M = 2..4 when the
- * whole-row GEMV does not apply, or K / 128 odd), whose partial sums may be
- * added in another order.
+ * call, bit for bit, except on the split-K CUDA-core GEMV, which serves M = 1..4
+ * when the whole-row kernels do not apply (K / 128 odd, or activations too
+ * large to stage) and whose partial sums may be added in another order.
  *
  *   x        fp16 [M][K], device.     y  fp16 [M][N], device (output).
  *   qweight, scales, zeros as produced by awq_quantize_pack (layout v1).
