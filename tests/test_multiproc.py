@@ -67,3 +67,23 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     d = bench.Dist(2)
     assert bench.run_reference(None, d) is None
+
+
+def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic comes from a committed ncu summary only while the
+    kernel source still hashes to the profiled one; otherwise it is reported as null."""
+    import hashlib
+    import json
+
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    entry = {"source": "k.cu", "source_sha256": hashlib.sha256(b"kernel v1").hexdigest(),
+             "dram_bytes_per_launch": 123}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"k": entry}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k") == 123
+    assert bench.profiled_traffic("other") is None
+    src.write_text("kernel v2")
+    assert bench.profiled_traffic("k") is None
