@@ -161,3 +161,17 @@ def test_group_steps_come_from_the_swept_block():
     assert np.array_equal(d[:, 1], d1[:, 0]) and np.array_equal(z[:, 1], z1[:, 0])
     d_orig, _ = oracle.group_params(w0[:, group:], 3, oracle.ASYM, group)
     assert not np.array_equal(d[:, 1], d_orig[:, 0]), "the case must tell the two readings apart"
+
+
+def test_reversed_factorization_gives_the_same_factor():
+    """The construction the GPU uses: with P the reversal of the index order, P H P = L L^T and
+    G = P L^-1 P is upper triangular with a positive diagonal and G^T G = H^-1, so it equals
+    Cholesky(H^-1)^T (uniqueness); no inverse of H is formed."""
+    rng = np.random.default_rng(19)
+    K = 48
+    H = oracle.gptq_hessian(_correlated_x(rng, 80, K, mix=1.5))
+    P = np.eye(K)[::-1]
+    L = np.linalg.cholesky(P @ H @ P)
+    G = P @ np.linalg.solve(L, np.eye(K)) @ P
+    assert np.allclose(G, np.triu(G), atol=0) and np.all(np.diag(G) > 0)
+    np.testing.assert_allclose(G, oracle.gptq_factor(H), rtol=1e-9, atol=1e-12 * np.abs(G).max())
