@@ -345,6 +345,28 @@ W4A16_API w4a16_status w4a16_gemv_noalloc(const void* x, const uint32_t* qweight
 /* Size in bytes of the fixed scratch array used by w4a16_gemv_noalloc. */
 W4A16_API size_t w4a16_gemv_noalloc_max_scratch(void);
 
+/*
+ * w4a16_gemv_noalloc_check -- the w4a16_gemm_check of the allocation-free GEMV
+ * (the pages have no counterpart).  Synchronizes `stream`, reads the status
+ * word of the current device's scratch array and clears it.  Returns
+ * W4A16_ERR_DEVICE if a w4a16_gemv_noalloc kernel since the last call gave up
+ * waiting for its weight tiles (its y is then incomplete), W4A16_ERR_CUDA if
+ * the stream reports an error, else W4A16_OK.  Every w4a16_gemv_noalloc call
+ * clears the status word when it starts, so check after a call and before the
+ * next one.  Allocates nothing.
+ */
+W4A16_API w4a16_status w4a16_gemv_noalloc_check(w4a16_stream_t stream);
+
+/*
+ * w4a16_gemv_noalloc_timeout_selftest -- w4a16_wait_timeout_selftest aimed at
+ * the scratch array's status word: one small kernel on `stream` waits on a
+ * barrier nothing completes, gives up after `limit_us` microseconds
+ * (1 .. 1000000) and records the timeout, so that w4a16_gemv_noalloc_check
+ * then returns W4A16_ERR_DEVICE.  Nothing faults or hangs.  Returns
+ * W4A16_ERR_ARG for a limit out of range, W4A16_ERR_CUDA if the launch fails.
+ */
+W4A16_API w4a16_status w4a16_gemv_noalloc_timeout_selftest(int limit_us, w4a16_stream_t stream);
+
 /* Message for the last error on this thread ("" if none). */
 W4A16_API const char* w4a16_last_error(void);
 

@@ -109,6 +109,12 @@ def test_gemm_check_validation(lib):
     assert lib.w4a16_gemm_check(None, None) == ERR_ARG
 
 
+def test_noalloc_timeout_selftest_validation(lib):
+    assert lib.w4a16_gemv_noalloc_timeout_selftest(0, None) == ERR_ARG
+    assert lib.w4a16_gemv_noalloc_timeout_selftest(1000001, None) == ERR_ARG
+    assert "limit_us" in _err(lib)
+
+
 def test_wait_timeout_selftest_validation(lib):
     """Argument checks happen before any launch (no GPU needed)."""
     assert lib.w4a16_wait_timeout_selftest(None, 1000, None) == ERR_ARG

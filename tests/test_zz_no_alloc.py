@@ -1,11 +1,14 @@
-"""w4a16_gemv_noalloc, the allocation-free GEMV entry point, against w4a16_gemm.
+"""w4a16_gemv_noalloc, the allocation-free GEMV entry point, against the oracle.
 
-Some callers cannot allocate device memory (fixed-budget servers, plug-ins
-without an allocator), so the library offers a GEMV that keeps its scratch in
-a fixed device array.  This file checks, through the C ABI, that two calls in
-a row give the same output as the regular entry point within the tolerance of
-the other GEMV tests.  It is named to be collected last, and passes both alone
-and after the other tests.
+Some callers cannot allocate device memory: servers that reserve every buffer
+at start-up, plug-ins handed only the tensors they work on, hosts without a
+device allocator.  The library gives them a GEMV that keeps its scratch in a
+fixed device array.  This file checks, through the C ABI, that two calls in a
+row each match the oracle's exact product within the tolerance of the other
+GEMV tests, that the two agree with each other up to the last-bit freedom of
+the split-K reduction (fp32 atomics), and that a timed-out wait in that path is
+reported by w4a16_gemv_noalloc_check.  It is named to be collected last, and
+passes both alone and after the other tests.
 """
 import numpy as np
 import pytest
@@ -27,22 +30,43 @@ def dev():
     return torch.device("cuda:0")
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (3, 1000, 11008), (4, 8192, 2048)])
-def test_noalloc_matches_regular_entry_point_twice(dev, M, N, K):
+def _case(dev, M, N, K):
     W, x = inputs.random_case(7 * N + M, N, K, M)
     qo, so, zo = oracle.quantize_pack(W, None, 128, 4, oracle.ASYM)
     args = [torch.from_numpy(a).to(dev) for a in (x, qo.view(np.int32), so, zo)]
-    y_ref = w4.w4a16_gemm(*args).cpu().numpy().astype(np.float64)
-    _, B = oracle.gemm(x, qo, so, zo)
-    tol = 2e-3 * B + 1e-3
+    y_ref, B = oracle.gemm(x, qo, so, zo)
+    return args, y_ref, 2e-3 * B + 1e-3
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (2, 3000, 1152), (3, 1000, 11008), (4, 8192, 2048)])
+def test_noalloc_matches_oracle_twice(dev, M, N, K):
+    args, y_ref, tol = _case(dev, M, N, K)
     out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ys = []
     for _ in range(2):
         out.fill_(float("nan"))
         y = w4.w4a16_gemv_noalloc(*args, out=out)
-        torch.cuda.synchronize()
-        diff = np.abs(y.cpu().numpy().astype(np.float64) - y_ref)
+        w4.gemv_noalloc_check(dev)
+        yh = y.cpu().numpy()
+        diff = np.abs(yh.astype(np.float64) - y_ref)
         assert np.all(np.isfinite(diff))
         assert np.all(diff <= tol)
+        ys.append(yh)
+    # the split-K partial sums are added with fp32 atomics, so the order of
+    # addition (and at most the last bit of the fp16 result) may change
+    ulp = np.spacing(np.abs(ys[0]).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(ys[0].astype(np.float64) - ys[1].astype(np.float64)) <= ulp)
+
+
+def test_noalloc_timeout_is_reported_then_cleared(dev):
+    w4.gemv_noalloc_timeout_selftest(limit_us=2000, device=dev)
+    with pytest.raises(w4.W4A16Error, match="gave up waiting"):
+        w4.gemv_noalloc_check(dev)
+    w4.gemv_noalloc_check(dev)  # the check cleared the status word
+    args, y_ref, tol = _case(dev, 2, 512, 1024)
+    y = w4.w4a16_gemv_noalloc(*args)
+    w4.gemv_noalloc_check(dev)
+    assert np.all(np.abs(y.cpu().numpy().astype(np.float64) - y_ref) <= tol)
 
 
 def test_noalloc_rejects_oversized_scratch(dev):

@@ -53,6 +53,10 @@ def load_library():
     lib.w4a16_gemv_noalloc.restype = i
     lib.w4a16_gemv_noalloc_max_scratch.argtypes = []
     lib.w4a16_gemv_noalloc_max_scratch.restype = sz
+    lib.w4a16_gemv_noalloc_check.argtypes = [vp]
+    lib.w4a16_gemv_noalloc_check.restype = i
+    lib.w4a16_gemv_noalloc_timeout_selftest.argtypes = [i, vp]
+    lib.w4a16_gemv_noalloc_timeout_selftest.restype = i
     lib.awq_search_workspace_size.argtypes = [i, i, i, i, i]
     lib.awq_search_workspace_size.restype = sz
     lib.awq_search_alpha.argtypes = [vp, vp, i, i, i, vp, i, i, i, i, vp, vp, vp, sz, vp]
@@ -247,6 +251,23 @@ def w4a16_gemv_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Ten
         _check(lib.w4a16_gemv_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), M, N, K, group, _ptr(y),
                                       _stream(x.device)), "w4a16_gemv_noalloc")
     return y
+
+
+def gemv_noalloc_check(device=None) -> None:
+    """Synchronizes and raises if a w4a16_gemv_noalloc kernel gave up waiting
+    since the last check (the scratch array's status word; cleared here)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib.w4a16_gemv_noalloc_check(_stream(dev)), "w4a16_gemv_noalloc_check")
+
+
+def gemv_noalloc_timeout_selftest(limit_us: int = 1000, device=None) -> None:
+    """Runs the bounded-wait probe on the scratch array's status word (see gemv_noalloc_check)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib.w4a16_gemv_noalloc_timeout_selftest(limit_us, _stream(dev)), "w4a16_gemv_noalloc_timeout_selftest")
 
 
 def search_workspace_size(N: int, K: int, T: int, n_alpha: int, group: int = GROUP) -> int:

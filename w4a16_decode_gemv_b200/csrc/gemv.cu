@@ -338,6 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_multi_kernel(const GemvArgs 
     }
     ++contrib;
     if (++kc == a.units_k) kc = 0, ++rb;
+    // every lane's reads of the stage are ordered before the copy that refills it
+    release_stage_reads();
     __syncwarp();
     if (i + STAGES < cnt) issue_unit<kRm>(a, rb_f, kc_f, ring + slot * kUnitMBytes, &bars[slot], lane, pol);
     if (++kc_f == a.units_k) kc_f = 0, ++rb_f;

@@ -41,6 +41,30 @@ w4a16_status noalloc_fail(w4a16_status st, const char* msg) {
   return st;
 }
 
+// Device address of the scratch array on the current device, looked up on the
+// first use and cached; null (with the message set) on failure.
+void* scratch_base(const char* who) {
+  char buf[160];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    snprintf(buf, sizeof(buf), "%s: no usable current device", who);
+    set_last_error(buf);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      snprintf(buf, sizeof(buf), "%s: cudaGetSymbolAddress failed", who);
+      set_last_error(buf);
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 }  // namespace w4a16
 
@@ -75,20 +99,8 @@ W4A16_API w4a16_status w4a16_gemv_noalloc(const void* x, const uint32_t* qweight
   }
 
   // device address of the scratch array on the current device (looked up once)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc: no usable current device");
-  void* base = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-      void* p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess || !p) return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc: cudaGetSymbolAddress failed");
-      g_noalloc_ptr[dev] = p;
-    }
-    base = g_noalloc_ptr[dev];
-  }
+  void* base = scratch_base("w4a16_gemv_noalloc");
+  if (!base) return W4A16_ERR_CUDA;
 
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // the kernel expects zeroed partial sums, counters and status word
@@ -98,6 +110,38 @@ W4A16_API w4a16_status w4a16_gemv_noalloc(const void* x, const uint32_t* qweight
                 static_cast<const __half*>(zeros), static_cast<__half*>(y), M, N, K};
   const cudaError_t e = launch_gemv(p, carve_workspace(base, M, N, K), st);
   if (e != cudaSuccess) return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc: kernel launch failed");
+  return W4A16_OK;
+}
+
+W4A16_API w4a16_status w4a16_gemv_noalloc_check(w4a16_stream_t stream) {
+  set_last_error("");
+  void* base = scratch_base("w4a16_gemv_noalloc_check");
+  if (!base) return W4A16_ERR_CUDA;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess)
+    return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc_check: the stream reports an error");
+  // the status word is the first word of the array (carve_workspace)
+  uint32_t flag = 0;
+  if (cudaMemcpy(&flag, base, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc_check: reading the status word failed");
+  if (flag != kDevOk) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(base, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc_check: clearing the status word failed");
+    return noalloc_fail(W4A16_ERR_DEVICE, "w4a16_gemv_noalloc: a kernel gave up waiting for its weight tiles");
+  }
+  return W4A16_OK;
+}
+
+W4A16_API w4a16_status w4a16_gemv_noalloc_timeout_selftest(int limit_us, w4a16_stream_t stream) {
+  set_last_error("");
+  if (limit_us < 1 || limit_us > 1000000)
+    return noalloc_fail(W4A16_ERR_ARG, "w4a16_gemv_noalloc_timeout_selftest: limit_us must be 1 .. 1000000");
+  void* base = scratch_base("w4a16_gemv_noalloc_timeout_selftest");
+  if (!base) return W4A16_ERR_CUDA;
+  if (launch_wait_timeout_probe(static_cast<uint32_t*>(base), static_cast<uint64_t>(limit_us) * 1000ull,
+                                reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return noalloc_fail(W4A16_ERR_CUDA, "w4a16_gemv_noalloc_timeout_selftest: launch failed");
   return W4A16_OK;
 }
 
