@@ -537,9 +537,14 @@ def other_workloads(args, dev):
               "prefill_8192": [(M, 8192, 8192) for M in (128, 200, 512)]}
     only = args.only
     if only is not None:
-        # one workload alone (for profiling): a name, or skinny_8192:M for one M
-        name, _, m = only.partition(":")
-        shapes = {k: [e for e in v if not m or e[0] == int(m)] for k, v in shapes.items() if k == name}
+        # some workloads alone (for profiling): comma-separated names, or skinny_8192:M for one M
+        picked = {}
+        for item in only.split(","):
+            name, _, m = item.partition(":")
+            if name in shapes:
+                picked.setdefault(name, []).extend(e for e in shapes[name] if not m or e[0] == int(m))
+        shapes = picked
+        only = {item.partition(":")[0] for item in only.split(",")}
     for name, lst in shapes.items():
         entries = []
         for M, N, K in lst:
@@ -557,19 +562,19 @@ def other_workloads(args, dev):
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries
-    if only is not None and only not in ("quantize_pack_11008x4096", "awq_search_11008x4096", "gptq_11008x4096"):
+    if only is not None and not only & {"quantize_pack_11008x4096", "awq_search_11008x4096", "gptq_11008x4096"}:
         return res
     W, X, _ = inputs.quant_workload()
     Wd = torch.from_numpy(W).to(dev)
     Xd = torch.from_numpy(X).to(dev)
-    if only is None or only == "awq_search_11008x4096":
+    if only is None or "awq_search_11008x4096" in only:
         res["awq_search_11008x4096"] = search_workload(Wd, Xd, dev)
-    if only is None or only == "gptq_11008x4096":
+    if only is None or "gptq_11008x4096" in only:
         try:
             res["gptq_11008x4096"] = gptq_workload(Wd, Xd, dev)
         except Exception as e:  # report, never hide
             res["gptq_11008x4096"] = {"error": str(e)[:300]}
-    if only is not None and only != "quantize_pack_11008x4096":
+    if only is not None and "quantize_pack_11008x4096" not in only:
         return res
     # quantize + pack of the 11008 x 4096 AWQ workload (4-bit asym and 3-bit sym)
     s = w4.awq_act_scale(Xd, 0.5)
@@ -678,7 +683,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--only", default=None,
-                    help="run one of the other workloads only (gemv_4096x4096, llama7b_decode, llama65b_decode, "
+                    help="run some of the other workloads only, comma-separated (gemv_4096x4096, llama7b_decode, llama65b_decode, "
                          "skinny_8192 or skinny_8192:M, prefill_8192 or prefill_8192:M, quantize_pack_11008x4096, "
                          "awq_search_11008x4096, gptq_11008x4096); for profiling")
     args = ap.parse_args()

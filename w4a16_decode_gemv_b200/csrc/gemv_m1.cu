@@ -9,12 +9,13 @@
 // bit masks and the dequantization is fused into the product (Lecture 13 guide,
 // §TinyChat, slides 36-37).
 //
-// Work split.  Row blocks of 4 rows are dealt to the CTAs (one per SM) in
-// contiguous, balanced ranges, so a CTA owns whole rows and no partial sum
-// leaves the SM.  A CTA's row blocks are cut into units of 4 rows x 2048 input
-// channels (4 KiB of codes plus the 4 x 16 Delta and z of those rows), and warp
-// w of the CTA takes units w, w + W, w + 2W, ... (W = 16 warps, or 12 when
-// the staged activations of a large K leave room for only 12 rings)  Each warp streams its own
+// Work split.  Row blocks of 4 rows are dealt to the CTAs (one per SM and
+// layer) in contiguous, balanced ranges, so a CTA owns whole rows and no
+// partial sum leaves the SM.  A CTA's row blocks are cut into units of 4 rows x
+// 2048 input channels (4 KiB of codes plus the 4 x 16 Delta and z of those
+// rows), and warp w of the CTA takes units w, w + W, w + 2W, ... (W = 8 warps
+// when two CTAs share an SM, else 16, or 12 when the staged activations of a
+// large K leave room for only 12 rings; see the kernel).  Each warp streams its own
 // units through a private ring of shared-memory stages: one lane issues a 2-D
 // tensor copy (TMA, box of 4 rows x 256 words, zero fill past the matrix edge)
 // per unit and all lanes copy the Delta / z tile with cp.async, all completing
@@ -119,10 +120,17 @@ __device__ __forceinline__ void issue_unit(const M1Args& a, const CUtensorMap* t
   cp_async_arrive(bar);
 }
 
-// WARPS = 16, or 12 when 16 rings do not fit beside the staged activations
-// (large K).
-template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1)
+// Two shapes.  CTAS = 2: 8 warps and at most half of an SM's shared memory, so
+// that a CTA of the next layer's GEMV can sit on the SM beside one of this
+// layer's.  That CTA fills its whole ring before it waits for this layer to
+// finish (the weights do not depend on it), so the SM's share of the next
+// layer's weights is already streaming while this layer computes, and the
+// start-up of a layer (release, activation staging) and the unequal ends of its
+// warps no longer leave HBM idle.  CTAS = 1: 16 warps (12 when 16 rings do not
+// fit beside the staged activations of a large K) owning the whole SM, with
+// only the first stage fetched before the wait.
+template <int WARPS, int CTAS>
+__global__ void __launch_bounds__(WARPS * 32, CTAS)
     gemv_m1_kernel(const M1Args a, const __grid_constant__ CUtensorMap tmap) {
   constexpr int kWarps = WARPS;
   constexpr int kThreads = WARPS * 32;
@@ -148,9 +156,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
   }
   __syncwarp();
   const uint64_t pol = l2_evict_first_policy();
-  // prologue: the first stage of the ring (codes, Delta and z are read-only, so
-  // this overlaps the previous kernel's tail).  Only one: the activations are
-  // loaded right after griddep_wait and should not queue behind more weights.
+  // prologue: codes, Delta and z are read-only, so they may be fetched before
+  // the previous kernel has finished.  With one CTA per SM only the first
+  // stage: the activations are loaded right after griddep_wait and should not
+  // queue behind more weights.  With two, the whole ring: the CTA starts while
+  // the previous layer still runs, and its copies land long before the wait
+  // returns.
+  const int pre = CTAS > 1 ? S : 1;
   int rb_f = rb0 + warp / a.units_k, kc_f = warp % a.units_k;
   int jf = warp;
   auto issue_next = [&](int s) {
@@ -159,7 +171,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     rb_f += drb, kc_f += dkc;
     if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
   };
-  if (jf < U) issue_next(0);
+  for (int s = 0; s < pre && jf < U; ++s) issue_next(s);
 
   // x, y and anything earlier kernels produce are touched only after this
   griddep_wait();
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
   }
   __syncthreads();
   // the rest of the ring
-  for (int s = 1; s < S && jf < U; ++s) issue_next(s);
+  for (int s = pre; s < S && jf < U; ++s) issue_next(s);
 
   // Lanes with bit 2 set read the second 16-byte half of their 32 bytes of a
   // weight row first, so that the 32-byte lane stride does not put two lanes of
@@ -325,23 +337,53 @@ int smem_for(int warps, int stages, int x_bytes, int max_units) {
   return x_bytes + warps * stages * kStage + round128(max_units * kR * 4) + warps * stages * 8;
 }
 
-// Warps per CTA: 16 if two ring stages per warp fit, else 12, else 0.
-int m1_warps(int N, int K, int& max_units) {
+// Shared memory of an SM (228 KiB) less 1 KiB the system reserves per CTA,
+// split between two CTAs.
+constexpr int kMaxSmemPair = (228 * 1024) / 2 - 1024;
+
+struct M1Config {
+  int warps, ctas, stages, smem, grid, max_units;
+};
+
+// Two 8-warp CTAs per SM when a CTA's ring holds all of its units, so that the
+// whole layer is fetched before the previous layer ends (on B200 that paid at
+// 4096 x 4096: 3.65 against 4.23 us per layer; for larger layers the shallower
+// rings of two CTAs lost more than the overlap gained: 10.5 against 9.2 us at
+// 8192 x 8192); else one CTA of 16 warps (12 if 16 two-stage rings do not
+// fit); the deepest ring (up to 6 stages) that fits.  False when nothing fits.
+bool m1_config(int N, int K, M1Config& c) {
   const int sms = device_sm_count();
   const int row_blocks = (N + kR - 1) / kR;
-  const int grid = min(sms, row_blocks);
-  max_units = ((row_blocks + grid - 1) / grid) * ((K / 8 + kUW - 1) / kUW);
-  for (int w : {16, 12})
-    if (smem_for(w, 2, x_bytes_for(K), max_units) <= kMaxSmem) return w;
-  return 0;
+  c.grid = min(sms, row_blocks);
+  c.max_units = ((row_blocks + c.grid - 1) / c.grid) * ((K / 8 + kUW - 1) / kUW);
+  const int xb = x_bytes_for(K);
+  const struct {
+    int warps, ctas, limit;
+  } shapes[3] = {{8, 2, kMaxSmemPair}, {16, 1, kMaxSmem}, {12, 1, kMaxSmem}};
+  for (const auto& sh : shapes) {
+    if (smem_for(sh.warps, 2, xb, c.max_units) > sh.limit) continue;
+    if (sh.ctas == 2) {
+      int st = 6;
+      while (st > 2 && smem_for(sh.warps, st, xb, c.max_units) > sh.limit) --st;
+      if (sh.warps * st < c.max_units) continue;  // the ring cannot hold the CTA's units
+    }
+    int st = 6;
+    while (st > 2 && smem_for(sh.warps, st, xb, c.max_units) > sh.limit) --st;
+    c.warps = sh.warps;
+    c.ctas = sh.ctas;
+    c.stages = st;
+    c.smem = smem_for(sh.warps, st, xb, c.max_units);
+    return true;
+  }
+  return false;
 }
 
 }  // namespace
 
 bool gemv_m1_supports(int N, int K) {
   if ((K / kGroup) % 2) return false;  // Delta/z pairs are copied 4 bytes at a time
-  int max_units;
-  return m1_warps(N, K, max_units) != 0;
+  M1Config c;
+  return m1_config(N, K, c);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -372,17 +414,13 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   a.Kg = p.K / kGroup;
   a.units_k = (a.Kw + kUW - 1) / kUW;
   a.row_blocks = (p.N + kR - 1) / kR;
-  const int grid = min(device_sm_count(), a.row_blocks);
-  a.max_units = ((a.row_blocks + grid - 1) / grid) * a.units_k;
+  M1Config c;
+  if (!m1_config(p.N, p.K, c)) return cudaErrorNotSupported;
+  const int grid = c.grid;
+  a.max_units = c.max_units;
   a.x_bytes = x_bytes_for(p.K);
-  int mu;
-  const int warps = m1_warps(p.N, p.K, mu);
-  if (warps == 0) return cudaErrorNotSupported;
-  // deepest per-warp ring that fits
-  int stages = 6;
-  while (stages > 2 && smem_for(warps, stages, a.x_bytes, a.max_units) > kMaxSmem) --stages;
-  a.stages = stages;
-  const int smem = smem_for(warps, stages, a.x_bytes, a.max_units);
+  a.stages = c.stages;
+  const int smem = c.smem;
 
   // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256.
   // The map depends only on the pointer and the shape, so the maps of the
@@ -420,12 +458,15 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
     cache_next = (cache_next + 1) % kMapCache;
   }
 
-  auto kern = warps == 16 ? gemv_m1_kernel<16> : gemv_m1_kernel<12>;
+  auto kern = c.ctas == 2 ? gemv_m1_kernel<8, 2> : (c.warps == 16 ? gemv_m1_kernel<16, 1> : gemv_m1_kernel<12, 1>);
   cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e == cudaSuccess)
+    e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(warps * 32);
+  cfg.blockDim = dim3(c.warps * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
