@@ -83,7 +83,7 @@ def test_workspace_size(lib):
     assert ws(4, 100, 256, 128) >= 4 * 100 * 4
     assert ws(0, 8, 128, 128) == 0
     # M above one launch's 128 tokens runs in chunks on the M = 128 workspace
-    assert ws(200, 8, 128, 128) == ws(128, 8, 128, 128) > ws(64, 8, 128, 128)
+    assert ws(300, 8, 128, 128) == ws(256, 8, 128, 128) > ws(128, 8, 128, 128) > ws(64, 8, 128, 128)
     assert ws(1 << 20, 4096, 4096, 128) == 0
     assert ws(1, 8, 100, 128) == 0
     assert ws(1, 8, 128, 64) == 0

@@ -1,5 +1,5 @@
-"""Parity of the tensor-core GEMM (M = 5..128 per launch, larger M in chunks of
-128 tokens) with the CPU oracle.
+"""Parity of the tensor-core GEMM (M = 5..256 per launch, larger M in chunks of
+256 tokens) with the CPU oracle.
 
 Every case goes through the C ABI (``w4a16_gemm``).  The output must satisfy,
 per element, |y - y_ref| <= 2e-3 * B + 1e-3 with B = sum_k |x * w_hat| and
@@ -83,11 +83,14 @@ def test_tc_wide_token_tiles(dev, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (129, 300, 1024),     # 128 + 1: the tail runs on the M = 1 GEMV
-    (130, 256, 2048),     # 128 + 2: the tail on the whole-row GEMV for M = 2..4
-    (200, 513, 1152),     # 128 + 72, odd groups per row
-    (300, 256, 4096),     # 128 + 128 + 44
-    (512, 384, 2048),     # four full chunks
+    (129, 300, 1024),     # token tile 192
+    (150, 1000, 11008),   # token tile 192, up to 22 CTAs share a tile
+    (200, 513, 1152),     # token tile 256, odd groups per row (a pair of one group)
+    (256, 384, 2048),     # one full chunk of 256
+    (257, 300, 1024),     # 256 + 1: the tail runs on the M = 1 GEMV
+    (258, 256, 2048),     # 256 + 2: the tail on the whole-row GEMV for M = 2..4
+    (300, 256, 4096),     # 256 + 44
+    (512, 384, 2048),     # two full chunks
 ])
 def test_tc_large_m_chunks(dev, M, N, K):
     case(dev, M, N, K, seed=M * 7919 + N)
@@ -155,9 +158,9 @@ def test_tc_repeated_calls_identical(dev):
     check(y2, *ref)
 
 
-@pytest.mark.parametrize("M", [16, 128, 300])
+@pytest.mark.parametrize("M", [16, 128, 200, 300])
 def test_tc_bit_identical_across_calls(dev, M):
-    """The partial sums of shared row blocks are added in CTA order, so y must not
+    """The partial tiles of shared row tiles are added in CTA order, so y must not
     change by a single bit from call to call.  At 8192 x 8192 every CTA streams
     about 14 units through its rings, which exposes a ring stage overwritten
     while it is still being read (the tolerance of the parity tests can hide it)."""

@@ -103,25 +103,27 @@ static size_t gemv_acc_bytes(int M, int N) {
 
 size_t workspace_bytes(int M, int N, int K) {
   (void)K;
-  if (M <= kMaxGemvM) return 16 + counter_bytes(N) + static_cast<size_t>(M) * N * 4;
-  return 16 + counter_bytes(N) + gemv_acc_bytes(kMaxGemvM, N) + tc_partial_bytes(M);
+  const size_t head = 16 + kFlagBytes + counter_bytes(N);
+  if (M <= kMaxGemvM) return head + static_cast<size_t>(M) * N * 4;
+  return head + gemv_acc_bytes(kMaxGemvM, N) + tc_partial_bytes(M);
 }
 
 Workspace carve_workspace(void* base, int M, int N, int K) {
   (void)K;
   uint8_t* p = static_cast<uint8_t*>(base);
+  const size_t head = 16 + kFlagBytes + counter_bytes(N);
   Workspace w;
   w.status = reinterpret_cast<uint32_t*>(p);
-  w.counters = reinterpret_cast<uint32_t*>(p + 16);
-  w.acc = reinterpret_cast<float*>(p + 16 + counter_bytes(N));
-  w.part = M <= kMaxGemvM ? nullptr
-                          : reinterpret_cast<float*>(p + 16 + counter_bytes(N) + gemv_acc_bytes(kMaxGemvM, N));
+  w.flags = reinterpret_cast<uint32_t*>(p + 16);
+  w.counters = reinterpret_cast<uint32_t*>(p + 16 + kFlagBytes);
+  w.acc = reinterpret_cast<float*>(p + head);
+  w.part = M <= kMaxGemvM ? nullptr : reinterpret_cast<float*>(p + head + gemv_acc_bytes(kMaxGemvM, N));
   return w;
 }
 
 // The kernels for an M x N x K problem with M <= kMaxM: M = 1 on whole rows when
 // the activation fits the kernel's staging, M = 2..4 on whole rows or split-K,
-// M = 5..128 on the tensor cores.
+// M = 5..256 on the tensor cores.
 static cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
   if (p.M == 1 && gemv_m1_supports(p.N, p.K)) return launch_gemv_m1(p, ws.status, st);
   if (gemv_mt_supports(p.M, p.N, p.K)) return launch_gemv_mt(p, ws.status, st);
@@ -131,10 +133,10 @@ static cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cuda
 
 cudaError_t gemm_chunks(const GemmProblem& p, void* workspace, cudaStream_t st) {
   // Chunk c starts kMaxM * c tokens in: its x and y offsets are multiples of
-  // 256 bytes per input and per output channel, so both stay 16-byte aligned.
+  // 512 bytes per input and per output channel, so both stay 16-byte aligned.
   // Stream order keeps the chunks' uses of the workspace apart (a chunk's
-  // partial sums are written only after its griddepcontrol.wait, which waits
-  // for the previous chunk's finalize to complete).
+  // partial tiles and flags are touched only after its griddepcontrol.wait,
+  // which waits for the previous chunk to complete).
   for (int t0 = 0; t0 < p.M; t0 += kMaxM) {
     GemmProblem c = p;
     c.M = p.M - t0 < kMaxM ? p.M - t0 : kMaxM;
@@ -465,8 +467,8 @@ w4a16_status w4a16_gemm_check(void* workspace, w4a16_stream_t stream) {
   e = cudaMemcpy(&flag, workspace, sizeof(flag), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm_check: read status");
   if (flag != kDevOk) {
-    const uint32_t zero = 0;
-    e = cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    // a kernel that gave up may have left partial-tile flags set: clear them with the status word
+    e = cudaMemset(workspace, 0, 16 + kFlagBytes);
     if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm_check: clear status");
     return fail(W4A16_ERR_DEVICE, "w4a16_gemm: a kernel gave up waiting for its weight tiles (status %u)", flag);
   }

@@ -1,5 +1,5 @@
-// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05) for M = 5..128
-// (larger M runs as chunks of 128 tokens, one launch pair per chunk).
+// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05), M = 5..256 per
+// launch (larger M runs as chunks of 256 tokens, one launch per chunk).
 //
 //   y[m][n] = sum_k x[m][k] * w_hat[n][k],   w_hat = Delta[n][g] * (u[n][k] - z[n][g])
 //
@@ -7,82 +7,79 @@
 // belongs on the tensor cores ("MIT 6.5940 Fall 2024 Lecture 13: LLM
 // Deployment" reading guide, §SmoothQuant: batching moves the work from
 // memory-bound GEMV towards compute).  Up to M = 64 it is still bound by reading
-// the packed weights, so the kernel is built to stream them at HBM speed and keep
-// the dequantization and the MMAs under that time.
+// the packed weights, so every stage of the kernel is a separate role working
+// on its own ring, and the roles overlap: codes stream from HBM, warps turn them
+// into w_hat, the tensor cores multiply, and the last tile's sums are read out,
+// all at the same time.
 //
-// Swap-AB.  The weight rows are the MMA's M dimension (128 rows per MMA) and the
-// tokens its N dimension (the token tile MP: M rounded up to 16 up to 64, then
-// 96 or 128): D[n][m] = sum_k A[n][k] B[m][k]
-// with A = w_hat (fp16) and B = x (fp16, K-major in shared memory), fp32
-// accumulators in tensor memory (TMEM lane = weight row, column = token).
+// Swap-AB.  Weight rows are the MMA's M dimension (a tile of 128 rows = the 128
+// lanes of tensor memory) and tokens its N dimension (the token tile MP: 16, 32,
+// 64, 96, 128, 192 or 256): D[n][m] = sum_k A[n][k] B[m][k], with A = w_hat in
+// tensor memory (fp16 pairs, one 32-bit column per two inputs, written by
+// tcgen05.st) and B = x in shared memory (K-major, 128-byte swizzle, rows past M
+// zero-filled by the tensor copy), fp32 accumulators in tensor memory.  Keeping
+// A out of shared memory leaves shared memory to the copies alone.
 //
-// w_hat lives in shared memory, in the K-major 128-byte-swizzled layout of an
-// MMA operand: the dequantizing thread of a weight row writes its fp16 pairs
-// straight into that row's line of a w_hat buffer, and the MMA reads A through
-// a shared-memory descriptor, as it reads x.  Tensor memory then holds only the
-// accumulators.  (An earlier version wrote w_hat into tensor memory with
-// tcgen05.st; on B200 those stores slowed the MMAs' reads of A from tensor
-// memory, and this version is faster at every M.)
+// Work split (stream-K).  Units are (tile of 128 rows, pair of groups = 256
+// inputs), ordered tile-major and dealt to a persistent grid (one CTA per SM) in
+// contiguous, equal ranges.  A CTA's range covers at most a few tiles; it
+// accumulates each one (a segment) in a tensor-memory accumulator.  A tile no
+// single CTA covers is finished by the lowest CTA that covers part of it (its
+// owner), for which the tile is the last segment: every other contributor has
+// the tile as its first segment, publishes its fp32 partial tile to a workspace
+// slot and sets a flag; the owner, after its own MMAs, waits for those flags
+// (bounded), adds the partials in CTA order and writes y.  y does not depend on
+// timing, and no second kernel is needed.
 //
-// Work split.  Units are (row block of 256 rows, group of 128 inputs), ordered
-// row-block-major and dealt to a persistent grid (one CTA per SM) in contiguous,
-// equal ranges.  A CTA accumulates its units of one row block in two 128 x MP
-// TMEM accumulators (double-buffered, so the next row block's MMAs overlap the
-// read-out of the last).  A CTA that covers a whole row block writes y
-// directly; otherwise it writes its fp32 partial tile to one of its two slots
-// in the workspace (the row block its range starts in, and the one it ends
-// in), and gemm_tc_finalize, launched next on the stream, adds the slots of
-// each shared row block in CTA order: y does not depend on timing.
-//
-// Roles (18 warps):
-//   warps 0-15  dequantization and read-out: warp w holds tile t = (w >> 2) & 1
-//               (128 rows), TMEM lane quarter q = w & 3 and part p = w >> 3;
-//               lane i owns weight row t*128 + q*32 + i of the block, converts
-//               words 4p .. 4p + 3 of each 64-input half of a group into w_hat
-//               and writes them into one of the shared-memory w_hat buffers;
-//               after a row block's MMAs it reads out its rows' accumulator
-//               columns;
-//   warp 16     one thread issues the tensor copies (TMA) of each unit into a
-//               ring of stages: the 256 x 16-word code tile (64-byte swizzle)
-//               and the two 64-input halves of the x tile (128-byte swizzle,
-//               rows past M zero-filled);
-//   warp 17     allocates TMEM; one thread issues tcgen05.mma (8 per 64-input
-//               half) and tcgen05.commit.
+// Roles (16 warps):
+//   warp 0       one thread streams the code tiles: one tensor copy per unit
+//                (128 rows x 128 bytes, 128-byte swizzle) into a ring of Sc stages;
+//   warp 1       allocates tensor memory; one thread issues the MMAs (8 of
+//                128 x MP x 16 per group) and their commits;
+//   warp 2       one thread streams the x tiles (per group: two boxes of MP rows x
+//                64 inputs) into a ring of Sx stages, after griddepcontrol.wait;
+//   warps 4-11   dequantization: warp w covers tensor-memory lane quarter w & 3
+//                (rows 32 (w & 3) .. + 31 of the tile) and group h = (w - 4) >> 2
+//                of each pair; lane i reads its row's 64 code bytes, converts them
+//                into 64 columns of w_hat and stores them with tcgen05.st;
+//   warps 12-15  epilogue: accumulator read-out, y, partial tiles, the owner's sums.
 // Dequantization of a code pair: (w >> 4t) & 0x000F000F | 0x64006400 (one LOP3)
 // reads as the fp16 pair 1024 + q; subtracting 1024 + z is exact and the
 // multiply by Delta rounds once (Lecture 13 guide, §TinyChat, slides 36-37;
 // "CMU 11-868 Model Quantization" guide, §BF16/HFMA2).
 //
-// Every wait on an mbarrier is bounded; a timeout sets the workspace status word,
-// all roles leave their loops, copies and MMAs in flight are waited for, and TMEM
-// is freed before the CTA exits.
+// Every wait is bounded: a timeout sets the workspace status word and an abort
+// flag, every role leaves its loop, copies and MMAs in flight are waited for and
+// tensor memory is freed before the CTA exits.
 #include "common.cuh"
 #include "internal.h"
 
 namespace w4a16 {
 namespace {
 
-constexpr int kDqWarps = 16;                    // dequantization + epilogue warps
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kThreads = 32 * 18;
-constexpr int kRows = 256;                      // weight rows per row block (two MMA tiles)
-constexpr int kCodeBytes = kRows * 16 * 4;      // 16 KiB: one group of codes for the block
+constexpr int kRows = 128;                 // weight rows per tile
+constexpr int kCodeStage = kRows * 128;    // 16 KiB: one pair of groups of a tile
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kMaxStages = 12;
-constexpr int kCtrlBytes = 512;
+constexpr int kMaxCodeStages = 12;
+constexpr int kMaxXStages = 8;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kCodeWarp = 0, kMmaWarp = 1, kXWarp = 2;
+constexpr int kDqWarp0 = 4, kDqWarps = 8;
+constexpr int kEpiWarp0 = 12, kEpiWarps = 4;
+constexpr int kCtrlBytes = 1024;
+constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
-  const uint32_t* qweight;
   const __half* scales;
   const __half* zeros;
   __half* y;
-  float4* ws_part;      // [2 x grid slots][MP / 4][256 rows] partial sums
-  uint32_t* ws_status;
-  int M, N, Kw, Kg;
-  int dz_w;             // groups per Delta / z load: the largest of 8, 4, 2, 1 dividing Kg
-  int total_units;
-  int stages;
+  float4* part;       // [grid][MP / 4][128] partial tiles
+  uint32_t* flags;    // [grid] partial tile published (left zero after each call)
+  uint32_t* status;
+  int M, N, G, P;     // tokens, rows, groups per row, group pairs per row
+  int total;          // units = tiles x P
+  int sc, sx;         // code and x ring depths
 };
 
 // ---- tcgen05 / TMEM wrappers ---------------------------------------------------
@@ -99,22 +96,17 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T: A (128 rows x 16 inputs) and B both
-// described by shared-memory matrix descriptors.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+// D[tmem] (+)= A[tmem] * B[smem]^T: A is 128 rows x 16 inputs (fp16 pairs in 8
+// consecutive columns), B is described by a shared-memory matrix descriptor.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                            bool accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
       : "memory");
 }
-
-// The w_hat of one code word: 4 fp16 pairs, inputs 8j .. 8j + 7 in order.
-struct Word4 {
-  uint32_t v[4];
-};
 
 // Arrives once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -122,15 +114,30 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// 32 lanes x 8 consecutive 32-bit columns: thread i gets lane (base + i), columns c..c+7.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns into registers: thread i reads lane (base + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -142,12 +149,12 @@ __device__ __forceinline__ uint64_t sw128_desc(const void* p) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// kind::f16 instruction descriptor: fp32 D, fp16 A and B, both K-major, M = 128.
+// kind::f16 instruction descriptor: fp32 D, fp16 A and B, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_f16(int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-// ---- waits, arrivals, barriers --------------------------------------------------
+// ---- waits, arrivals -------------------------------------------------------------
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -170,41 +177,43 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits (bounded) until a partial-tile flag reaches `want`.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, volatile uint32_t* abort_flag,
+                                          uint32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (ld_acquire(flag) >= want) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(status, kDevWaitTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
 __device__ __forceinline__ uint32_t lop3_nib(uint32_t w) {
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
   return r;
 }
 
-// W consecutive fp16 values (W = 1, 2, 4 or 8, the address aligned to 2W bytes)
-// into the low halves of w[0..3], lowest address first.
-__device__ __forceinline__ void ld_nc_halves(const __half* p, int W, uint32_t (&w)[4]) {
-  w[0] = w[1] = w[2] = w[3] = 0;
-  if (W == 8)
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "l"(p));
-  else if (W == 4)
-    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "l"(p));
-  else if (W == 2)
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
-  else
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(w[0]) : "l"(p));
-}
-
-// The idx-th fp16 value (0..7) of four packed words, zero-extended.
-__device__ __forceinline__ uint32_t pick_half(const uint32_t (&w)[4], int idx) {
-  const uint32_t v = (idx & 4) ? ((idx & 2) ? w[3] : w[2]) : ((idx & 2) ? w[1] : w[0]);
-  return (idx & 1) ? (v >> 16) : (v & 0xFFFFu);
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, const Word4& v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.v[0]), "r"(v.v[1]), "r"(v.v[2]),
-               "r"(v.v[3])
-               : "memory");
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ld_nc_u16(const __half* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
 }
 
@@ -215,28 +224,19 @@ __device__ __forceinline__ uint32_t dq_pair(uint32_t v, __half2 nz, __half2 dd) 
   return as_u32(__hmul2(__hfma2(as_h2(lop3_nib(v)), __float2half2_rn(1.0f), nz), dd));
 }
 
-__device__ __forceinline__ Word4 dq_word(uint32_t w, __half2 zz, __half2 dd) {
-  return Word4{{dq_pair(w, zz, dd), dq_pair(w >> 4, zz, dd), dq_pair(w >> 8, zz, dd), dq_pair(w >> 12, zz, dd)}};
-}
-
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
-// Tensor memory holds only the accumulators: 2 buffers x 2 tiles x MP columns,
-// allocated as the next power of two of at least 32 columns.
-__host__ __device__ constexpr uint32_t tmem_cols(int mp) {
-  return 4 * mp <= 32 ? 32u : 4 * mp <= 64 ? 64u : 4 * mp <= 128 ? 128u : 4 * mp <= 256 ? 256u : 512u;
+// Accumulator buffers: two (double-buffered across segments) up to MP = 128, one
+// above.  The w_hat slots (one per unit: two groups of 64 columns) take the
+// columns from kACol0 up.
+__host__ __device__ constexpr int n_acc(int mp) { return mp <= 128 ? 2 : 1; }
+__host__ __device__ constexpr int n_aslots(int mp) {
+  return (512 - n_acc(mp) * mp) / 128 > 3 ? 3 : (512 - n_acc(mp) * mp) / 128;
 }
-// w_hat lives in shared memory: kABufs buffers, each one 64-input half of a
-// unit (2 tiles x 128 rows x 128 bytes, K-major with the 128-byte swizzle, the
-// layout the MMA's shared-memory descriptor reads).
-constexpr int kABufs = 4;
-constexpr int kMaxABufs = kABufs;
-constexpr int kTileBytes = 128 * 128;
-constexpr int kABufBytes = 2 * kTileBytes;
 
 // Unit u of the range partition: the CTA whose range holds it.
 __host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
@@ -245,51 +245,58 @@ __host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
 }
 
 template <int MP>
-__global__ void __maxnreg__(96)
+__global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tx) {
-  constexpr int kXHalf = MP * 128;                // one 64-input half of the x tile
-  constexpr int kStageBytes = kCodeBytes + 2 * kXHalf;
+  constexpr int kXBox = MP * 128;          // one 64-input box of x
+  constexpr int kXStage = 2 * kXBox;       // one group of x
   constexpr uint32_t kIdesc = idesc_f16(MP);
-  constexpr uint32_t kTmemCols = tmem_cols(MP);
-  static_assert(kABufs >= 4, "a unit writes two w_hat buffers; four keep the MMAs one unit behind");
-  static_assert(kStageBytes % 1024 == 0, "w_hat buffers must stay 1024-byte aligned");
+  constexpr int kAcc = n_acc(MP);
+  constexpr int kASlots = n_aslots(MP);
+  constexpr uint32_t kACol0 = kTmemCols - 128u * kASlots;
+  static_assert(kAcc * MP <= static_cast<int>(kACol0), "accumulators and w_hat slots exceed tensor memory");
+  static_assert(kASlots >= 2, "w_hat needs at least two slots");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = a.stages;
-  uint8_t* stages = smem;                        // S x kStageBytes: code tile, then x tile
-  uint8_t* abuf = stages + S * kStageBytes;      // kABufs x kABufBytes of w_hat
-  uint64_t* bars = reinterpret_cast<uint64_t*>(abuf + kABufs * kABufBytes);
-  uint64_t* full = bars;                         // [S] codes and x landed
-  uint64_t* rempty = bars + kMaxStages;          // [S] codes read and x consumed
-  uint64_t* wfull = bars + 2 * kMaxStages;       // [kABufs] w_hat half written to shared memory
-  uint64_t* wempty = wfull + kMaxABufs;          // [kABufs] w_hat half consumed by the MMAs
-  uint64_t* afull = wempty + kMaxABufs;          // [2] accumulator complete
-  uint64_t* aempty = afull + 2;                  // [2] accumulator read out
-  uint64_t* tdown = aempty + 2;                  // teardown: all MMAs complete
+  const int Sc = a.sc, Sx = a.sx;
+  uint8_t* cstage = smem;                                  // Sc x 16 KiB of codes
+  uint8_t* xstage = cstage + Sc * kCodeStage;              // Sx x kXStage of x
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xstage + Sx * kXStage);
+  uint64_t* cfull = bars;                                  // [Sc] codes landed
+  uint64_t* cempty = cfull + kMaxCodeStages;               // [Sc] codes read
+  uint64_t* xfull = cempty + kMaxCodeStages;               // [Sx] x landed
+  uint64_t* xempty = xfull + kMaxXStages;                  // [Sx] x consumed by the MMAs
+  uint64_t* afull = xempty + kMaxXStages;                  // [kASlots] w_hat written
+  uint64_t* aempty = afull + 3;                            // [kASlots] w_hat consumed
+  uint64_t* accfull = aempty + 3;                          // [kAcc] segment's MMAs complete
+  uint64_t* accempty = accfull + 2;                        // [kAcc] accumulator read out
+  uint64_t* tdown = accempty + 2;                          // teardown: all MMAs complete
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tdown + 1);
   volatile uint32_t* abort_flag = tslot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int base = a.total_units / static_cast<int>(gridDim.x);
-  const int rem = a.total_units - base * static_cast<int>(gridDim.x);
-  const int bx = static_cast<int>(blockIdx.x);
+  const int grid = static_cast<int>(gridDim.x), bx = static_cast<int>(blockIdx.x);
+  const int base = a.total / grid, rem = a.total - base * grid;
   const int u0 = bx * base + min(bx, rem);
   const int cnt = base + (bx < rem ? 1 : 0);
-  const int rb0 = u0 / a.Kg;
+  const int P = a.P;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&rempty[s], kDqWarps + 1);  // dequantization warps + 1 MMA commit
+    for (int s = 0; s < Sc; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], kDqWarps);
     }
-    for (int b = 0; b < kABufs; ++b) {
-      mbar_init(&wfull[b], kDqWarps);
-      mbar_init(&wempty[b], 1);
+    for (int s = 0; s < Sx; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&afull[b], 1);
-      mbar_init(&aempty[b], kDqWarps);
+    for (int b = 0; b < kASlots; ++b) {
+      mbar_init(&afull[b], kDqWarps);
+      mbar_init(&aempty[b], 1);
+    }
+    for (int b = 0; b < kAcc; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], kEpiWarps);
     }
     mbar_init(tdown, 1);
     *abort_flag = 0;
@@ -300,90 +307,99 @@ __global__ void __maxnreg__(96)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  // the next kernel on the stream (the partial-sum finalize) may begin launching
+  // the next kernel on the stream may begin its prologue (it waits for this
+  // grid's completion before it reads y or reuses the workspace)
   griddep_launch_dependents();
 
-  if (warp == kProducerWarp) {
-    // ---------------- producer: tensor copies of codes and x ----------------
+  if (warp == kCodeWarp) {
+    // ---------------- codes: one tensor copy per unit ----------------
     if (lane == 0) {
-      const uint64_t pol_q = l2_evict_first_policy();
-      const uint64_t pol_x = l2_evict_last_policy();
-      auto code_copy = [&](int i) {
-        const int u = u0 + i, rb = u / a.Kg, g = u - rb * a.Kg;
-        const int s = i % S;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(stages + s * kStageBytes, &tq, g * 16, rb * kRows, &full[s], pol_q);
-      };
-      auto x_copy = [&](int i) {
-        const int g = (u0 + i) % a.Kg;
-        const int s = i % S;
-        uint8_t* xs = stages + s * kStageBytes + kCodeBytes;
-        tma_load_2d(xs, &tx, g * 128, 0, &full[s], pol_x);
-        tma_load_2d(xs + kXHalf, &tx, g * 128 + 64, 0, &full[s], pol_x);
-      };
-      // the weights do not depend on the previous kernel: start streaming them first
-      const int pre = min(S, cnt);
-      for (int i = 0; i < pre; ++i) code_copy(i);
-      griddep_wait();  // x may be the previous kernel's output
-      for (int i = 0; i < pre; ++i) x_copy(i);
-      int issued = pre;
-      for (int i = pre; i < cnt; ++i) {
-        const int s = i % S;
-        if (!wait_or_abort(&rempty[s], static_cast<uint32_t>(i / S - 1) & 1u, abort_flag, a.ws_status)) break;
-        code_copy(i);
-        x_copy(i);
+      const uint64_t pol = l2_evict_first_policy();
+      int issued = 0;
+      // the weights do not depend on the previous kernel: no griddepcontrol.wait
+      for (int i = 0; i < cnt; ++i) {
+        const int s = i % Sc;
+        if (i >= Sc && !wait_or_abort(&cempty[s], static_cast<uint32_t>(i / Sc - 1) & 1u, abort_flag, a.status))
+          break;
+        const int u = u0 + i, t = u / P, p = u - t * P;
+        mbar_arrive_expect_tx(&cfull[s], kCodeStage);
+        tma_load_2d(cstage + s * kCodeStage, &tq, p * 32, t * kRows, &cfull[s], pol);
         issued = i + 1;
       }
-      // copies still in flight must land before the CTA may exit
-      for (int j = max(0, issued - S); j < issued; ++j)
-        mbar_wait_bounded(&full[j % S], static_cast<uint32_t>(j / S) & 1u);
+      for (int j = max(0, issued - Sc); j < issued; ++j)
+        mbar_wait_bounded(&cfull[j % Sc], static_cast<uint32_t>(j / Sc) & 1u);
+    }
+  } else if (warp == kXWarp) {
+    // ---------------- x: one stage per group ----------------
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_last_policy();
+      griddep_wait();  // x may be the previous kernel's output
+      int j = 0;
+      bool ok = true;
+      for (int i = 0; i < cnt && ok; ++i) {
+        const int u = u0 + i, p = u % P;
+        for (int h = 0; h < 2; ++h) {
+          const int g = 2 * p + h;
+          if (g >= a.G) break;
+          const int s = j % Sx;
+          if (j >= Sx && !wait_or_abort(&xempty[s], static_cast<uint32_t>(j / Sx - 1) & 1u, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = xstage + s * kXStage;
+          mbar_arrive_expect_tx(&xfull[s], kXStage);
+          tma_load_2d(dst, &tx, g * 128, 0, &xfull[s], pol);
+          tma_load_2d(dst + kXBox, &tx, g * 128 + 64, 0, &xfull[s], pol);
+          ++j;
+        }
+      }
+      for (int jj = max(0, j - Sx); jj < j; ++jj)
+        mbar_wait_bounded(&xfull[jj % Sx], static_cast<uint32_t>(jj / Sx) & 1u);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      bool any = false;
-      int hb = 0, f = 0;
-      for (int i = 0; i < cnt; ++i) {
-        const int s = i % S;
-        const int g = (u0 + i) % a.Kg;
-        const bool first = (i == 0) || (g == 0);
-        const bool last = (i == cnt - 1) || (g == a.Kg - 1);
-        const int ab = f & 1;
-        if (first && f >= 2 && !wait_or_abort(&aempty[ab], static_cast<uint32_t>(f / 2 - 1) & 1u, abort_flag, a.ws_status))
+      bool any = false, ok = true;
+      int j = 0, seg = 0;
+      for (int i = 0; i < cnt && ok; ++i) {
+        const int u = u0 + i, p = u % P;
+        const bool first = (i == 0) || (p == 0);
+        const bool last = (i == cnt - 1) || (p == P - 1);
+        const int ab = seg % kAcc;
+        if (first && seg >= kAcc &&
+            !wait_or_abort(&accempty[ab], static_cast<uint32_t>(seg / kAcc - 1) & 1u, abort_flag, a.status))
           break;
-        if (!wait_or_abort(&full[s], static_cast<uint32_t>(i / S) & 1u, abort_flag, a.ws_status)) break;
-        bool ok = true;
-        const uint8_t* xs = stages + s * kStageBytes + kCodeBytes;
+        const int b = i % kASlots;
+        if (!wait_or_abort(&afull[b], static_cast<uint32_t>(i / kASlots) & 1u, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t d = tbase + static_cast<uint32_t>(ab * MP);
         for (int h = 0; h < 2; ++h) {
-          const int b = hb % kABufs;
-          if (!wait_or_abort(&wfull[b], static_cast<uint32_t>(hb / kABufs) & 1u, abort_flag, a.ws_status)) {
+          const int g = 2 * p + h;
+          if (g >= a.G) break;
+          const int s = j % Sx;
+          if (!wait_or_abort(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // Addresses computed once per half: the B descriptor's start-address
-          // field advances by 32 bytes (2 in 16-byte units) per 16 inputs, A
-          // and D are tensor-memory columns at fixed offsets.  This thread
-          // shares its scheduler with dequantizing warps, so few instructions
-          // per MMA matter.
-          const uint64_t bd0 = sw128_desc(xs + h * kXHalf);
-          const uint64_t ad0 = sw128_desc(abuf + b * kABufBytes);
-          const uint32_t d0 = tbase + static_cast<uint32_t>(ab * 2 * MP);
-          const bool acc0 = !(first && h == 0);
+          const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * 128 + h * 64);
+          const uint64_t bd0 = sw128_desc(xstage + s * kXStage);
+          const uint64_t bd1 = sw128_desc(xstage + s * kXStage + kXBox);
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ss(d0 + t * MP, ad0 + t * (kTileBytes >> 4) + 2 * kk, bd0 + 2 * kk, kIdesc, kk > 0 || acc0);
+          for (int kk = 0; kk < 8; ++kk) {
+            // the descriptor's start address advances 32 bytes (2 x 16) per 16 inputs
+            const uint64_t bd = (kk < 4 ? bd0 : bd1) + 2u * static_cast<uint32_t>(kk & 3);
+            mma_f16_ts(d, acol + 8u * kk, bd, kIdesc, !(first && h == 0 && kk == 0));
+          }
           any = true;
-          mma_commit(&wempty[b]);
-          ++hb;
+          mma_commit(&xempty[s]);
+          ++j;
         }
         if (!ok) break;
-        mma_commit(&rempty[s]);
+        mma_commit(&aempty[b]);
         if (last) {
-          mma_commit(&afull[ab]);
-          ++f;
+          mma_commit(&accfull[ab]);
+          ++seg;
         }
       }
       if (any) {
@@ -391,153 +407,166 @@ __global__ void __maxnreg__(96)
         mbar_wait_bounded(tdown, 0);
       }
     }
-  } else if (warp < kDqWarps) {
-    // ---------------- dequantization and epilogue ----------------
-    // Warp w: tile t = (w >> 2) & 1, TMEM lane quarter q = w & 3, part p = w >> 3.
-    // Its lanes own rows t*128 + q*32 + lane of the block; of each 64-input half
-    // of a group it converts words 4p .. 4p + 3 (TMEM columns 16p .. 16p + 15 of
-    // the tile), and at the end of a row block it reads out accumulator columns
-    // p*MP/2 .. (p+1)*MP/2 - 1 of its rows.
-    const int t = (warp >> 2) & 1, q = warp & 3, p = warp >> 3;
-    const int rloc = t * 128 + q * 32 + lane;
-    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    // this lane's w_hat row in a buffer: tile t, row q * 32 + lane, 128 bytes
-    // with the 16-byte chunk j at j ^ (row & 7)
-    const int arow = q * 32 + lane;
-    const uint32_t arow0 = smem_u32(abuf) + static_cast<uint32_t>(t * kTileBytes + arow * 128);
-    const uint32_t asw = static_cast<uint32_t>(arow & 7);
-    const uint32_t st0 = smem_u32(stages);
-    const uint32_t sw_ld = static_cast<uint32_t>((rloc >> 1) & 3);
-    // Delta and z come a block of W groups at a time (W = 1, 2, 4 or 8 divides
-    // K / 128, so the W values of a row are one aligned load), one block ahead.
-    const int W = a.dz_w;
-    uint32_t dc[4], zc[4], dn[4], zn[4];
-    auto issue_dz = [&](int ub) {
-      const int rb = ub / a.Kg, g = ub - rb * a.Kg, g0 = g & ~(W - 1);
-      const int n = rb * kRows + rloc;
-      if (n < a.N) {
-        const size_t o = static_cast<size_t>(n) * a.Kg + g0;
-        ld_nc_halves(a.scales + o, W, dn);
-        ld_nc_halves(a.zeros + o, W, zn);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dn[j] = zn[j] = 0;
-      }
-    };
-    int hb = 0, f = 0, start = 0;
-    int pend = -1, pend_rb = 0, pend_contrib = 0;  // a row block whose accumulator awaits read-out
-    bool ok = true;
-    // Read-out of the accumulator of flush number f (row block rb, `contrib` units).
-    auto flush = [&](int fl, int rb, int contrib) {
-      const int ab = fl & 1;
-      const bool okw = wait_or_abort(&afull[ab], static_cast<uint32_t>(fl / 2) & 1u, abort_flag, a.ws_status);
-      if (__any_sync(0xffffffffu, !okw)) {
-        ok = false;
-        return;
-      }
-      tc_fence_after();
-      const bool owner = contrib == a.Kg;
-      const int n = rb * kRows + rloc;
-      // a CTA has at most two partial row blocks: the one its range starts in
-      // (slot 0) and the one it ends in (slot 1); blocks in between are whole
-      float4* slot = a.ws_part + static_cast<size_t>(bx * 2 + (rb == rb0 ? 0 : 1)) * (kRows * MP / 4);
-#pragma unroll
-      for (int c = 0; c < MP / 16; ++c) {
-        const int m0 = p * (MP / 2) + c * 8;
-        float v[8];
-        tmem_ld8(tbase + lane_addr + static_cast<uint32_t>(ab * 2 * MP + t * MP + m0), v);
-        if (n < a.N) {
-          if (owner) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (m0 + j < a.M) a.y[static_cast<size_t>(m0 + j) * a.N + n] = __float2half_rn(v[j]);
-          } else {
-            slot[(m0 / 4) * kRows + rloc] = make_float4(v[0], v[1], v[2], v[3]);
-            slot[(m0 / 4 + 1) * kRows + rloc] = make_float4(v[4], v[5], v[6], v[7]);
-          }
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
+    // ---------------- dequantization into tensor memory ----------------
+    const int q = warp & 3, h = (warp - kDqWarp0) >> 2;
+    const int r = q * 32 + lane;  // row within the tile
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + static_cast<uint32_t>(h * 64);
+    const uint32_t row_smem = smem_u32(cstage) + static_cast<uint32_t>(r * 128);
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    // Delta and z of the next units, fetched a few units ahead
+    constexpr int kLook = 3;
+    uint16_t pd[kLook], pz[kLook];
+    auto fetch = [&](int i, uint16_t& dv, uint16_t& zv) {
+      dv = zv = 0;
+      if (i < cnt) {
+        const int u = u0 + i, t = u / P, g = 2 * (u - t * P) + h;
+        const int n = t * kRows + r;
+        if (n < a.N && g < a.G) {
+          const size_t o = static_cast<size_t>(n) * a.G + g;
+          dv = ld_nc_u16(a.scales + o);
+          zv = ld_nc_u16(a.zeros + o);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&aempty[ab]);
     };
-    const int uend = u0 + cnt;
-    int cur_end = u0;  // the Delta / z block in dc / zc covers units up to cur_end - 1
-    issue_dz(u0);
-    for (int i = 0; i < cnt && ok; ++i) {
-      const int u = u0 + i;
-      const int g = u % a.Kg;
-      if (u >= cur_end) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          dc[j] = dn[j];
-          zc[j] = zn[j];
-        }
-        cur_end = u + min(W - (g & (W - 1)), a.Kg - g);
-        if (cur_end < uend) issue_dz(cur_end);
+    for (int l = 0; l < kLook; ++l) fetch(l, pd[l], pz[l]);
+    for (int i = 0; i < cnt; ++i) {
+      const int u = u0 + i, t = u / P, p = u - t * P;
+      const bool valid = 2 * p + h < a.G;
+      const uint16_t dv = pd[0], zv = pz[0];
+#pragma unroll
+      for (int l = 0; l + 1 < kLook; ++l) {
+        pd[l] = pd[l + 1];
+        pz[l] = pz[l + 1];
       }
-      const int s = i % S;
-      const bool okf = wait_or_abort(&full[s], static_cast<uint32_t>(i / S) & 1u, abort_flag, a.ws_status);
-      if (__any_sync(0xffffffffu, !okf)) {
-        ok = false;
-        break;
+      fetch(i + kLook, pd[kLook - 1], pz[kLook - 1]);
+      const int s = i % Sc;
+      const bool okc = wait_or_abort(&cfull[s], static_cast<uint32_t>(i / Sc) & 1u, abort_flag, a.status);
+      if (__any_sync(0xffffffffu, !okc)) break;
+      uint4 cw[4];
+      if (valid) {
+        const uint32_t row = row_smem + static_cast<uint32_t>(s * kCodeStage);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cw[c] = lds128(row + (((static_cast<uint32_t>(4 * h + c)) ^ rsw) << 4));
       }
-      const uint32_t row = st0 + static_cast<uint32_t>(s * kStageBytes + rloc * 64);
-      const uint4 c0 = lds128(row + ((static_cast<uint32_t>(p) ^ sw_ld) << 4));
-      const uint4 c1 = lds128(row + ((static_cast<uint32_t>(2 + p) ^ sw_ld) << 4));
+      // every lane's reads are ordered before the copy that refills the stage
       release_stage_reads();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&rempty[s]);  // codes are in registers
-      const uint32_t dv = pick_half(dc, g & (W - 1)), zv = pick_half(zc, g & (W - 1));
-      const __half2 dd = as_h2(dv | (dv << 16));
-      // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
-      const __half zh = __hneg(__hadd(__ushort_as_half(static_cast<unsigned short>(zv)), __float2half_rn(1024.0f)));
-      const __half2 zz = __halves2half2(zh, zh);
-      const int b0 = hb % kABufs, b1 = (hb + 1) % kABufs;
-      bool okw = hb < kABufs ||
-                 wait_or_abort(&wempty[b0], static_cast<uint32_t>(hb / kABufs - 1) & 1u, abort_flag, a.ws_status);
-      okw = okw && (hb + 1 < kABufs || wait_or_abort(&wempty[b1], static_cast<uint32_t>((hb + 1) / kABufs - 1) & 1u,
-                                                    abort_flag, a.ws_status));
-      if (__any_sync(0xffffffffu, !okw)) {
-        ok = false;
-        break;
-      }
+      if (lane == 0) mbar_arrive(&cempty[s]);
+      const int b = i % kASlots;
+      const bool oka = i < kASlots ||
+                       wait_or_abort(&aempty[b], static_cast<uint32_t>(i / kASlots - 1) & 1u, abort_flag, a.status);
+      if (__any_sync(0xffffffffu, !oka)) break;
       tc_fence_after();
-      {
-        const uint32_t r0 = arow0 + static_cast<uint32_t>(b0 * kABufBytes);
-        const uint32_t r1 = arow0 + static_cast<uint32_t>(b1 * kABufBytes);
-        const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
-        const uint32_t cv[4] = {c1.x, c1.y, c1.z, c1.w};
+      if (valid) {
+        const __half2 dd = as_h2(static_cast<uint32_t>(dv) | (static_cast<uint32_t>(dv) << 16));
+        // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
+        const __half zh = __hneg(__hadd(__ushort_as_half(zv), __float2half_rn(1024.0f)));
+        const __half2 nz = __halves2half2(zh, zh);
+        const uint32_t col = lane_base + static_cast<uint32_t>(b * 128);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t j = static_cast<uint32_t>(4 * p + i);  // word of the half = 16-byte chunk
-          sts128(r0 + (((j ^ asw) & 7u) << 4), dq_word(cw[i], zz, dd));
-          sts128(r1 + (((j ^ asw) & 7u) << 4), dq_word(cv[i], zz, dd));
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t wv[4] = {cw[c].x, cw[c].y, cw[c].z, cw[c].w};
+          uint32_t v[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            v[4 * k + 0] = dq_pair(wv[k], nz, dd);
+            v[4 * k + 1] = dq_pair(wv[k] >> 4, nz, dd);
+            v[4 * k + 2] = dq_pair(wv[k] >> 8, nz, dd);
+            v[4 * k + 3] = dq_pair(wv[k] >> 12, nz, dd);
+          }
+          tmem_st16(col + static_cast<uint32_t>(16 * c), v);
         }
-        // the MMAs read these rows through the async proxy
-        fence_proxy_async_smem();
+        tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&wfull[b0]);
-        mbar_arrive(&wfull[b1]);
-      }
-      hb += 2;
-      // the previous row block's accumulator is complete by now: read it out
-      if (pend >= 0) {
-        flush(pend, pend_rb, pend_contrib);
-        pend = -1;
-        if (!ok) break;
-      }
-      if (i == 0 || g == 0) start = i;
-      if (i == cnt - 1 || g == a.Kg - 1) {
-        pend = f++;
-        pend_rb = u / a.Kg;
-        pend_contrib = i - start + 1;
-      }
+      if (lane == 0) mbar_arrive(&afull[b]);
     }
-    if (ok && pend >= 0) flush(pend, pend_rb, pend_contrib);
+  } else if (warp >= kEpiWarp0) {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    griddep_wait();  // y and the workspace slots may still be in use by the previous kernel
+    int seg = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const int u = u0 + i, t = u / P, p = u - t * P;
+      if (!(i == cnt - 1 || p == P - 1)) continue;  // only at the end of a segment
+      const int ia = (seg == 0) ? 0 : i - p;        // segment start (a later segment starts at p = 0)
+      const bool covers_first = (u0 + ia) == t * P;
+      const bool covers_last = (p == P - 1);
+      const int ab = seg % kAcc;
+      const bool okw = wait_or_abort(&accfull[ab], static_cast<uint32_t>(seg / kAcc) & 1u, abort_flag, a.status);
+      if (__any_sync(0xffffffffu, !okw)) break;
+      tc_fence_after();
+      const int n = t * kRows + r;
+      const uint32_t acc = lane_base + static_cast<uint32_t>(ab * MP);
+      bool okw2 = true;
+      if (!covers_first) {
+        // a contributor: publish the partial tile; each epilogue warp adds 1 to
+        // the CTA's flag once its rows are stored, so 4 means the tile is complete
+        float4* slot = a.part + static_cast<size_t>(bx) * (MP / 4) * kRows;
+#pragma unroll 1
+        for (int c = 0; c < MP / 16; ++c) {
+          float v[16];
+          tmem_ld16(acc + static_cast<uint32_t>(16 * c), v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            slot[(4 * c + e) * kRows + r] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(a.flags + bx, 1u);
+        }
+      } else {
+        // alone, or the owner: add the later contributors' partial tiles in CTA order
+        const int c_hi = covers_last ? bx : owner_cta(t * P + P - 1, base, rem);
+        for (int cc = bx + 1; cc <= c_hi && okw2; ++cc) {
+          bool okf = true;
+          if (lane == 0) okf = wait_flag(a.flags + cc, kEpiWarps, abort_flag, a.status);
+          okw2 = __shfl_sync(0xffffffffu, okf, 0);
+          if (okw2) (void)ld_acquire(a.flags + cc);  // every lane acquires what the publisher released
+        }
+        if (okw2) {
+#pragma unroll 1
+          for (int c = 0; c < MP / 16; ++c) {
+            float v[16];
+            tmem_ld16(acc + static_cast<uint32_t>(16 * c), v);
+            for (int cc = bx + 1; cc <= c_hi; ++cc) {
+              const float4* slot = a.part + static_cast<size_t>(cc) * (MP / 4) * kRows;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float4 w = __ldcg(slot + (4 * c + e) * kRows + r);
+                v[4 * e] += w.x;
+                v[4 * e + 1] += w.y;
+                v[4 * e + 2] += w.z;
+                v[4 * e + 3] += w.w;
+              }
+            }
+            if (n < a.N) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (16 * c + e < a.M) a.y[static_cast<size_t>(16 * c + e) * a.N + n] = __float2half_rn(v[e]);
+            }
+          }
+          // Each owner warp adds 1 once it has read a flag's tile; the last of
+          // the four (seeing 2 x 4 - 1) puts the flag back to zero for the next
+          // call, which starts only after this grid has ended.
+          __syncwarp();
+          if (lane == 0)
+            for (int cc = bx + 1; cc <= c_hi; ++cc)
+              if (atomicAdd(a.flags + cc, 1u) == 2 * kEpiWarps - 1) atomicExch(a.flags + cc, 0u);
+        }
+      }
+      if (!okw2) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+      ++seg;
+    }
   }
 
   tc_fence_before();
@@ -548,67 +577,22 @@ __global__ void __maxnreg__(96)
   }
 }
 
-// Sums the partial-sum slots of the row blocks no single CTA covered, in CTA
-// order (so y does not depend on timing), and writes y.  Block (rb, cy) covers
-// the 256 rows of row block rb and tokens 16 cy .. 16 cy + 15; thread (r, j)
-// takes row r and tokens 16 cy + 4 j .. + 3.  A thread issues the loads of up
-// to kFinBatch contributing CTAs before adding any of them, so the slots cost
-// one trip to L2 per batch rather than one per CTA.
-constexpr int kFinBatch = 8;
-template <int MP>
-__global__ void __launch_bounds__(kRows * 4) gemm_tc_finalize(const TcArgs a, int grid_main) {
-  // the next layer's main kernel may start its prologue and weight prefetch; it
-  // reads x (this kernel's y) only after its own griddepcontrol.wait
-  griddep_launch_dependents();
-  griddep_wait();
-  const int rb = blockIdx.x;
-  const int base = a.total_units / grid_main;
-  const int rem = a.total_units - base * grid_main;
-  const int c0 = owner_cta(rb * a.Kg, base, rem);
-  const int c1 = owner_cta(rb * a.Kg + a.Kg - 1, base, rem);
-  if (c0 == c1) return;  // one CTA covered the row block and wrote y itself
-  const int r = threadIdx.x, cg = blockIdx.y * 4 + threadIdx.y;
-  const int n = rb * kRows + r;
-  if (n >= a.N || cg >= MP / 4) return;
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  for (int cb = c0; cb <= c1; cb += kFinBatch) {
-    float4 v[kFinBatch];
-#pragma unroll
-    for (int j = 0; j < kFinBatch; ++j) {
-      const int c = cb + j;
-      if (c <= c1) {
-        const int rbc = (c * base + min(c, rem)) / a.Kg;  // row block where c's range starts
-        v[j] = __ldcg(a.ws_part + static_cast<size_t>(c * 2 + (rb == rbc ? 0 : 1)) * (kRows * MP / 4) + cg * kRows + r);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kFinBatch; ++j) {
-      if (cb + j <= c1) {
-        s0 += v[j].x;
-        s1 += v[j].y;
-        s2 += v[j].z;
-        s3 += v[j].w;
-      }
-    }
-  }
-  const float sv[4] = {s0, s1, s2, s3};
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    if (cg * 4 + j < a.M) a.y[static_cast<size_t>(cg * 4 + j) * a.N + n] = __float2half_rn(sv[j]);
-}
-
-int stages_for(int mp) {
-  const int stage = kCodeBytes + 2 * mp * 128;
-  int s = (kMaxSmem - 1024 - kCtrlBytes - kABufs * kABufBytes) / stage;
-  return s > kMaxStages ? kMaxStages : s;
+// Ring depths: x stages for about 64 KiB of x (2 to 8), the rest of shared
+// memory for code stages (at most 12).
+void ring_depths(int mp, int& sc, int& sx) {
+  const int xs = 2 * mp * 128;
+  sx = (64 * 1024) / xs;
+  sx = sx < 2 ? 2 : (sx > kMaxXStages ? kMaxXStages : sx);
+  sc = (kMaxSmem - 1024 - kCtrlBytes - sx * xs) / kCodeStage;
+  sc = sc > kMaxCodeStages ? kMaxCodeStages : sc;
 }
 
 template <int MP>
 cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap& tx, int grid, cudaStream_t st) {
   TcArgs a = a0;
-  a.stages = stages_for(MP);
-  if (a.stages < 2) return cudaErrorNotSupported;
-  const int smem = 1024 + a.stages * (kCodeBytes + 2 * MP * 128) + kABufs * kABufBytes + kCtrlBytes;
+  ring_depths(MP, a.sc, a.sx);
+  if (a.sc < 2) return cudaErrorNotSupported;
+  const int smem = 1024 + a.sc * kCodeStage + a.sx * 2 * MP * 128 + kCtrlBytes;
   cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_kernel<MP>),
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -624,52 +608,41 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<MP>, a, tq, tx);
   if (e != cudaSuccess) return e;
-  // the partial sums of row blocks shared by several CTAs; asking for the same
-  // shared-memory carveout as the main kernel spares the SMs a reconfiguration
-  // between the two launches
-  e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_finalize<MP>), cudaFuncAttributePreferredSharedMemoryCarveout,
-                       cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
-  const int row_blocks = (a.N + kRows - 1) / kRows;
-  cudaLaunchConfig_t fin = {};
-  fin.gridDim = dim3(row_blocks, (MP / 4 + 3) / 4);
-  fin.blockDim = dim3(kRows, 4);
-  fin.stream = st;
-  fin.attrs = attr;
-  fin.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&fin, gemm_tc_finalize<MP>, a, grid);
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
-}
-
-// The token tile of a launch: M rounded up to 16 up to 64, then 96 or 128.
-int tc_tile(int M) {
-  const int mp = (M + 15) / 16 * 16;
-  return mp <= 64 ? mp : (mp <= 96 ? 96 : 128);
 }
 
 }  // namespace
 
+// The token tile of a launch of M <= kMaxM tokens.
+int tc_tile(int M) {
+  const int mp = (M + 15) / 16 * 16;
+  if (mp <= 32) return mp <= 16 ? 16 : 32;
+  if (mp <= 64) return 64;
+  if (mp <= 96) return 96;
+  if (mp <= 128) return 128;
+  return mp <= 192 ? 192 : 256;
+}
+
 size_t tc_partial_bytes(int M) {
   const size_t mp = static_cast<size_t>(tc_tile(M));
-  return 2 * static_cast<size_t>(device_sm_count()) * kRows * mp * 4;
+  return static_cast<size_t>(device_sm_count()) * kRows * mp * 4;
 }
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
-  if (p.M < 1 || p.M > kMaxM || !ws.part) return cudaErrorNotSupported;
+  if (p.M < 1 || p.M > kMaxM || !ws.part || !ws.flags) return cudaErrorNotSupported;
   const int mp = tc_tile(p.M);
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
 
-  // codes: u32 [N][K/8], boxes of 256 rows x 16 words (one group), 64-byte swizzle
+  // codes: u32 [N][K/8], boxes of 128 rows x 32 words (a pair of groups), 128-byte swizzle
   CUtensorMap tq, tx;
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K / 8), static_cast<cuuint64_t>(p.N)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 8) * 4};
-    const cuuint32_t box[2] = {16, static_cast<cuuint32_t>(kRows)};
+    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
@@ -686,28 +659,29 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
   }
 
   TcArgs a;
-  a.qweight = p.qweight;
   a.scales = p.scales;
   a.zeros = p.zeros;
   a.y = p.y;
-  a.ws_part = reinterpret_cast<float4*>(ws.part);
-  a.ws_status = ws.status;
+  a.part = reinterpret_cast<float4*>(ws.part);
+  a.flags = ws.flags;
+  a.status = ws.status;
   a.M = p.M;
   a.N = p.N;
-  a.Kw = p.K / 8;
-  a.Kg = p.K / kGroup;
-  a.dz_w = a.Kg % 8 == 0 ? 8 : (a.Kg % 4 == 0 ? 4 : (a.Kg % 2 == 0 ? 2 : 1));
-  const int row_blocks = (p.N + kRows - 1) / kRows;
-  a.total_units = row_blocks * a.Kg;
-  a.stages = 0;
-  const int grid = min(device_sm_count(), a.total_units);
+  a.G = p.K / kGroup;
+  a.P = (a.G + 1) / 2;
+  const int tiles = (p.N + kRows - 1) / kRows;
+  a.total = tiles * a.P;
+  a.sc = a.sx = 0;
+  const int grid = min(device_sm_count(), a.total);
+  if (grid > kMaxFlags) return cudaErrorNotSupported;
   switch (mp) {
     case 16: return launch_mp<16>(a, tq, tx, grid, st);
     case 32: return launch_mp<32>(a, tq, tx, grid, st);
-    case 48: return launch_mp<48>(a, tq, tx, grid, st);
     case 64: return launch_mp<64>(a, tq, tx, grid, st);
     case 96: return launch_mp<96>(a, tq, tx, grid, st);
-    default: return launch_mp<128>(a, tq, tx, grid, st);
+    case 128: return launch_mp<128>(a, tq, tx, grid, st);
+    case 192: return launch_mp<192>(a, tq, tx, grid, st);
+    default: return launch_mp<256>(a, tq, tx, grid, st);
   }
 }
 

@@ -12,7 +12,8 @@ namespace w4a16 {
 
 constexpr int kGroup = 128;        // group size along K (the only one supported)
 constexpr int kMaxGemvM = 4;       // largest M the CUDA-core GEMV handles
-constexpr int kMaxM = 128;         // largest M of one launch sequence; larger M runs in chunks of it
+constexpr int kMaxM = 256;         // largest M of one launch sequence; larger M runs in chunks of it
+constexpr int kMaxFlags = 1024;    // partial-tile flags of the tensor-core path (one per CTA)
 
 // Replaces the calling thread's message returned by w4a16_last_error().
 void set_last_error(const char* msg);
@@ -35,18 +36,21 @@ cudaError_t launch_act_scale(const __half* X, int T, int K, double alpha, __half
 cudaError_t launch_quantize_pack(const __half* W, const __half* s, int N, int K, int bits, int mode,
                                  uint32_t* qweight, __half* scales, __half* zeros, cudaStream_t st);
 
-// Workspace: [status word | padding to 16 B] [row-block counters, padded to
-// 16 B] [fp32 partial sums M x N of the CUDA-core GEMV, M <= 4] and, for
-// M >= 5, after room for 4 x N GEMV partials: the tensor-core path's
-// partial-sum slots (2 per CTA of 256 x MP fp32, MP the launch's token tile).
-// The counters and GEMV partials must be zero when a kernel starts and are
-// left zero; the slots are scratch, written before they are read.
+// Workspace: [status word | padding to 16 B] [kMaxFlags partial-tile flags of
+// the tensor-core path] [row-block counters, padded to 16 B] [fp32 partial sums
+// M x N of the CUDA-core GEMV, M <= 4] and, for M >= 5, after room for 4 x N
+// GEMV partials: the tensor-core path's partial tiles (one per CTA of 128 x MP
+// fp32, MP the launch's token tile).  The flags, counters and GEMV partials must
+// be zero when a kernel starts and are left zero; the partial tiles are
+// scratch, written before they are read.
 struct Workspace {
   uint32_t* status;
+  uint32_t* flags;
   uint32_t* counters;
   float* acc;
-  float* part;  // tensor-core partial-sum slots (M >= 5 only), after the GEMV region
+  float* part;  // tensor-core partial tiles (M >= 5 only), after the GEMV region
 };
+constexpr size_t kFlagBytes = kMaxFlags * 4;
 size_t workspace_bytes(int M, int N, int K);
 Workspace carve_workspace(void* base, int M, int N, int K);
 
@@ -72,8 +76,8 @@ cudaError_t launch_gemv_mt(const GemmProblem& p, uint32_t* status, cudaStream_t 
 bool gemv_supports(int M, int K);
 cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 
-// The tensor-core GEMM (gemm_tc.cu), M = 5..128 per launch, and the bytes of
-// its partial-sum slots on the current device.
+// The tensor-core GEMM (gemm_tc.cu), M = 5..256 per launch, and the bytes of
+// its partial tiles on the current device.
 size_t tc_partial_bytes(int M);
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st);
 // One CTA waits on a shared-memory barrier that nothing completes, gives up
