@@ -296,6 +296,67 @@ W4A16_API w4a16_status gptq_quantize(const void* W, const void* X, int N, int K,
                                      size_t workspace_bytes, w4a16_stream_t stream);
 
 /*
+ * ---- W4A8 with progressive group quantization ------------------------------
+ * "MIT 6.5940 Fall 2024 Lecture 13: LLM Deployment" reading guide, §QServe
+ * (slides 47-57): 4-bit weights whose group scale is applied before the zero
+ * point, so that the dequantized weight is an int8 value; 8-bit per-token
+ * activations; int8 tensor cores; the conversion to floating point at the end.
+ * The pages give no formulas; the readings these calls implement:
+ *   level 1, per output channel n: s1[n] = fp16(max_k |W[n][k]| / 119)
+ *     (fp16(1/119) for a zero row), w8 = clip(Round(W / s1), -119, 119);
+ *   level 2, per group of 128 inputs: mx = max(max w8, 0), mn = min(min w8, 0),
+ *     s2 = max(1, ceil((mx - mn) / 15)), z2 = clip(Round(-mn / s2), 0, 15),
+ *     u = clip(Round(w8 / s2) + z2, 0, 15); zs = z2 * s2 (<= 240);
+ *   the dequantized weight is w8_hat = u * s2 - zs (always within int8);
+ *   activations, per token m: s_x[m] = fp16(max_k |x[m][k]| / 127) (fp16(1/127)
+ *     for a zero token), x8 = clip(Round(x / s_x), -127, 127);
+ *   acc[m][n] = sum_k x8[m][k] * w8_hat[n][k] exactly (int32),
+ *   y[m][n] = fp16((acc * s_x[m]) * s1[n]), each product in fp64, one rounding.
+ * Round is half-to-even; every quotient decides its integer exactly.  119 is
+ * the largest level-1 range for which no w8_hat leaves int8.
+ */
+
+/*
+ * w4a8_quantize_weight -- the two-level quantization above.
+ *   W        fp16 [N][K], row-major (device).
+ *   qweight  u32 [N][K/8] layout v1 codes (device, written).
+ *   s1       fp16 [N];  s2, zs  uint8 [N][K/group] (device, written).
+ * group == 128; K a multiple of 128, at most 65536.  Asynchronous on `stream`.
+ */
+W4A16_API w4a16_status w4a8_quantize_weight(const void* W, int N, int K, int group, uint32_t* qweight,
+                                            void* s1, uint8_t* s2, uint8_t* zs, w4a16_stream_t stream);
+
+/*
+ * w4a8_quantize_act -- per-token int8 activations.
+ *   x   fp16 [M][K] (device);  x8  int8 [M][K] (device, written);  sx  fp16 [M] (device, written).
+ * 1 <= M <= 65535.  Asynchronous on `stream`.
+ */
+W4A16_API w4a16_status w4a8_quantize_act(const void* x, int M, int K, int8_t* x8, void* sx,
+                                         w4a16_stream_t stream);
+
+/* Workspace bytes w4a8_gemm needs (0 for invalid sizes); same layout rules as w4a16_gemm's. */
+W4A16_API size_t w4a8_gemm_workspace_size(int M, int N, int K, int group);
+
+/*
+ * w4a8_gemm -- y = fp16((acc * s_x) * s1) with acc = x8 . w8_hat^T exact.
+ *   x8 int8 [M][K], sx fp16 [M] (w4a8_quantize_act);  qweight, s1, s2, zs
+ *   (w4a8_quantize_weight);  y fp16 [M][N] (written);  acc int32 [M][N] or NULL
+ *   (written when given: the exact accumulators).  All device pointers,
+ *   16-byte aligned.
+ * M = 1..4 runs on CUDA cores (dp4a, the zero point taken out once per group);
+ * larger M on the int8 tensor cores (tcgen05.mma kind::i8, w8_hat formed in
+ * registers: one multiply by s2 per four codes and a bytewise subtraction of
+ * zs), in chunks of 256 tokens.  Integer sums make y independent of the order
+ * of addition.  The workspace (w4a8_gemm_workspace_size bytes) follows the
+ * rules of w4a16_gemm's: zero-filled once by the caller, left so by each call.
+ * Errors as w4a16_gemm; w4a16_gemm_check reports wait timeouts.
+ */
+W4A16_API w4a16_status w4a8_gemm(const int8_t* x8, const void* sx, const uint32_t* qweight, const void* s1,
+                                 const uint8_t* s2, const uint8_t* zs, int M, int N, int K, int group, void* y,
+                                 int32_t* acc, void* workspace, size_t workspace_bytes,
+                                 w4a16_stream_t stream);
+
+/*
  * w4a16_gemm_check -- synchronizes `stream` and reads the workspace's device
  * status word.  Returns W4A16_ERR_DEVICE if any earlier w4a16_gemm with this
  * workspace gave up waiting for its weight tiles (bounded waits, about 2 s),

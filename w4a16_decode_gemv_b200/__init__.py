@@ -75,6 +75,14 @@ def load_library():
     lib.gptq_quantize_workspace_size.restype = sz
     lib.gptq_quantize.argtypes = [vp, vp, i, i, i, d, i, i, i, vp, vp, vp, vp, sz, vp]
     lib.gptq_quantize.restype = i
+    lib.w4a8_quantize_weight.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp]
+    lib.w4a8_quantize_weight.restype = i
+    lib.w4a8_quantize_act.argtypes = [vp, i, i, vp, vp, vp]
+    lib.w4a8_quantize_act.restype = i
+    lib.w4a8_gemm_workspace_size.argtypes = [i, i, i, i]
+    lib.w4a8_gemm_workspace_size.restype = sz
+    lib.w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, sz, vp]
+    lib.w4a8_gemm.restype = i
     lib.w4a16_gemm_check.argtypes = [vp, vp]
     lib.w4a16_gemm_check.restype = i
     lib.w4a16_wait_timeout_selftest.argtypes = [vp, i, vp]
@@ -268,6 +276,73 @@ def gemv_noalloc_timeout_selftest(limit_us: int = 1000, device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         _check(lib.w4a16_gemv_noalloc_timeout_selftest(limit_us, _stream(dev)), "w4a16_gemv_noalloc_timeout_selftest")
+
+
+def w4a8_quantize_weight(W: torch.Tensor, group: int = GROUP):
+    """W fp16 [N, K] -> (qweight int32 [N, K/8] layout v1, s1 fp16 [N], s2 uint8 [N, K/128], zs uint8 [N, K/128])."""
+    lib = load_library()
+    N, K = W.shape
+    _expect(W, torch.float16, (N, K), "W")
+    dev = W.device
+    q = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+    s1 = torch.empty((N,), dtype=torch.float16, device=dev)
+    s2 = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+    zs = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.w4a8_quantize_weight(_ptr(W), N, K, group, _ptr(q), _ptr(s1), _ptr(s2), _ptr(zs), _stream(dev)),
+               "w4a8_quantize_weight")
+    return q, s1, s2, zs
+
+
+def w4a8_quantize_act(x: torch.Tensor):
+    """x fp16 [M, K] -> (x8 int8 [M, K], s_x fp16 [M])."""
+    lib = load_library()
+    M, K = x.shape
+    _expect(x, torch.float16, (M, K), "x")
+    x8 = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    sx = torch.empty((M,), dtype=torch.float16, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(lib.w4a8_quantize_act(_ptr(x), M, K, _ptr(x8), _ptr(sx), _stream(x.device)), "w4a8_quantize_act")
+    return x8, sx
+
+
+def w4a8_gemm_workspace_size(M: int, N: int, K: int, group: int = GROUP) -> int:
+    return int(load_library().w4a8_gemm_workspace_size(M, N, K, group))
+
+
+def w4a8_gemm(x8: torch.Tensor, sx: torch.Tensor, qweight: torch.Tensor, s1: torch.Tensor, s2: torch.Tensor,
+              zs: torch.Tensor, group: int = GROUP, out: torch.Tensor | None = None, acc: bool | torch.Tensor = False,
+              workspace: torch.Tensor | None = None):
+    """y fp16 [M, N] = fp16((acc * s_x) * s1), acc = x8 . (u * s2 - zs)^T exact.
+
+    With acc=True (or an int32 [M, N] tensor) also returns the exact accumulators: (y, acc).
+    """
+    lib = load_library()
+    M, K = x8.shape
+    N = qweight.shape[0]
+    dev = x8.device
+    _expect(x8, torch.int8, (M, K), "x8")
+    _expect(sx, torch.float16, (M,), "sx")
+    _expect(qweight, torch.int32, (N, K // 8), "qweight")
+    _expect(s1, torch.float16, (N,), "s1")
+    _expect(s2, torch.uint8, (N, K // group), "s2")
+    _expect(zs, torch.uint8, (N, K // group), "zs")
+    y = torch.empty((M, N), dtype=torch.float16, device=dev) if out is None else out
+    _expect(y, torch.float16, (M, N), "out")
+    acc_t = None
+    if isinstance(acc, torch.Tensor):
+        acc_t = acc
+        _expect(acc_t, torch.int32, (M, N), "acc")
+    elif acc:
+        acc_t = torch.empty((M, N), dtype=torch.int32, device=dev)
+    need = w4a8_gemm_workspace_size(M, N, K, group)
+    if workspace is None:
+        workspace = workspace_for(dev, need)
+    with torch.cuda.device(dev):
+        _check(lib.w4a8_gemm(_ptr(x8), _ptr(sx), _ptr(qweight), _ptr(s1), _ptr(s2), _ptr(zs), M, N, K, group,
+                             _ptr(y), _ptr(acc_t) if acc_t is not None else None, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(dev)), "w4a8_gemm")
+    return (y, acc_t) if acc_t is not None else y
 
 
 def search_workspace_size(N: int, K: int, T: int, n_alpha: int, group: int = GROUP) -> int:

@@ -181,6 +181,7 @@ static SearchLayout search_layout(int N, int K, int T, int n_alpha) {
 }
 
 constexpr int kMaxAlphas = 4096;
+constexpr int kMaxW4A8K = 65536;  // |acc| < K * 127 * 127 stays below 2^31
 constexpr int kMaxSearchTokens = 1 << 20;  // the target GEMM's grid holds T / 64 in its y dimension
 
 }  // namespace w4a16
@@ -443,6 +444,80 @@ w4a16_status gptq_quantize(const void* W, const void* X, int N, int K, int T, do
     e = launch_gptq_sweep(static_cast<const __half*>(W), G, N, K, bits, static_cast<int>(mode), qweight,
                           static_cast<__half*>(scales), static_cast<__half*>(zeros), sws, st);
   if (e != cudaSuccess) return cuda_fail(e, "gptq_quantize launch");
+  return ok();
+}
+
+w4a16_status w4a8_quantize_weight(const void* W, int N, int K, int group, uint32_t* qweight, void* s1, uint8_t* s2,
+                                  uint8_t* zs, w4a16_stream_t stream) {
+  if (!W || !qweight || !s1 || !s2 || !zs) return fail(W4A16_ERR_ARG, "w4a8_quantize_weight: null pointer");
+  if (N < 1 || K < 1) return fail(W4A16_ERR_ARG, "w4a8_quantize_weight: N=%d K=%d must be >= 1", N, K);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "w4a8_quantize_weight: group=%d (only 128)", group);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "w4a8_quantize_weight: K=%d not a multiple of group=%d", K, group);
+  if (K > kMaxW4A8K) return fail(W4A16_ERR_SHAPE, "w4a8_quantize_weight: K=%d (at most %d)", K, kMaxW4A8K);
+  if (static_cast<long long>(N) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "w4a8_quantize_weight: N*K too large");
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(s1) || !aligned16(s2) || !aligned16(zs))
+    return fail(W4A16_ERR_ALIGN, "w4a8_quantize_weight: pointers must be 16-byte aligned");
+  const cudaError_t e = launch_w4a8_quantize_weight(static_cast<const __half*>(W), N, K, qweight,
+                                                    static_cast<__half*>(s1), s2, zs,
+                                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "w4a8_quantize_weight launch");
+  return ok();
+}
+
+w4a16_status w4a8_quantize_act(const void* x, int M, int K, int8_t* x8, void* sx, w4a16_stream_t stream) {
+  if (!x || !x8 || !sx) return fail(W4A16_ERR_ARG, "w4a8_quantize_act: null pointer");
+  if (M < 1 || K < 1) return fail(W4A16_ERR_ARG, "w4a8_quantize_act: M=%d K=%d must be >= 1", M, K);
+  if (M > 65535) return fail(W4A16_ERR_SHAPE, "w4a8_quantize_act: M=%d (at most 65535)", M);
+  if (static_cast<long long>(M) * K >= kMaxElems) return fail(W4A16_ERR_SHAPE, "w4a8_quantize_act: M*K too large");
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(sx))
+    return fail(W4A16_ERR_ALIGN, "w4a8_quantize_act: pointers must be 16-byte aligned");
+  const cudaError_t e = launch_w4a8_quantize_act(static_cast<const __half*>(x), M, K, x8, static_cast<__half*>(sx),
+                                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "w4a8_quantize_act launch");
+  return ok();
+}
+
+size_t w4a8_gemm_workspace_size(int M, int N, int K, int group) {
+  if (M < 1 || N < 1 || K < 1 || group != kGroup || K % group || K > kMaxW4A8K) return 0;
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(M) * K >= kMaxElems ||
+      static_cast<long long>(M) * N >= kMaxElems)
+    return 0;
+  return workspace_bytes(M < kMaxM ? M : kMaxM, N, K);
+}
+
+w4a16_status w4a8_gemm(const int8_t* x8, const void* sx, const uint32_t* qweight, const void* s1, const uint8_t* s2,
+                       const uint8_t* zs, int M, int N, int K, int group, void* y, int32_t* acc, void* workspace,
+                       size_t workspace_bytes_, w4a16_stream_t stream) {
+  if (!x8 || !sx || !qweight || !s1 || !s2 || !zs || !y) return fail(W4A16_ERR_ARG, "w4a8_gemm: null pointer");
+  if (M < 1 || N < 1 || K < 1) return fail(W4A16_ERR_ARG, "w4a8_gemm: M=%d N=%d K=%d must be >= 1", M, N, K);
+  if (group != kGroup) return fail(W4A16_ERR_UNSUPPORTED, "w4a8_gemm: group=%d (only 128)", group);
+  if (K % group) return fail(W4A16_ERR_SHAPE, "w4a8_gemm: K=%d not a multiple of group=%d", K, group);
+  if (K > kMaxW4A8K) return fail(W4A16_ERR_SHAPE, "w4a8_gemm: K=%d (at most %d)", K, kMaxW4A8K);
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(M) * K >= kMaxElems ||
+      static_cast<long long>(M) * N >= kMaxElems)
+    return fail(W4A16_ERR_SHAPE, "w4a8_gemm: N*K, M*K or M*N too large");
+  if (!aligned16(x8) || !aligned16(sx) || !aligned16(qweight) || !aligned16(s1) || !aligned16(s2) ||
+      !aligned16(zs) || !aligned16(y) || (acc && !aligned16(acc)))
+    return fail(W4A16_ERR_ALIGN, "w4a8_gemm: pointers must be 16-byte aligned");
+  const size_t need = workspace_bytes(M < kMaxM ? M : kMaxM, N, K);
+  if (!workspace || workspace_bytes_ < need)
+    return fail(W4A16_ERR_WORKSPACE, "w4a8_gemm: workspace of %zu bytes needed, %zu given", need, workspace_bytes_);
+  if (!aligned16(workspace)) return fail(W4A16_ERR_ALIGN, "w4a8_gemm: workspace must be 16-byte aligned");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  // chunks of kMaxM tokens: x8, s_x, y and acc offsets stay 16-byte aligned (kMaxM * 2 bytes per token of s_x)
+  for (int t0 = 0; t0 < M && e == cudaSuccess; t0 += kMaxM) {
+    W4A8Problem c{x8 + static_cast<size_t>(t0) * K, static_cast<const __half*>(sx) + t0, qweight,
+                  static_cast<const __half*>(s1), s2, zs, static_cast<__half*>(y) + static_cast<size_t>(t0) * N,
+                  acc ? acc + static_cast<size_t>(t0) * N : nullptr, M - t0 < kMaxM ? M - t0 : kMaxM, N, K};
+    const Workspace ws = carve_workspace(workspace, c.M, N, K);
+    if (w4a8_gemv_supports(c.M, N, K))
+      e = launch_w4a8_gemv(c, ws.status, st);
+    else
+      e = launch_w4a8_gemm_tc(c, ws, st);
+  }
+  if (e == cudaErrorNotSupported) return fail(W4A16_ERR_UNSUPPORTED, "w4a8_gemm: M=%d N=%d K=%d not supported", M, N, K);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a8_gemm launch");
   return ok();
 }
 

@@ -686,3 +686,10 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
 }
 
 }  // namespace w4a16
+
+namespace w4a16 {
+cudaError_t launch_w4a8_gemm_tc(const W4A8Problem& p, const Workspace& ws, cudaStream_t st) {
+  (void)p, (void)ws, (void)st;
+  return cudaErrorNotSupported;
+}
+}  // namespace w4a16

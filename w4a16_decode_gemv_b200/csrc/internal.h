@@ -111,6 +111,26 @@ cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspac
 cudaError_t launch_gptq_sweep(const __half* W, const double* G, int N, int K, int bits, int mode, uint32_t* qweight,
                               __half* scales, __half* zeros, void* workspace, cudaStream_t st);
 
+// W4A8 (w4a8_quant.cu, w4a8_gemv.cu, gemm_tc.cu): the weight and activation
+// quantizers, and the product on CUDA cores (M <= 4) or tensor cores (int8 MMA).
+struct W4A8Problem {
+  const int8_t* x8;
+  const __half* sx;
+  const uint32_t* qweight;
+  const __half* s1;
+  const uint8_t* s2;
+  const uint8_t* zs;
+  __half* y;
+  int32_t* acc;  // optional exact accumulators [M][N]
+  int M, N, K;
+};
+cudaError_t launch_w4a8_quantize_weight(const __half* W, int N, int K, uint32_t* qweight, __half* s1, uint8_t* s2,
+                                        uint8_t* zs, cudaStream_t st);
+cudaError_t launch_w4a8_quantize_act(const __half* x, int M, int K, int8_t* x8, __half* sx, cudaStream_t st);
+bool w4a8_gemv_supports(int M, int N, int K);
+cudaError_t launch_w4a8_gemv(const W4A8Problem& p, uint32_t* status, cudaStream_t st);
+cudaError_t launch_w4a8_gemm_tc(const W4A8Problem& p, const Workspace& ws, cudaStream_t st);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if absent).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
