@@ -248,17 +248,20 @@ def search_workload(Wd, Xd, dev, n_alpha=20, reps=3):
 
 
 def gptq_workload(Wd, Xd, dev, reps=3):
-    """GPTQ's GPU steps on the 11008 x 4096 layer and its 512 calibration tokens: the
-    damped Hessian (gptq_hessian) and the column sweep (gptq_sweep).  The factor G is
-    the caller's step for now; here torch.linalg computes it, outside the timed calls."""
+    """GPTQ on the 11008 x 4096 layer and its 512 calibration tokens, through the product
+    entry point gptq_quantize (Hessian, factor and sweep on one stream), with each of its
+    three steps also timed alone (gptq_hessian, gptq_factor, gptq_sweep)."""
     import torch
 
     import w4a16_decode_gemv_b200 as w4
     N, K = Wd.shape
     T = Xd.shape[0]
+    lib = w4.load_library()
     H = w4.gptq_hessian(Xd)
-    G = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H)), upper=True).contiguous()
-    ws = torch.empty(int(w4.load_library().gptq_sweep_workspace_size(N, K, 128)), dtype=torch.uint8, device=dev)
+    fws = torch.empty(int(lib.gptq_factor_workspace_size(K)), dtype=torch.uint8, device=dev)
+    G = w4.gptq_factor(H, workspace=fws)
+    sws = torch.empty(int(lib.gptq_sweep_workspace_size(N, K, 128)), dtype=torch.uint8, device=dev)
+    qws = torch.empty(int(lib.gptq_quantize_workspace_size(N, K, 128)), dtype=torch.uint8, device=dev)
     out = (torch.empty((N, K // 8), dtype=torch.int32, device=dev),
            torch.empty((N, K // 128), dtype=torch.float16, device=dev),
            torch.empty((N, K // 128), dtype=torch.float16, device=dev))
@@ -277,13 +280,63 @@ def gptq_workload(Wd, Xd, dev, reps=3):
             best = ms if best is None else min(best, ms)
         return best
 
+    q_ms = timed(lambda: w4.gptq_quantize(Wd, Xd, workspace=qws, out=out))
     h_ms = timed(lambda: w4.gptq_hessian(Xd, out=H))
-    s_ms = timed(lambda: w4.gptq_sweep(Wd, G, workspace=ws, out=out))
+    f_ms = timed(lambda: w4.gptq_factor(H, workspace=fws, out=G))
+    s_ms = timed(lambda: w4.gptq_sweep(Wd, G, workspace=sws, out=out))
     sweep_flop = N * K * K  # the updates right of each block: N K^2 / 2 multiply-add pairs
-    return {"N": N, "K": K, "T": T, "hessian_ms": round(h_ms, 4), "sweep_ms": round(s_ms, 3),
+    return {"N": N, "K": K, "T": T, "gptq_quantize_ms": round(q_ms, 3), "hessian_ms": round(h_ms, 4),
+            "factor_ms": round(f_ms, 3), "sweep_ms": round(s_ms, 3),
             "sweep_fp64_tflops": round(sweep_flop / (s_ms * 1e-3) / 1e12, 2),
             "hessian_fp64_tflops": round(2 * T * K * K / (h_ms * 1e-3) / 1e12, 2),
-            "timing": f"CUDA events, best of {reps}; the factor G from torch.linalg, not timed"}
+            "timing": f"CUDA events, best of {reps}; gptq_quantize is the product call, the steps are timed alone"}
+
+
+def w4a8_workload(dev, Ms=(1, 4, 16, 64, 128)):
+    """W4A8 (progressive group quantization) at K = N = 8192: w4a8_gemm per layer in a CUDA
+    graph over distinct weight copies larger than L2, random codes / s2 / zs (the time does
+    not depend on the values); HBM fraction of the algorithmic bytes (codes + s2 + zs + s1)
+    and int8 tensor fraction against the nominal int8 rate (2 x the measured bf16 peak)."""
+    import torch
+
+    import w4a16_decode_gemv_b200 as w4
+    N = K = 8192
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    wbytes = N * K // 2 + 2 * N * (K // 128) + 2 * N
+    copies = max(2, -(-4 * 126 * 2 ** 20 // wbytes))
+    layers = []
+    for _ in range(copies):
+        q = torch.randint(-2 ** 31, 2 ** 31 - 1, (N, K // 8), dtype=torch.int32, device=dev, generator=gen)
+        s2 = torch.randint(1, 17, (N, K // 128), dtype=torch.uint8, device=dev, generator=gen)
+        zs = (torch.randint(0, 16, (N, K // 128), dtype=torch.uint8, device=dev, generator=gen) * s2).to(torch.uint8)
+        s1 = (torch.rand((N,), device=dev, generator=gen) * 1e-3).half()
+        layers.append((q, s1, s2, zs))
+    hbm_peak, _ = measured_peaks()
+    tc_peak, _ = measured_tensor_peak()
+    out = []
+    for M in Ms:
+        x8 = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen)
+        sx = (torch.rand((M,), device=dev, generator=gen) * 1e-2).half()
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ws = torch.zeros(w4.w4a8_gemm_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+
+        def fn():
+            for q, s1, s2, zs in layers:
+                w4.w4a8_gemm(x8, sx, q, s1, s2, zs, out=y, workspace=ws)
+        try:
+            us = time_graph(fn, reps=max(3, 200 // copies)) * 1e3 / copies
+            w4.gemm_check(ws)
+            e = {"M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(wbytes / us / 1e3, 1),
+                 "hbm_frac": round(wbytes / us / 1e3 / hbm_peak, 4),
+                 "path": "CUDA cores (dp4a)" if M <= 4 else "tcgen05 kind::i8 tensor cores"}
+            if M > 4:
+                e["int8_tops"] = round(2 * M * N * K / us / 1e6, 2)
+                e["int8_tensor_frac_of_2x_bf16_peak"] = round(2 * M * N * K / us / 1e6 / (2 * tc_peak), 4)
+            out.append(e)
+        except Exception as ex:  # report, never hide
+            out.append({"M": M, "error": str(ex)[:200]})
+    return {"algorithmic_bytes": wbytes, "entries": out}
 
 
 def run_ours(args, dist):
@@ -562,6 +615,8 @@ def other_workloads(args, dev):
             except Exception as e:  # report, never hide
                 entries.append({"M": M, "N": N, "K": K, "error": str(e)[:200]})
         res[name] = entries
+    if only is None or "w4a8_8192" in only:
+        res["w4a8_8192"] = w4a8_workload(dev)
     if only is not None and not only & {"quantize_pack_11008x4096", "awq_search_11008x4096", "gptq_11008x4096"}:
         return res
     W, X, _ = inputs.quant_workload()
@@ -684,7 +739,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run some of the other workloads only, comma-separated (gemv_4096x4096, llama7b_decode, llama65b_decode, "
-                         "skinny_8192 or skinny_8192:M, prefill_8192 or prefill_8192:M, quantize_pack_11008x4096, "
+                         "skinny_8192 or skinny_8192:M, prefill_8192 or prefill_8192:M, w4a8_8192, quantize_pack_11008x4096, "
                          "awq_search_11008x4096, gptq_11008x4096); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:

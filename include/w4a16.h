@@ -208,6 +208,17 @@ W4A16_API w4a16_status awq_search_alpha(const void* W, const void* X, int N, int
                                         size_t workspace_bytes, w4a16_stream_t stream);
 
 /*
+ * awq_reference_product -- the target of the search above, y = X W^T, on its own.
+ *   X  fp16 [T][K], W fp16 [N][K], Y fp32 [T][N] (all device, 16-byte aligned).
+ * Each output is the fp32 sum, in k order, of the exact fp16 x fp16 products:
+ * the same kernel and order awq_search_alpha uses, offered so that a caller
+ * can check or reuse the search's target.  Asynchronous on `stream`.
+ *   N, K >= 1;  1 <= T <= 2^20;  N*K, T*K and T*N below 2^31.
+ */
+W4A16_API w4a16_status awq_reference_product(const void* X, const void* W, int T, int N, int K, float* Y,
+                                             w4a16_stream_t stream);
+
+/*
  * gptq_hessian -- the damped Hessian of GPTQ's layer objective.
  *
  *   H = 2 X^T X + lambda I,   lambda = damp * (sum_i (2 X^T X)[i][i]) / K

@@ -109,6 +109,30 @@ def test_gemm_check_validation(lib):
     assert lib.w4a16_gemm_check(None, None) == ERR_ARG
 
 
+def test_reference_product_validation(lib):
+    rp = lib.awq_reference_product
+    assert rp(None, A, 4, 8, 128, A, None) == ERR_ARG
+    assert rp(A, A, 0, 8, 128, A, None) == ERR_ARG
+    assert rp(A, A, (1 << 20) + 1, 8, 128, A, None) == ERR_SHAPE
+    assert rp(MIS, A, 4, 8, 128, A, None) == ERR_ALIGN
+
+
+def test_w4a8_validation(lib):
+    assert lib.w4a8_quantize_weight(None, 8, 128, 128, A, A, A, A, None) == ERR_ARG
+    assert lib.w4a8_quantize_weight(A, 8, 128, 64, A, A, A, A, None) == ERR_UNSUPPORTED
+    assert lib.w4a8_quantize_weight(A, 8, 200, 128, A, A, A, A, None) == ERR_SHAPE
+    assert lib.w4a8_quantize_weight(A, 8, 131072, 128, A, A, A, A, None) == ERR_SHAPE
+    assert lib.w4a8_quantize_act(A, 0, 128, A, A, None) == ERR_ARG
+    assert lib.w4a8_quantize_act(A, 70000, 128, A, A, None) == ERR_SHAPE
+    assert lib.w4a8_gemm_workspace_size(1, 8, 200, 128) == 0
+    assert lib.w4a8_gemm_workspace_size(4, 8, 128, 128) > 0
+    g = lib.w4a8_gemm
+    assert g(A, A, A, A, A, A, 1, 8, 128, 128, A, None, None, 0, None) == ERR_WORKSPACE
+    assert g(A, A, A, A, A, A, 1, 8, 128, 128, None, None, A, 1 << 20, None) == ERR_ARG
+    assert g(A, A, A, A, A, A, 1, 8, 128, 128, A, MIS, A, 1 << 20, None) == ERR_ALIGN
+    assert "w4a8_gemm" in _err(lib)
+
+
 def test_noalloc_timeout_selftest_validation(lib):
     assert lib.w4a16_gemv_noalloc_timeout_selftest(0, None) == ERR_ARG
     assert lib.w4a16_gemv_noalloc_timeout_selftest(1000001, None) == ERR_ARG

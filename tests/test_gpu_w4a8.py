@@ -148,3 +148,33 @@ def test_w4a8_gemv_repeats_bit_for_bit(dev):
     args, yo = _gemm_case(dev, 2, 700, 4096, seed=5)
     for _ in range(3):
         assert np.array_equal(bits(w4.w4a8_gemm(*args).cpu().numpy()), bits(yo))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (5, 300, 1024),      # token tile 16, ragged row tile
+    (16, 513, 1152),     # 9 groups: the last unit of a row holds one group
+    (33, 1000, 11008),   # 86 groups (two past the last unit), token tile 64
+    (64, 2048, 256),     # one unit per row
+    (100, 256, 2048),    # token tile 128
+    (150, 300, 4096),    # token tile 192
+    (200, 384, 4096),    # token tile 256
+    (300, 256, 8192),    # 256 + 44 tokens
+])
+def test_w4a8_tensor_core_exact(dev, M, N, K):
+    _gemm_case(dev, M, N, K, seed=M * 104729 + N)
+
+
+def test_w4a8_tensor_core_workload_rows(dev):
+    """K = N = 8192 at M = 16 and 64 (the bench's launches): sampled rows exact."""
+    (layer,) = inputs.layer_set(inputs.SKINNY)
+    qg, s1g, s2g, zsg = w4.w4a8_quantize_weight(to_dev(layer.W, dev))
+    rows = np.unique(np.concatenate([np.random.default_rng(64).choice(layer.N, 252, replace=False),
+                                     [0, 127, 128, layer.N - 1]]))
+    qo, s1o, s2o, zso = oracle.w4a8_quantize_weight(layer.W[rows])
+    for M in (16, 64):
+        x8, sx = w4.w4a8_quantize_act(to_dev(layer.x[:M], dev))
+        y, acc = w4.w4a8_gemm(x8, sx, qg, s1g, s2g, zsg, acc=True)
+        x8o, sxo = oracle.w4a8_quantize_act(layer.x[:M])
+        yo, acco = oracle.w4a8_gemm(x8o, sxo, qo, s1o, s2o, zso)
+        assert np.array_equal(acc.cpu().numpy()[:, rows].astype(np.int64), acco)
+        assert np.array_equal(bits(y.cpu().numpy()[:, rows]), bits(yo))

@@ -75,6 +75,8 @@ def load_library():
     lib.gptq_quantize_workspace_size.restype = sz
     lib.gptq_quantize.argtypes = [vp, vp, i, i, i, d, i, i, i, vp, vp, vp, vp, sz, vp]
     lib.gptq_quantize.restype = i
+    lib.awq_reference_product.argtypes = [vp, vp, i, i, i, vp, vp]
+    lib.awq_reference_product.restype = i
     lib.w4a8_quantize_weight.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp]
     lib.w4a8_quantize_weight.restype = i
     lib.w4a8_quantize_act.argtypes = [vp, i, i, vp, vp, vp]
@@ -343,6 +345,19 @@ def w4a8_gemm(x8: torch.Tensor, sx: torch.Tensor, qweight: torch.Tensor, s1: tor
                              _ptr(y), _ptr(acc_t) if acc_t is not None else None, _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(dev)), "w4a8_gemm")
     return (y, acc_t) if acc_t is not None else y
+
+
+def awq_reference_product(X: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
+    """Y fp32 [T, N] = X fp16 [T, K] @ W fp16 [N, K]^T, the alpha search's target (fp32 sums in k order)."""
+    lib = load_library()
+    T, K = X.shape
+    N = W.shape[0]
+    _expect(X, torch.float16, (T, K), "X")
+    _expect(W, torch.float16, (N, K), "W")
+    Y = torch.empty((T, N), dtype=torch.float32, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib.awq_reference_product(_ptr(X), _ptr(W), T, N, K, _ptr(Y), _stream(X.device)), "awq_reference_product")
+    return Y
 
 
 def search_workspace_size(N: int, K: int, T: int, n_alpha: int, group: int = GROUP) -> int:

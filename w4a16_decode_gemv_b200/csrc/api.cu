@@ -340,6 +340,22 @@ w4a16_status awq_search_alpha(const void* W, const void* X, int N, int K, int T,
   return ok();
 }
 
+w4a16_status awq_reference_product(const void* X, const void* W, int T, int N, int K, float* Y,
+                                   w4a16_stream_t stream) {
+  if (!X || !W || !Y) return fail(W4A16_ERR_ARG, "awq_reference_product: null pointer");
+  if (N < 1 || K < 1 || T < 1) return fail(W4A16_ERR_ARG, "awq_reference_product: N=%d K=%d T=%d must be >= 1", N, K, T);
+  if (T > kMaxSearchTokens) return fail(W4A16_ERR_SHAPE, "awq_reference_product: T=%d (at most %d)", T, kMaxSearchTokens);
+  if (static_cast<long long>(N) * K >= kMaxElems || static_cast<long long>(T) * K >= kMaxElems ||
+      static_cast<long long>(T) * N >= kMaxElems)
+    return fail(W4A16_ERR_SHAPE, "awq_reference_product: N*K, T*K or T*N too large");
+  if (!aligned16(X) || !aligned16(W) || !aligned16(Y))
+    return fail(W4A16_ERR_ALIGN, "awq_reference_product: pointers must be 16-byte aligned");
+  const cudaError_t e = launch_reference_gemm(static_cast<const __half*>(X), static_cast<const __half*>(W), T, N, K, Y,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "awq_reference_product launch");
+  return ok();
+}
+
 w4a16_status gptq_hessian(const void* X, int T, int K, double damp, double* H, w4a16_stream_t stream) {
   if (!X || !H) return fail(W4A16_ERR_ARG, "gptq_hessian: null pointer");
   if (T < 1 || K < 1) return fail(W4A16_ERR_ARG, "gptq_hessian: T=%d K=%d must be >= 1", T, K);

@@ -58,28 +58,33 @@ namespace w4a16 {
 namespace {
 
 constexpr int kRows = 128;                 // weight rows per tile
-constexpr int kCodeStage = kRows * 128;    // 16 KiB: one pair of groups of a tile
+constexpr int kCodeStage = kRows * 256;    // 32 KiB: the codes of one unit (4 groups of a tile)
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kMaxCodeStages = 12;
-constexpr int kMaxXStages = 8;
+constexpr int kMaxCodeStages = 8;
+constexpr int kMaxXStages = 4;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kCodeWarp = 0, kMmaWarp = 1, kXWarp = 2;
+constexpr int kCodeWarp = 0, kMmaWarp = 1, kXWarp = 2, kXWarp2 = 3;
 constexpr int kDqWarp0 = 4, kDqWarps = 8;
 constexpr int kEpiWarp0 = 12, kEpiWarps = 4;
 constexpr int kCtrlBytes = 1024;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
-  const __half* scales;
+  const __half* scales;   // W4A16: Delta and z, fp16 [N][G]
   const __half* zeros;
+  const uint8_t* s2;      // W4A8: level-2 step and scaled zero, bytes [N][G]
+  const uint8_t* zs;
+  const __half* xs;       // W4A8: token scales [M] and channel scales [N]
+  const __half* s1;
+  int32_t* acc;           // W4A8: optional exact accumulators [M][N]
   __half* y;
-  float4* part;       // [grid][MP / 4][128] partial tiles
-  uint32_t* flags;    // [grid] partial tile published (left zero after each call)
+  float4* part;           // [grid][MP / 4][128] partial tiles (fp32, or int32 bit patterns)
+  uint32_t* flags;        // [grid] partial tile published (left zero after each call)
   uint32_t* status;
-  int M, N, G, P;     // tokens, rows, groups per row, group pairs per row
-  int total;          // units = tiles x P
-  int sc, sx;         // code and x ring depths
+  int M, N, G, Q;         // tokens, rows, groups per row, units (4 groups) per row
+  int total;              // units = tiles x Q
+  int sc, sx;             // code and x ring depths
 };
 
 // ---- tcgen05 / TMEM wrappers ---------------------------------------------------
@@ -230,13 +235,74 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return p;
 }
 
-// Accumulator buffers: two (double-buffered across segments) up to MP = 128, one
-// above.  The w_hat slots (one per unit: two groups of 64 columns) take the
-// columns from kACol0 up.
-__host__ __device__ constexpr int n_acc(int mp) { return mp <= 128 ? 2 : 1; }
-__host__ __device__ constexpr int n_aslots(int mp) {
-  return (512 - n_acc(mp) * mp) / 128 > 3 ? 3 : (512 - n_acc(mp) * mp) / 128;
+// ---- the two arithmetics ------------------------------------------------------
+// W4A16: A = w_hat fp16 (one 32-bit column per two inputs: 64 columns per
+// group), B = x fp16 (a 128-byte chunk of a token row holds 64 inputs: two
+// chunks per group), kind::f16 MMAs of K = 16, fp32 accumulators.
+// W4A8 ("MIT 6.5940 Fall 2024 Lecture 13" reading guide, §QServe): A = w8_hat =
+// u * s2 - zs int8 (one column per four inputs: 32 per group), B = x8 int8 (one
+// chunk per group), kind::i8 MMAs of K = 32, exact int32 accumulators.
+// Either way an MMA reads 32 bytes of each A and B row (8 columns of A, one
+// 32-byte step of the B descriptor), and a group is four MMAs per chunk.
+template <bool I8>
+struct Arith {
+  static constexpr int kACols = I8 ? 32 : 64;          // tensor-memory columns of A per group
+  static constexpr int kChunks = I8 ? 1 : 2;           // 128-byte x chunks per group
+  static constexpr int kMmas = 4 * kChunks;            // MMAs per group
+};
+
+// kind::i8 instruction descriptor: s32 D, signed 8-bit A and B, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
 }
+
+__device__ __forceinline__ void mma_i8_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      : "memory");
+}
+
+__device__ __forceinline__ uint16_t ld_nc_b8(const uint8_t* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// Bytewise a - b modulo 256 in each of the four bytes (no borrow between bytes):
+// (a | 0x80) - (b & 0x7F) cannot borrow, and the top bit is then fixed up.
+__device__ __forceinline__ uint32_t sub_bytes(uint32_t a, uint32_t b_low7, uint32_t b_top_not) {
+  return ((a | 0x80808080u) - b_low7) ^ ((a & 0x80808080u) ^ b_top_not);
+}
+
+// W4A8 level-2 dequantization of one code word (inputs 8j .. 8j + 7): two
+// columns of four int8 values each, inputs in order.  Layout v1 puts element i
+// in nibble slot [0,4,1,5,2,6,3,7][i]: w & 0x0F0F0F0F holds elements 0,4,1,5
+// in its bytes and (w >> 4) & 0x0F0F0F0F elements 2,6,3,7.  One multiply per
+// four codes applies s2 (u * s2 <= 240 fits a byte, so no carries) before the
+// zero point is subtracted byte by byte (the progressive order).
+__device__ __forceinline__ void dq8_word(uint32_t w, uint32_t s2, uint32_t zlo7, uint32_t ztop, uint32_t& c0,
+                                         uint32_t& c1) {
+  const uint32_t lo = sub_bytes((w & 0x0F0F0F0Fu) * s2, zlo7, ztop);
+  const uint32_t hi = sub_bytes(((w >> 4) & 0x0F0F0F0Fu) * s2, zlo7, ztop);
+  c0 = __byte_perm(lo, hi, 0x6420);  // elements 0, 1, 2, 3
+  c1 = __byte_perm(lo, hi, 0x7531);  // elements 4, 5, 6, 7
+}
+
+// Accumulator buffers: two (double-buffered across segments) up to MP = 128, one
+// above.  The w_hat slots (one group each) take the columns from kACol0 up.
+__host__ __device__ constexpr int n_acc(int mp) { return mp <= 128 ? 2 : 1; }
+template <bool I8>
+__host__ __device__ constexpr int n_aslots(int mp) {
+  return (512 - n_acc(mp) * mp) / Arith<I8>::kACols > 8 ? 8 : (512 - n_acc(mp) * mp) / Arith<I8>::kACols;
+}
+// Groups of x per x stage: the x of a whole unit up to MP = 32, half of it up
+// to 128, one group above.
+__host__ __device__ constexpr int x_groups(int mp) { return mp <= 32 ? 4 : (mp <= 128 ? 2 : 1); }
 
 // Unit u of the range partition: the CTA whose range holds it.
 __host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
@@ -244,31 +310,33 @@ __host__ __device__ __forceinline__ int owner_cta(int u, int base, int rem) {
   return u < big ? u / (base + 1) : rem + (u - big) / base;
 }
 
-template <int MP>
+template <int MP, bool I8>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tx) {
-  constexpr int kXBox = MP * 128;          // one 64-input box of x
-  constexpr int kXStage = 2 * kXBox;       // one group of x
-  constexpr uint32_t kIdesc = idesc_f16(MP);
+  using AR = Arith<I8>;
+  constexpr int kXG = x_groups(MP);                           // groups per x stage
+  constexpr int kXChunk = MP * 128;                           // one 128-byte chunk of every token
+  constexpr int kXStage = kXG * AR::kChunks * kXChunk;
+  constexpr uint32_t kIdesc = I8 ? idesc_i8(MP) : idesc_f16(MP);
   constexpr int kAcc = n_acc(MP);
-  constexpr int kASlots = n_aslots(MP);
-  constexpr uint32_t kACol0 = kTmemCols - 128u * kASlots;
+  constexpr int kASlots = n_aslots<I8>(MP);
+  constexpr uint32_t kACol0 = kTmemCols - static_cast<uint32_t>(AR::kACols * kASlots);
   static_assert(kAcc * MP <= static_cast<int>(kACol0), "accumulators and w_hat slots exceed tensor memory");
-  static_assert(kASlots >= 2, "w_hat needs at least two slots");
+  static_assert(kASlots >= 4, "w_hat needs a unit's worth of slots");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int Sc = a.sc, Sx = a.sx;
-  uint8_t* cstage = smem;                                  // Sc x 16 KiB of codes
+  uint8_t* cstage = smem;                                  // Sc x 32 KiB of codes
   uint8_t* xstage = cstage + Sc * kCodeStage;              // Sx x kXStage of x
   uint64_t* bars = reinterpret_cast<uint64_t*>(xstage + Sx * kXStage);
   uint64_t* cfull = bars;                                  // [Sc] codes landed
   uint64_t* cempty = cfull + kMaxCodeStages;               // [Sc] codes read
   uint64_t* xfull = cempty + kMaxCodeStages;               // [Sx] x landed
   uint64_t* xempty = xfull + kMaxXStages;                  // [Sx] x consumed by the MMAs
-  uint64_t* afull = xempty + kMaxXStages;                  // [kASlots] w_hat written
-  uint64_t* aempty = afull + 3;                            // [kASlots] w_hat consumed
-  uint64_t* accfull = aempty + 3;                          // [kAcc] segment's MMAs complete
+  uint64_t* afull = xempty + kMaxXStages;                  // [kASlots] w_hat of a group written
+  uint64_t* aempty = afull + 8;                            // [kASlots] w_hat of a group consumed
+  uint64_t* accfull = aempty + 8;                          // [kAcc] segment's MMAs complete
   uint64_t* accempty = accfull + 2;                        // [kAcc] accumulator read out
   uint64_t* tdown = accempty + 2;                          // teardown: all MMAs complete
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tdown + 1);
@@ -279,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int base = a.total / grid, rem = a.total - base * grid;
   const int u0 = bx * base + min(bx, rem);
   const int cnt = base + (bx < rem ? 1 : 0);
-  const int P = a.P;
+  const int Q = a.Q;
+  const int xper = 4 / kXG;  // x stages per unit
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Sc; ++s) {
@@ -291,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&xempty[s], 1);
     }
     for (int b = 0; b < kASlots; ++b) {
-      mbar_init(&afull[b], kDqWarps);
+      mbar_init(&afull[b], 4);  // the four lane-quarter warps of the group
       mbar_init(&aempty[b], 1);
     }
     for (int b = 0; b < kAcc; ++b) {
@@ -312,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
 
   if (warp == kCodeWarp) {
-    // ---------------- codes: one tensor copy per unit ----------------
+    // ---------------- codes: two adjacent 16 KiB boxes per unit ----------------
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
       int issued = 0;
@@ -321,82 +390,99 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % Sc;
         if (i >= Sc && !wait_or_abort(&cempty[s], static_cast<uint32_t>(i / Sc - 1) & 1u, abort_flag, a.status))
           break;
-        const int u = u0 + i, t = u / P, p = u - t * P;
+        const int u = u0 + i, t = u / Q, q4 = u - t * Q;
+        uint8_t* dst = cstage + s * kCodeStage;
         mbar_arrive_expect_tx(&cfull[s], kCodeStage);
-        tma_load_2d(cstage + s * kCodeStage, &tq, p * 32, t * kRows, &cfull[s], pol);
+        tma_load_2d(dst, &tq, q4 * 64, t * kRows, &cfull[s], pol);
+        tma_load_2d(dst + kCodeStage / 2, &tq, q4 * 64 + 32, t * kRows, &cfull[s], pol);
         issued = i + 1;
       }
-      for (int j = max(0, issued - Sc); j < issued; ++j)
-        mbar_wait_bounded(&cfull[j % Sc], static_cast<uint32_t>(j / Sc) & 1u);
+      // After an abort the copies in flight must land before the CTA may exit
+      // (otherwise every stage was consumed): the last Sc issues, one per stage.
+      if (*abort_flag)
+        for (int j = max(0, issued - Sc); j < issued; ++j)
+          mbar_wait_bounded(&cfull[j % Sc], static_cast<uint32_t>(j / Sc) & 1u);
     }
-  } else if (warp == kXWarp) {
-    // ---------------- x: one stage per group ----------------
+  } else if (warp == kXWarp || warp == kXWarp2) {
+    // ---------------- x: one 3-D box per stage; the two x warps alternate stages ----------------
     if (lane == 0) {
       const uint64_t pol = l2_evict_last_policy();
       griddep_wait();  // x may be the previous kernel's output
-      int j = 0;
-      bool ok = true;
-      for (int i = 0; i < cnt && ok; ++i) {
-        const int u = u0 + i, p = u % P;
-        for (int h = 0; h < 2; ++h) {
-          const int g = 2 * p + h;
-          if (g >= a.G) break;
-          const int s = j % Sx;
-          if (j >= Sx && !wait_or_abort(&xempty[s], static_cast<uint32_t>(j / Sx - 1) & 1u, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* dst = xstage + s * kXStage;
-          mbar_arrive_expect_tx(&xfull[s], kXStage);
-          tma_load_2d(dst, &tx, g * 128, 0, &xfull[s], pol);
-          tma_load_2d(dst + kXBox, &tx, g * 128 + 64, 0, &xfull[s], pol);
-          ++j;
-        }
+      const int total_x = cnt * xper;
+      int latest[kMaxXStages];  // this warp's latest issue into each stage
+#pragma unroll
+      for (int s = 0; s < kMaxXStages; ++s) latest[s] = -1;
+      for (int j = (warp == kXWarp ? 0 : 1); j < total_x; j += 2) {
+        const int s = j % Sx;
+        if (j >= Sx && !wait_or_abort(&xempty[s], static_cast<uint32_t>(j / Sx - 1) & 1u, abort_flag, a.status))
+          break;
+        const int i = j / xper, u = u0 + i, q4 = u % Q;
+        const int g0 = 4 * q4 + (j - i * xper) * kXG;  // first group of the stage
+        mbar_arrive_expect_tx(&xfull[s], kXStage);
+        tma_load_3d(xstage + s * kXStage, &tx, 0, 0, g0 * AR::kChunks, &xfull[s], pol);
+        latest[s] = j;
       }
-      for (int jj = max(0, j - Sx); jj < j; ++jj)
-        mbar_wait_bounded(&xfull[jj % Sx], static_cast<uint32_t>(jj / Sx) & 1u);
+      // after an abort, this warp's copies in flight land before the CTA may exit
+      if (*abort_flag)
+        for (int s = 0; s < Sx; ++s)
+          if (latest[s] >= 0) mbar_wait_bounded(&xfull[s], static_cast<uint32_t>(latest[s] / Sx) & 1u);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       bool any = false, ok = true;
-      int j = 0, seg = 0;
+      int seg = 0;
       for (int i = 0; i < cnt && ok; ++i) {
-        const int u = u0 + i, p = u % P;
-        const bool first = (i == 0) || (p == 0);
-        const bool last = (i == cnt - 1) || (p == P - 1);
+        const int u = u0 + i, q4 = u % Q;
+        const bool first = (i == 0) || (q4 == 0);
+        const bool last = (i == cnt - 1) || (q4 == Q - 1);
         const int ab = seg % kAcc;
         if (first && seg >= kAcc &&
             !wait_or_abort(&accempty[ab], static_cast<uint32_t>(seg / kAcc - 1) & 1u, abort_flag, a.status))
           break;
-        const int b = i % kASlots;
-        if (!wait_or_abort(&afull[b], static_cast<uint32_t>(i / kASlots) & 1u, abort_flag, a.status)) break;
-        tc_fence_after();
         const uint32_t d = tbase + static_cast<uint32_t>(ab * MP);
-        for (int h = 0; h < 2; ++h) {
-          const int g = 2 * p + h;
-          if (g >= a.G) break;
+        for (int gg = 0; gg < 4; ++gg) {
+          const int j = i * xper + gg / kXG;  // x stage of this group
           const int s = j % Sx;
-          if (!wait_or_abort(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u, abort_flag, a.status)) {
+          if (gg % kXG == 0 &&
+              !wait_or_abort(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u, abort_flag, a.status)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * 128 + h * 64);
-          const uint64_t bd0 = sw128_desc(xstage + s * kXStage);
-          const uint64_t bd1 = sw128_desc(xstage + s * kXStage + kXBox);
+          // every group position of a unit takes its w_hat slot, a position past the
+          // last group (K / 128 not a multiple of 4) with no MMAs, so that each slot's
+          // uses follow one another in order
+          {
+            const int ga = 4 * i + gg, b = ga % kASlots;
+            if (!wait_or_abort(&afull[b], static_cast<uint32_t>(ga / kASlots) & 1u, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (4 * q4 + gg < a.G) {
+              const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * AR::kACols);
+              const uint8_t* xg = xstage + s * kXStage + (gg % kXG) * AR::kChunks * kXChunk;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // the descriptor's start address advances 32 bytes (2 x 16) per 16 inputs
-            const uint64_t bd = (kk < 4 ? bd0 : bd1) + 2u * static_cast<uint32_t>(kk & 3);
-            mma_f16_ts(d, acol + 8u * kk, bd, kIdesc, !(first && h == 0 && kk == 0));
+              for (int c = 0; c < AR::kChunks; ++c) {
+                const uint64_t bd = sw128_desc(xg + c * kXChunk);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  // the descriptor's start address advances 32 bytes (2 x 16) per MMA
+                  const uint32_t at = acol + 8u * (4 * c + kk);
+                  const bool accum = !(first && gg == 0 && c == 0 && kk == 0);
+                  if constexpr (I8)
+                    mma_i8_ts(d, at, bd + 2u * kk, kIdesc, accum);
+                  else
+                    mma_f16_ts(d, at, bd + 2u * kk, kIdesc, accum);
+                }
+              }
+              any = true;
+            }
+            mma_commit(&aempty[b]);
           }
-          any = true;
-          mma_commit(&xempty[s]);
-          ++j;
+          if (gg % kXG == kXG - 1) mma_commit(&xempty[s]);
         }
         if (!ok) break;
-        mma_commit(&aempty[b]);
         if (last) {
           mma_commit(&accfull[ab]);
           ++seg;
@@ -409,80 +495,120 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
     // ---------------- dequantization into tensor memory ----------------
+    // warp (q, h): rows 32 q .. 32 q + 31 of the tile, groups h and h + 2 of each unit
     const int q = warp & 3, h = (warp - kDqWarp0) >> 2;
     const int r = q * 32 + lane;  // row within the tile
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + static_cast<uint32_t>(h * 64);
-    const uint32_t row_smem = smem_u32(cstage) + static_cast<uint32_t>(r * 128);
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
-    // Delta and z of the next units, fetched a few units ahead
-    constexpr int kLook = 3;
+    // per-group parameters of the next items (unit, group), fetched a few items ahead
+    constexpr int kLook = 4;
     uint16_t pd[kLook], pz[kLook];
-    auto fetch = [&](int i, uint16_t& dv, uint16_t& zv) {
+    auto fetch = [&](int it, uint16_t& dv, uint16_t& zv) {
       dv = zv = 0;
+      const int i = it >> 1;
       if (i < cnt) {
-        const int u = u0 + i, t = u / P, g = 2 * (u - t * P) + h;
+        const int u = u0 + i, t = u / Q, g = 4 * (u - t * Q) + h + 2 * (it & 1);
         const int n = t * kRows + r;
         if (n < a.N && g < a.G) {
           const size_t o = static_cast<size_t>(n) * a.G + g;
-          dv = ld_nc_u16(a.scales + o);
-          zv = ld_nc_u16(a.zeros + o);
+          if constexpr (I8) {
+            dv = ld_nc_b8(a.s2 + o);
+            zv = ld_nc_b8(a.zs + o);
+          } else {
+            dv = ld_nc_u16(a.scales + o);
+            zv = ld_nc_u16(a.zeros + o);
+          }
         }
       }
     };
 #pragma unroll
     for (int l = 0; l < kLook; ++l) fetch(l, pd[l], pz[l]);
-    for (int i = 0; i < cnt; ++i) {
-      const int u = u0 + i, t = u / P, p = u - t * P;
-      const bool valid = 2 * p + h < a.G;
-      const uint16_t dv = pd[0], zv = pz[0];
-#pragma unroll
-      for (int l = 0; l + 1 < kLook; ++l) {
-        pd[l] = pd[l + 1];
-        pz[l] = pz[l + 1];
-      }
-      fetch(i + kLook, pd[kLook - 1], pz[kLook - 1]);
+    bool ok = true;
+    for (int i = 0; i < cnt && ok; ++i) {
+      const int u = u0 + i, t = u / Q, q4 = u - t * Q;
       const int s = i % Sc;
       const bool okc = wait_or_abort(&cfull[s], static_cast<uint32_t>(i / Sc) & 1u, abort_flag, a.status);
       if (__any_sync(0xffffffffu, !okc)) break;
-      uint4 cw[4];
-      if (valid) {
-        const uint32_t row = row_smem + static_cast<uint32_t>(s * kCodeStage);
+      // this lane's 64 code bytes of groups h and h + 2 (box h... the pair box gg / 2, half gg % 2)
+      uint4 cw[2][4];
+      bool valid[2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) cw[c] = lds128(row + (((static_cast<uint32_t>(4 * h + c)) ^ rsw) << 4));
+      for (int e = 0; e < 2; ++e) {
+        const int gg = h + 2 * e;
+        valid[e] = 4 * q4 + gg < a.G;
+        if (valid[e]) {
+          const uint32_t row = smem_u32(cstage) + static_cast<uint32_t>(s * kCodeStage + (gg >> 1) * (kCodeStage / 2) + r * 128);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            cw[e][c] = lds128(row + (((static_cast<uint32_t>(4 * (gg & 1) + c)) ^ rsw) << 4));
+        }
       }
       // every lane's reads are ordered before the copy that refills the stage
       release_stage_reads();
       __syncwarp();
       if (lane == 0) mbar_arrive(&cempty[s]);
-      const int b = i % kASlots;
-      const bool oka = i < kASlots ||
-                       wait_or_abort(&aempty[b], static_cast<uint32_t>(i / kASlots - 1) & 1u, abort_flag, a.status);
-      if (__any_sync(0xffffffffu, !oka)) break;
-      tc_fence_after();
-      if (valid) {
-        const __half2 dd = as_h2(static_cast<uint32_t>(dv) | (static_cast<uint32_t>(dv) << 16));
-        // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
-        const __half zh = __hneg(__hadd(__ushort_as_half(zv), __float2half_rn(1024.0f)));
-        const __half2 nz = __halves2half2(zh, zh);
-        const uint32_t col = lane_base + static_cast<uint32_t>(b * 128);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wv[4] = {cw[c].x, cw[c].y, cw[c].z, cw[c].w};
-          uint32_t v[16];
+      for (int e = 0; e < 2; ++e) {
+        const int gg = h + 2 * e;
+        const uint16_t dv = pd[0], zv = pz[0];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            v[4 * k + 0] = dq_pair(wv[k], nz, dd);
-            v[4 * k + 1] = dq_pair(wv[k] >> 4, nz, dd);
-            v[4 * k + 2] = dq_pair(wv[k] >> 8, nz, dd);
-            v[4 * k + 3] = dq_pair(wv[k] >> 12, nz, dd);
+        for (int l = 0; l + 1 < kLook; ++l) {
+          pd[l] = pd[l + 1];
+          pz[l] = pz[l + 1];
+        }
+        fetch(2 * i + e + kLook, pd[kLook - 1], pz[kLook - 1]);
+        const int ga = 4 * i + gg, b = ga % kASlots;
+        const bool oka = ga < kASlots ||
+                         wait_or_abort(&aempty[b], static_cast<uint32_t>(ga / kASlots - 1) & 1u, abort_flag, a.status);
+        if (__any_sync(0xffffffffu, !oka)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t col = lane_base + static_cast<uint32_t>(b * AR::kACols);
+        if (!valid[e]) {
+          // a position past the last group: no w_hat, but the slot is passed on in turn
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[b]);
+          continue;
+        }
+        if constexpr (I8) {
+          const uint32_t s2 = dv, zs4 = static_cast<uint32_t>(zv) * 0x01010101u;
+          const uint32_t zlo7 = zs4 & 0x7F7F7F7Fu, ztop = ~zs4 & 0x80808080u;
+#pragma unroll
+          for (int c = 0; c < 4; c += 2) {
+            uint32_t v[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              dq8_word((&cw[e][c].x)[k], s2, zlo7, ztop, v[2 * k], v[2 * k + 1]);
+              dq8_word((&cw[e][c + 1].x)[k], s2, zlo7, ztop, v[8 + 2 * k], v[8 + 2 * k + 1]);
+            }
+            tmem_st16(col + static_cast<uint32_t>(8 * c), v);
           }
-          tmem_st16(col + static_cast<uint32_t>(16 * c), v);
+        } else {
+          const __half2 dd = as_h2(static_cast<uint32_t>(dv) | (static_cast<uint32_t>(dv) << 16));
+          // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
+          const __half zh = __hneg(__hadd(__ushort_as_half(zv), __float2half_rn(1024.0f)));
+          const __half2 nz = __halves2half2(zh, zh);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t wv[4] = {cw[e][c].x, cw[e][c].y, cw[e][c].z, cw[e][c].w};
+            uint32_t v[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              v[4 * k + 0] = dq_pair(wv[k], nz, dd);
+              v[4 * k + 1] = dq_pair(wv[k] >> 4, nz, dd);
+              v[4 * k + 2] = dq_pair(wv[k] >> 8, nz, dd);
+              v[4 * k + 3] = dq_pair(wv[k] >> 12, nz, dd);
+            }
+            tmem_st16(col + static_cast<uint32_t>(16 * c), v);
+          }
         }
         tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[b]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[b]);
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------- epilogue ----------------
@@ -492,11 +618,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_wait();  // y and the workspace slots may still be in use by the previous kernel
     int seg = 0;
     for (int i = 0; i < cnt; ++i) {
-      const int u = u0 + i, t = u / P, p = u - t * P;
-      if (!(i == cnt - 1 || p == P - 1)) continue;  // only at the end of a segment
-      const int ia = (seg == 0) ? 0 : i - p;        // segment start (a later segment starts at p = 0)
-      const bool covers_first = (u0 + ia) == t * P;
-      const bool covers_last = (p == P - 1);
+      const int u = u0 + i, t = u / Q, q4 = u - t * Q;
+      if (!(i == cnt - 1 || q4 == Q - 1)) continue;  // only at the end of a segment
+      const int ia = (seg == 0) ? 0 : i - q4;        // segment start (a later segment starts at q4 = 0)
+      const bool covers_first = (u0 + ia) == t * Q;
+      const bool covers_last = (q4 == Q - 1);
       const int ab = seg % kAcc;
       const bool okw = wait_or_abort(&accfull[ab], static_cast<uint32_t>(seg / kAcc) & 1u, abort_flag, a.status);
       if (__any_sync(0xffffffffu, !okw)) break;
@@ -523,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // alone, or the owner: add the later contributors' partial tiles in CTA order
-        const int c_hi = covers_last ? bx : owner_cta(t * P + P - 1, base, rem);
+        const int c_hi = covers_last ? bx : owner_cta(t * Q + Q - 1, base, rem);
         for (int cc = bx + 1; cc <= c_hi && okw2; ++cc) {
           bool okf = true;
           if (lane == 0) okf = wait_flag(a.flags + cc, kEpiWarps, abort_flag, a.status);
@@ -531,6 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (okw2) (void)ld_acquire(a.flags + cc);  // every lane acquires what the publisher released
         }
         if (okw2) {
+          const double s1n = I8 && n < a.N ? static_cast<double>(__half2float(a.s1[n])) : 0.0;
 #pragma unroll 1
           for (int c = 0; c < MP / 16; ++c) {
             float v[16];
@@ -540,16 +667,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float4 w = __ldcg(slot + (4 * c + e) * kRows + r);
-                v[4 * e] += w.x;
-                v[4 * e + 1] += w.y;
-                v[4 * e + 2] += w.z;
-                v[4 * e + 3] += w.w;
+                if constexpr (I8) {
+                  // the int32 sums travel as their bit patterns; integer addition is exact
+                  v[4 * e] = __int_as_float(__float_as_int(v[4 * e]) + __float_as_int(w.x));
+                  v[4 * e + 1] = __int_as_float(__float_as_int(v[4 * e + 1]) + __float_as_int(w.y));
+                  v[4 * e + 2] = __int_as_float(__float_as_int(v[4 * e + 2]) + __float_as_int(w.z));
+                  v[4 * e + 3] = __int_as_float(__float_as_int(v[4 * e + 3]) + __float_as_int(w.w));
+                } else {
+                  v[4 * e] += w.x;
+                  v[4 * e + 1] += w.y;
+                  v[4 * e + 2] += w.z;
+                  v[4 * e + 3] += w.w;
+                }
               }
             }
             if (n < a.N) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (16 * c + e < a.M) a.y[static_cast<size_t>(16 * c + e) * a.N + n] = __float2half_rn(v[e]);
+              for (int e = 0; e < 16; ++e) {
+                const int m = 16 * c + e;
+                if (m >= a.M) continue;
+                if constexpr (I8) {
+                  const int iv = __float_as_int(v[e]);
+                  const double yv = (static_cast<double>(iv) * static_cast<double>(__half2float(a.xs[m]))) * s1n;
+                  uint16_t hb;
+                  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(hb) : "d"(yv));
+                  a.y[static_cast<size_t>(m) * a.N + n] = __ushort_as_half(hb);
+                  if (a.acc) a.acc[static_cast<size_t>(m) * a.N + n] = iv;
+                } else {
+                  a.y[static_cast<size_t>(m) * a.N + n] = __float2half_rn(v[e]);
+                }
+              }
             }
           }
           // Each owner warp adds 1 once it has read a flag's tile; the last of
@@ -577,23 +724,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Ring depths: x stages for about 64 KiB of x (2 to 8), the rest of shared
-// memory for code stages (at most 12).
-void ring_depths(int mp, int& sc, int& sx) {
-  const int xs = 2 * mp * 128;
+// Ring depths: x stages for about 64 KiB of x (2 to 4), the rest of shared
+// memory for code stages (at most kMaxCodeStages).
+template <int MP, bool I8>
+void ring_depths(int& sc, int& sx) {
+  const int xs = x_groups(MP) * Arith<I8>::kChunks * MP * 128;
   sx = (64 * 1024) / xs;
-  sx = sx < 2 ? 2 : (sx > kMaxXStages ? kMaxXStages : sx);
+  sx = sx < 2 ? 2 : (sx > 4 ? 4 : sx);
   sc = (kMaxSmem - 1024 - kCtrlBytes - sx * xs) / kCodeStage;
   sc = sc > kMaxCodeStages ? kMaxCodeStages : sc;
 }
 
-template <int MP>
+template <int MP, bool I8>
 cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap& tx, int grid, cudaStream_t st) {
   TcArgs a = a0;
-  ring_depths(MP, a.sc, a.sx);
+  ring_depths<MP, I8>(a.sc, a.sx);
   if (a.sc < 2) return cudaErrorNotSupported;
-  const int smem = 1024 + a.sc * kCodeStage + a.sx * 2 * MP * 128 + kCtrlBytes;
-  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_kernel<MP>),
+  const int smem = 1024 + a.sc * kCodeStage + a.sx * x_groups(MP) * Arith<I8>::kChunks * MP * 128 + kCtrlBytes;
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gemm_tc_kernel<MP, I8>),
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
@@ -606,12 +754,10 @@ cudaError_t launch_mp(const TcArgs& a0, const CUtensorMap& tq, const CUtensorMap
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<MP>, a, tq, tx);
+  e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<MP, I8>, a, tq, tx);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
-
-}  // namespace
 
 // The token tile of a launch of M <= kMaxM tokens.
 int tc_tile(int M) {
@@ -623,6 +769,66 @@ int tc_tile(int M) {
   return mp <= 192 ? 192 : 256;
 }
 
+// Tensor maps of a launch: codes u32 [N][K/8] in boxes of 128 rows x 32 words
+// (one pair of groups; a unit takes two), and x as a 3-D view [K / E][M][E]
+// (E = 64 fp16 or 128 int8: one 128-byte chunk) in boxes of E x MP x the
+// chunks of one x stage, all with the 128-byte swizzle.
+bool encode_maps(const uint32_t* qweight, const void* x, bool i8, int M, int N, int K, int mp, CUtensorMap& tq,
+                 CUtensorMap& tx) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 8), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 8) * 4};
+    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qweight), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    const int elem = i8 ? 1 : 2, E = 128 / elem;
+    const int chunks_per_stage = x_groups(mp) * (i8 ? 1 : 2);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(E), static_cast<cuuint64_t>(M),
+                                static_cast<cuuint64_t>(K / E)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * elem, 128};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(E), static_cast<cuuint32_t>(mp),
+                               static_cast<cuuint32_t>(chunks_per_stage)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tx, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(x), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+template <bool I8>
+cudaError_t launch_tc(TcArgs& a, const uint32_t* qweight, const void* x, int K, cudaStream_t st) {
+  const int mp = tc_tile(a.M);
+  CUtensorMap tq, tx;
+  if (!encode_maps(qweight, x, I8, a.M, a.N, K, mp, tq, tx)) return cudaErrorInvalidValue;
+  a.G = K / kGroup;
+  a.Q = (a.G + 3) / 4;
+  const int tiles = (a.N + kRows - 1) / kRows;
+  a.total = tiles * a.Q;
+  a.sc = a.sx = 0;
+  const int grid = min(device_sm_count(), a.total);
+  if (grid > kMaxFlags) return cudaErrorNotSupported;
+  switch (mp) {
+    case 16: return launch_mp<16, I8>(a, tq, tx, grid, st);
+    case 32: return launch_mp<32, I8>(a, tq, tx, grid, st);
+    case 64: return launch_mp<64, I8>(a, tq, tx, grid, st);
+    case 96: return launch_mp<96, I8>(a, tq, tx, grid, st);
+    case 128: return launch_mp<128, I8>(a, tq, tx, grid, st);
+    case 192: return launch_mp<192, I8>(a, tq, tx, grid, st);
+    default: return launch_mp<256, I8>(a, tq, tx, grid, st);
+  }
+}
+
+}  // namespace
+
 size_t tc_partial_bytes(int M) {
   const size_t mp = static_cast<size_t>(tc_tile(M));
   return static_cast<size_t>(device_sm_count()) * kRows * mp * 4;
@@ -630,35 +836,7 @@ size_t tc_partial_bytes(int M) {
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
   if (p.M < 1 || p.M > kMaxM || !ws.part || !ws.flags) return cudaErrorNotSupported;
-  const int mp = tc_tile(p.M);
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
-
-  // codes: u32 [N][K/8], boxes of 128 rows x 32 words (a pair of groups), 128-byte swizzle
-  CUtensorMap tq, tx;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K / 8), static_cast<cuuint64_t>(p.N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 8) * 4};
-    const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kRows)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  // x: fp16 [M][K], boxes of MP rows (rows past M read as zero) x 64 inputs, 128-byte swizzle
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(mp)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(p.x), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-
-  TcArgs a;
+  TcArgs a = {};
   a.scales = p.scales;
   a.zeros = p.zeros;
   a.y = p.y;
@@ -667,29 +845,24 @@ cudaError_t launch_gemm_tc(const GemmProblem& p, const Workspace& ws, cudaStream
   a.status = ws.status;
   a.M = p.M;
   a.N = p.N;
-  a.G = p.K / kGroup;
-  a.P = (a.G + 1) / 2;
-  const int tiles = (p.N + kRows - 1) / kRows;
-  a.total = tiles * a.P;
-  a.sc = a.sx = 0;
-  const int grid = min(device_sm_count(), a.total);
-  if (grid > kMaxFlags) return cudaErrorNotSupported;
-  switch (mp) {
-    case 16: return launch_mp<16>(a, tq, tx, grid, st);
-    case 32: return launch_mp<32>(a, tq, tx, grid, st);
-    case 64: return launch_mp<64>(a, tq, tx, grid, st);
-    case 96: return launch_mp<96>(a, tq, tx, grid, st);
-    case 128: return launch_mp<128>(a, tq, tx, grid, st);
-    case 192: return launch_mp<192>(a, tq, tx, grid, st);
-    default: return launch_mp<256>(a, tq, tx, grid, st);
-  }
+  return launch_tc<false>(a, p.qweight, p.x, p.K, st);
 }
 
-}  // namespace w4a16
-
-namespace w4a16 {
 cudaError_t launch_w4a8_gemm_tc(const W4A8Problem& p, const Workspace& ws, cudaStream_t st) {
-  (void)p, (void)ws, (void)st;
-  return cudaErrorNotSupported;
+  if (p.M < 1 || p.M > kMaxM || !ws.part || !ws.flags) return cudaErrorNotSupported;
+  TcArgs a = {};
+  a.s2 = p.s2;
+  a.zs = p.zs;
+  a.xs = p.sx;
+  a.s1 = p.s1;
+  a.acc = p.acc;
+  a.y = p.y;
+  a.part = reinterpret_cast<float4*>(ws.part);
+  a.flags = ws.flags;
+  a.status = ws.status;
+  a.M = p.M;
+  a.N = p.N;
+  return launch_tc<true>(a, p.qweight, p.x8, p.K, st);
 }
+
 }  // namespace w4a16

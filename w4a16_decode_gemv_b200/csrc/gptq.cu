@@ -239,71 +239,231 @@ __global__ void gptq_reverse_kernel(const double* __restrict__ H, int K, double*
   }
 }
 
-// Column j of L in place, left-looking, one warp per row: first the diagonal
-// (diag = true), L[j][j] = sqrt(A[j][j] - sum_k L[j][k]^2); then the rows below,
-// L[i][j] = (A[i][j] - sum_k L[i][k] L[j][k]) / L[j][j].
-__global__ void gptq_chol_col_kernel(double* __restrict__ L, int K, int j, bool diag) {
-  const int lane = threadIdx.x & 31;
-  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int i = diag ? j : j + 1 + w;
-  if (i >= K || (diag && w > 0)) return;
-  const double* li = L + static_cast<long long>(i) * K;
-  const double* lj = L + static_cast<long long>(j) * K;
-  double s = 0.0;
-  for (int k = lane; k < j; k += 32) s = fma(li[k], lj[k], s);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
-    double* d = L + static_cast<long long>(i) * K + j;
-    if (diag) *d = sqrt(*d - s);
-    else *d = (*d - s) / lj[j];
+// Blocked factorization in 64 x 64 tiles (K is a multiple of 128).  Right-looking
+// Cholesky: for each block column kb, the diagonal tile is factored (and its
+// triangular inverse formed) by one CTA, the panel below becomes
+// L[ib][kb] = A[ib][kb] inv(L[kb][kb])^T, and the trailing lower triangle is
+// updated, A[ib][jb] -= L[ib][kb] L[jb][kb]^T.  Then X = L^-1 by block rows:
+// X[ib][ib] = inv(L[ib][ib]) and, for kb < ib,
+// X[ib][kb] = -inv(L[ib][ib]) sum_{jb = kb}^{ib-1} L[ib][jb] X[jb][kb].
+// Every tile product is a 64 x 64 x 64 fp64 product: 256 threads, 4 x 4
+// outputs each, operands staged in shared memory with k outermost.
+constexpr int kB = 64;
+constexpr int kBP = kB + 2;  // padded row of a staged tile (doubles)
+
+// dst[k][x] = src[x][k] (transpose) or src[k][x]; src row stride ld.
+__device__ __forceinline__ void stage_tile(double (*dst)[kBP], const double* src, long long ld, bool transpose) {
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
+    const int a = e / kB, b = e % kB;  // b runs fastest: coalesced reads of src row a
+    const double v = src[static_cast<long long>(a) * ld + b];
+    if (transpose)
+      dst[b][a] = v;  // src[a][b] = P[x = a][k = b]
+    else
+      dst[a][b] = v;  // src[a][b] = Q[k = a][x = b]
   }
 }
 
-// Column c of X = L^-1 by forward substitution (one warp per column):
-// X[c][c] = 1 / L[c][c], X[i][c] = -(sum_{k=c}^{i-1} L[i][k] X[k][c]) / L[i][i];
-// written reversed into G: G[K-1-i][K-1-c] = X[i][c] (0 for i < c).
-__global__ void gptq_trinv_kernel(const double* __restrict__ L, int K, double* __restrict__ G,
-                                  double* __restrict__ scratch) {
-  const int lane = threadIdx.x & 31;
-  const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (c >= K) return;
-  double* x = scratch + static_cast<long long>(c) * K;
-  if (lane == 0) x[c] = 1.0 / L[static_cast<long long>(c) * K + c];
-  __syncwarp();
-  for (int i = c + 1; i < K; ++i) {
-    const double* li = L + static_cast<long long>(i) * K;
-    double s = 0.0;
-    for (int k = c + lane; k < i; k += 32) s = fma(li[k], x[k], s);
+// acc[i][j] += sum_k Ps[k][4 tr + i] * Qs[k][4 tc + j]
+__device__ __forceinline__ void tile_product(double (&acc)[4][4], const double (*Ps)[kBP], const double (*Qs)[kBP],
+                                             int tr, int tc) {
+#pragma unroll 4
+  for (int k = 0; k < kB; ++k) {
+    double p[4], q[4];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) x[i] = -s / li[i];
-    __syncwarp();
+    for (int i = 0; i < 4; ++i) {
+      p[i] = Ps[k][4 * tr + i];
+      q[i] = Qs[k][4 * tc + i];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fma(p[i], q[j], acc[i][j]);
   }
-  for (int i = c + lane; i < K; i += 32) G[static_cast<long long>(K - 1 - i) * K + (K - 1 - c)] = x[i];
-  for (int i = lane; i < c; i += 32) G[static_cast<long long>(K - 1 - i) * K + (K - 1 - c)] = 0.0;
+}
+
+// Diagonal tile kb: L[kb][kb] (lower) in place and Dinv[kb] = its inverse.
+__global__ void __launch_bounds__(256) gptq_chol_diag_kernel(double* __restrict__ L, int K, int kb,
+                                                             double* __restrict__ Dinv) {
+  extern __shared__ double sm[];
+  double(*a)[kB + 1] = reinterpret_cast<double(*)[kB + 1]>(sm);
+  double(*x)[kB + 1] = reinterpret_cast<double(*)[kB + 1]>(sm + kB * (kB + 1));
+  double* tile = L + static_cast<long long>(kb) * kB * K + static_cast<long long>(kb) * kB;
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) a[e / kB][e % kB] = tile[static_cast<long long>(e / kB) * K + e % kB];
+  __syncthreads();
+  for (int j = 0; j < kB; ++j) {
+    if (threadIdx.x == 0) a[j][j] = sqrt(a[j][j]);
+    __syncthreads();
+    for (int i = j + 1 + threadIdx.x; i < kB; i += blockDim.x) a[i][j] /= a[j][j];
+    __syncthreads();
+    // trailing update of the lower triangle: a[i][c] -= a[i][j] a[c][j], j < c <= i
+    for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
+      const int i = e / kB, c = e % kB;
+      if (c > j && c <= i) a[i][c] = fma(-a[i][j], a[c][j], a[i][c]);
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
+    const int i = e / kB, c = e % kB;
+    tile[static_cast<long long>(i) * K + c] = c <= i ? a[i][c] : 0.0;
+  }
+  // inverse by forward substitution, one column per thread
+  if (threadIdx.x < kB) {
+    const int c = threadIdx.x;
+    for (int i = 0; i < c; ++i) x[i][c] = 0.0;
+    x[c][c] = 1.0 / a[c][c];
+    for (int i = c + 1; i < kB; ++i) {
+      double sum = 0.0;
+      for (int k = c; k < i; ++k) sum = fma(a[i][k], x[k][c], sum);
+      x[i][c] = -sum / a[i][i];
+    }
+  }
+  __syncthreads();
+  double* dinv = Dinv + static_cast<long long>(kb) * kB * kB;
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) dinv[e] = x[e / kB][e % kB];
+}
+
+// Panel of block column kb: block row ib = kb + 1 + blockIdx.x,
+// L[ib][kb] = A[ib][kb] Dinv[kb]^T.
+__global__ void __launch_bounds__(256) gptq_chol_panel_kernel(double* __restrict__ L, int K, int kb,
+                                                              const double* __restrict__ Dinv) {
+  extern __shared__ double sm[];
+  double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
+  double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
+  const int ib = kb + 1 + blockIdx.x;
+  double* tile = L + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
+  stage_tile(Ps, tile, K, true);                                           // P[r][k] = A[ib][kb][r][k]
+  stage_tile(Qs, Dinv + static_cast<long long>(kb) * kB * kB, kB, true);   // Q[k][c] = Dinv[c][k]
+  __syncthreads();
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  double acc[4][4] = {};
+  tile_product(acc, Ps, Qs, tr, tc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = acc[i][j];
+}
+
+// Trailing update after block column kb: tile (ib, jb) with kb < jb <= ib, numbered
+// row by row over the lower triangle; A[ib][jb] -= L[ib][kb] L[jb][kb]^T.
+__global__ void __launch_bounds__(256) gptq_chol_update_kernel(double* __restrict__ L, int K, int kb) {
+  extern __shared__ double sm[];
+  double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
+  double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
+  // blockIdx.x = t (t + 1) / 2 + c for tile row t, column c <= t of the trailing triangle
+  const int b = blockIdx.x;
+  int t = static_cast<int>((sqrt(8.0 * b + 1.0) - 1.0) / 2.0);
+  while ((t + 1) * (t + 2) / 2 <= b) ++t;
+  while (t * (t + 1) / 2 > b) --t;
+  const int c = b - t * (t + 1) / 2;
+  const int ib = kb + 1 + t, jb = kb + 1 + c;
+  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB, K, true);
+  stage_tile(Qs, L + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, true);
+  __syncthreads();
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  double acc[4][4] = {};
+  tile_product(acc, Ps, Qs, tr, tc);
+  double* tile = L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double* d = tile + static_cast<long long>(4 * tr + i) * K + 4 * tc + j;
+      *d -= acc[i][j];
+    }
+}
+
+// Block row ib of X = L^-1: CTA kb < ib forms X[ib][kb]; CTA ib copies Dinv[ib].
+__global__ void __launch_bounds__(256) gptq_trinv_row_kernel(const double* __restrict__ L, int K, int ib,
+                                                             const double* __restrict__ Dinv, double* __restrict__ X) {
+  extern __shared__ double sm[];
+  double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
+  double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
+  const int kb = blockIdx.x;
+  double* out = X + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  if (kb == ib) {
+    const double* dinv = Dinv + static_cast<long long>(ib) * kB * kB;
+    for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) out[static_cast<long long>(e / kB) * K + e % kB] = dinv[e];
+    return;
+  }
+  double acc[4][4] = {};
+  for (int jb = kb; jb < ib; ++jb) {
+    __syncthreads();
+    stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB, K, true);  // L[ib][jb]
+    stage_tile(Qs, X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, false); // X[jb][kb]
+    __syncthreads();
+    tile_product(acc, Ps, Qs, tr, tc);
+  }
+  // X[ib][kb] = -Dinv[ib] S, S = acc (staged as Q[k][c] = S[k][c])
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Qs[4 * tr + i][4 * tc + j] = acc[i][j];
+  stage_tile(Ps, Dinv + static_cast<long long>(ib) * kB * kB, kB, true);
+  __syncthreads();
+  double r[4][4] = {};
+  tile_product(r, Ps, Qs, tr, tc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = -r[i][j];
+}
+
+// G[K-1-i][K-1-j] = X[i][j] on and below the diagonal of X, 0 elsewhere.
+__global__ void gptq_reverse_out_kernel(const double* __restrict__ X, int K, double* __restrict__ G) {
+  const long long n = static_cast<long long>(K) * K;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int gi = static_cast<int>(e / K), gj = static_cast<int>(e % K);
+    const int i = K - 1 - gi, j = K - 1 - gj;
+    G[e] = j <= i ? X[static_cast<long long>(i) * K + j] : 0.0;
+  }
 }
 
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
 
-size_t gptq_factor_workspace_bytes(int K) { return 2 * align256(static_cast<size_t>(K) * K * 8); }
+size_t gptq_factor_workspace_bytes(int K) {
+  return 2 * align256(static_cast<size_t>(K) * K * 8) + align256(static_cast<size_t>(K) * kB * 8);
+}
 
 cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspace, cudaStream_t st) {
-  double* L = static_cast<double*>(workspace);
-  double* scratch = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + align256(static_cast<size_t>(K) * K * 8));
-  gptq_reverse_kernel<<<4 * device_sm_count(), 256, 0, st>>>(H, K, L);
-  cudaError_t e = cudaGetLastError();
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* L = reinterpret_cast<double*>(ws);
+  double* X = reinterpret_cast<double*>(ws + align256(static_cast<size_t>(K) * K * 8));
+  double* Dinv = reinterpret_cast<double*>(ws + 2 * align256(static_cast<size_t>(K) * K * 8));
+  const int nb = K / kB;
+  const int smem = 2 * kB * kBP * 8, smem_diag = 2 * kB * (kB + 1) * 8;
+  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_diag_kernel),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_diag);
+  if (e == cudaSuccess)
+    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_panel_kernel),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_update_kernel),
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_row_kernel),
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  for (int j = 0; j < K; ++j) {
-    gptq_chol_col_kernel<<<1, 32, 0, st>>>(L, K, j, true);
-    const int rows = K - 1 - j;
-    if (rows > 0) gptq_chol_col_kernel<<<(rows + 7) / 8, 256, 0, st>>>(L, K, j, false);
+  gptq_reverse_kernel<<<4 * device_sm_count(), 256, 0, st>>>(H, K, L);
+  for (int kb = 0; kb < nb && e == cudaSuccess; ++kb) {
+    gptq_chol_diag_kernel<<<1, 256, smem_diag, st>>>(L, K, kb, Dinv);
+    const int m = nb - 1 - kb;
+    if (m > 0) {
+      gptq_chol_panel_kernel<<<m, 256, smem, st>>>(L, K, kb, Dinv);
+      gptq_chol_update_kernel<<<m * (m + 1) / 2, 256, smem, st>>>(L, K, kb);
+    }
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
   }
-  gptq_trinv_kernel<<<(K + 7) / 8, 256, 0, st>>>(L, K, G, scratch);
+  for (int ib = 0; ib < nb && e == cudaSuccess; ++ib) {
+    gptq_trinv_row_kernel<<<ib + 1, 256, smem, st>>>(L, K, ib, Dinv, X);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return e;
+  gptq_reverse_out_kernel<<<4 * device_sm_count(), 256, 0, st>>>(X, K, G);
   return cudaGetLastError();
 }
 
