@@ -315,6 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tx) {
   using AR = Arith<I8>;
   constexpr int kXG = x_groups(MP);                           // groups per x stage
+  // With at most two x stages per unit (MP <= 128; the ring holds at least two)
+  // the dequantizing warps wait for a unit's x before they release its w_hat,
+  // so the MMA thread waits on one barrier per unit.  Above, a unit's four x
+  // stages do not fit the ring at once and the MMA thread waits for each.
+  constexpr bool kXByDq = 4 / kXG <= 2;
   constexpr int kXChunk = MP * 128;                           // one 128-byte chunk of every token
   constexpr int kXStage = kXG * AR::kChunks * kXChunk;
   constexpr uint32_t kIdesc = I8 ? idesc_i8(MP) : idesc_f16(MP);
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* cempty = cfull + kMaxCodeStages;               // [Sc] codes read
   uint64_t* xfull = cempty + kMaxCodeStages;               // [Sx] x landed
   uint64_t* xempty = xfull + kMaxXStages;                  // [Sx] x consumed by the MMAs
-  uint64_t* afull = xempty + kMaxXStages;                  // [kASlots] w_hat of a group written
+  uint64_t* afull = xempty + kMaxXStages;                  // [2] w_hat of a unit written (units alternate)
   uint64_t* aempty = afull + 8;                            // [kASlots] w_hat of a group consumed
   uint64_t* accfull = aempty + 8;                          // [kAcc] segment's MMAs complete
   uint64_t* accempty = accfull + 2;                        // [kAcc] accumulator read out
@@ -359,10 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1);
     }
-    for (int b = 0; b < kASlots; ++b) {
-      mbar_init(&afull[b], 4);  // the four lane-quarter warps of the group
-      mbar_init(&aempty[b], 1);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&afull[b], kDqWarps);  // a unit's w_hat, alternate units
+    for (int b = 0; b < kASlots; ++b) mbar_init(&aempty[b], 1);
     for (int b = 0; b < kAcc; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], kEpiWarps);
@@ -429,6 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
+    // A wait on an mbarrier between MMAs costs this thread about as much as 5
+    // MMAs of 128 x 16 x 16 (B200 measurement), even when the phase is already
+    // complete, so w_hat is signalled per unit (32 MMAs), not per group.
     if (lane == 0) {
       bool any = false, ok = true;
       int seg = 0;
@@ -441,10 +447,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             !wait_or_abort(&accempty[ab], static_cast<uint32_t>(seg / kAcc - 1) & 1u, abort_flag, a.status))
           break;
         const uint32_t d = tbase + static_cast<uint32_t>(ab * MP);
+        // the unit's w_hat (all four groups) is in tensor memory (and, when kXByDq,
+        // its x stages have landed: the dequantizing warps wait for those first)
+        if (!wait_or_abort(&afull[i & 1], static_cast<uint32_t>(i >> 1) & 1u, abort_flag, a.status)) break;
+        tc_fence_after();
         for (int gg = 0; gg < 4; ++gg) {
           const int j = i * xper + gg / kXG;  // x stage of this group
           const int s = j % Sx;
-          if (gg % kXG == 0 &&
+          if (!kXByDq && gg % kXG == 0 &&
               !wait_or_abort(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u, abort_flag, a.status)) {
             ok = false;
             break;
@@ -452,34 +462,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every group position of a unit takes its w_hat slot, a position past the
           // last group (K / 128 not a multiple of 4) with no MMAs, so that each slot's
           // uses follow one another in order
-          {
-            const int ga = 4 * i + gg, b = ga % kASlots;
-            if (!wait_or_abort(&afull[b], static_cast<uint32_t>(ga / kASlots) & 1u, abort_flag, a.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (4 * q4 + gg < a.G) {
-              const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * AR::kACols);
-              const uint8_t* xg = xstage + s * kXStage + (gg % kXG) * AR::kChunks * kXChunk;
+          const int ga = 4 * i + gg, b = ga % kASlots;
+          if (4 * q4 + gg < a.G) {
+            const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * AR::kACols);
+            const uint8_t* xg = xstage + s * kXStage + (gg % kXG) * AR::kChunks * kXChunk;
 #pragma unroll
-              for (int c = 0; c < AR::kChunks; ++c) {
-                const uint64_t bd = sw128_desc(xg + c * kXChunk);
+            for (int c = 0; c < AR::kChunks; ++c) {
+              const uint64_t bd = sw128_desc(xg + c * kXChunk);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  // the descriptor's start address advances 32 bytes (2 x 16) per MMA
-                  const uint32_t at = acol + 8u * (4 * c + kk);
-                  const bool accum = !(first && gg == 0 && c == 0 && kk == 0);
-                  if constexpr (I8)
-                    mma_i8_ts(d, at, bd + 2u * kk, kIdesc, accum);
-                  else
-                    mma_f16_ts(d, at, bd + 2u * kk, kIdesc, accum);
-                }
+              for (int kk = 0; kk < 4; ++kk) {
+                // the descriptor's start address advances 32 bytes (2 x 16) per MMA
+                const uint32_t at = acol + 8u * (4 * c + kk);
+                const bool accum = !(first && gg == 0 && c == 0 && kk == 0);
+                if constexpr (I8)
+                  mma_i8_ts(d, at, bd + 2u * kk, kIdesc, accum);
+                else
+                  mma_f16_ts(d, at, bd + 2u * kk, kIdesc, accum);
               }
-              any = true;
             }
-            mma_commit(&aempty[b]);
+            any = true;
           }
+          mma_commit(&aempty[b]);
           if (gg % kXG == kXG - 1) mma_commit(&xempty[s]);
         }
         if (!ok) break;
@@ -566,12 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t col = lane_base + static_cast<uint32_t>(b * AR::kACols);
-        if (!valid[e]) {
-          // a position past the last group: no w_hat, but the slot is passed on in turn
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[b]);
-          continue;
-        }
+        // a position past the last group writes no w_hat, but its slot is taken in turn
+        if (!valid[e]) continue;  // uniform over the warp
         if constexpr (I8) {
           const uint32_t s2 = dv, zs4 = static_cast<uint32_t>(zv) * 0x01010101u;
           const uint32_t zlo7 = zs4 & 0x7F7F7F7Fu, ztop = ~zs4 & 0x80808080u;
@@ -604,11 +603,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(col + static_cast<uint32_t>(16 * c), v);
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[b]);
       }
+      if (!ok) break;
+      // the unit's x stages must have landed before the MMAs are released (the MMA
+      // thread then waits on one barrier per unit)
+      bool okx = true;
+      for (int jx = i * xper; kXByDq && jx < (i + 1) * xper && okx; ++jx)
+        okx = wait_or_abort(&xfull[jx % Sx], static_cast<uint32_t>(jx / Sx) & 1u, abort_flag, a.status);
+      if (__any_sync(0xffffffffu, !okx)) break;
+      // both of this warp's groups of the unit are in tensor memory
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[i & 1]);
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------- epilogue ----------------
@@ -724,13 +731,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Ring depths: x stages for about 64 KiB of x (2 to 4), the rest of shared
-// memory for code stages (at most kMaxCodeStages).
+// Ring depths: x stages for two units of x when that fits in 128 KiB (so that
+// the x of the next unit can land while the MMAs work on this one), else two
+// stages; the rest of shared memory for code stages (at most kMaxCodeStages).
 template <int MP, bool I8>
 void ring_depths(int& sc, int& sx) {
   const int xs = x_groups(MP) * Arith<I8>::kChunks * MP * 128;
-  sx = (64 * 1024) / xs;
-  sx = sx < 2 ? 2 : (sx > 4 ? 4 : sx);
+  const int xper = 4 / x_groups(MP);
+  sx = 2 * xper * xs <= 128 * 1024 ? 2 * xper : 2;
+  sx = sx > kMaxXStages ? kMaxXStages : sx;
   sc = (kMaxSmem - 1024 - kCtrlBytes - sx * xs) / kCodeStage;
   sc = sc > kMaxCodeStages ? kMaxCodeStages : sc;
 }

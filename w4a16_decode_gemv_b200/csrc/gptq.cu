@@ -290,18 +290,24 @@ __global__ void __launch_bounds__(256) gptq_chol_diag_kernel(double* __restrict_
   double* tile = L + static_cast<long long>(kb) * kB * K + static_cast<long long>(kb) * kB;
   for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) a[e / kB][e % kB] = tile[static_cast<long long>(e / kB) * K + e % kB];
   __syncthreads();
+  // Column j: d = sqrt(a[j][j]) (kept at a[j][j]); the trailing lower triangle
+  // takes a[i][c] -= a[i][j] a[c][j] / d^2 from the unscaled column, which is
+  // divided by d only once every later column is done.  Two barriers per column.
   for (int j = 0; j < kB; ++j) {
     if (threadIdx.x == 0) a[j][j] = sqrt(a[j][j]);
     __syncthreads();
-    for (int i = j + 1 + threadIdx.x; i < kB; i += blockDim.x) a[i][j] /= a[j][j];
-    __syncthreads();
-    // trailing update of the lower triangle: a[i][c] -= a[i][j] a[c][j], j < c <= i
+    const double inv_d2 = 1.0 / (a[j][j] * a[j][j]);
     for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
       const int i = e / kB, c = e % kB;
-      if (c > j && c <= i) a[i][c] = fma(-a[i][j], a[c][j], a[i][c]);
+      if (c > j && c <= i) a[i][c] = fma(-a[i][j] * inv_d2, a[c][j], a[i][c]);
     }
     __syncthreads();
   }
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
+    const int i = e / kB, c = e % kB;
+    if (i > c) a[i][c] /= a[c][c];
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
     const int i = e / kB, c = e % kB;
     tile[static_cast<long long>(i) * K + c] = c <= i ? a[i][c] : 0.0;
@@ -372,42 +378,58 @@ __global__ void __launch_bounds__(256) gptq_chol_update_kernel(double* __restric
     }
 }
 
-// Block row ib of X = L^-1: CTA kb < ib forms X[ib][kb]; CTA ib copies Dinv[ib].
-__global__ void __launch_bounds__(256) gptq_trinv_row_kernel(const double* __restrict__ L, int K, int ib,
-                                                             const double* __restrict__ Dinv, double* __restrict__ X) {
+// X = L^-1 by right-looking forward substitution on block rows, X in place of
+// the remaining right-hand side R (L X = I): at step jb, block row jb is final,
+// X[jb][kb] = Dinv[jb] R[jb][kb] for kb < jb and X[jb][jb] = Dinv[jb]; then every
+// later block row is updated, R[ib][kb] -= L[ib][jb] X[jb][kb] for kb <= jb < ib
+// (R starts as the identity: its first update, at jb = kb, is a plain product).
+// Each step is parallel over its tiles, so the critical path is 2 K / 64 launches.
+__global__ void __launch_bounds__(256) gptq_trinv_final_kernel(int K, int jb, const double* __restrict__ Dinv,
+                                                               double* __restrict__ X) {
   extern __shared__ double sm[];
   double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
   double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
-  const int kb = blockIdx.x;
-  double* out = X + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
-  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
-  if (kb == ib) {
-    const double* dinv = Dinv + static_cast<long long>(ib) * kB * kB;
-    for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) out[static_cast<long long>(e / kB) * K + e % kB] = dinv[e];
+  const int kb = blockIdx.x;  // 0 .. jb
+  double* tile = X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB;
+  const double* dinv = Dinv + static_cast<long long>(jb) * kB * kB;
+  if (kb == jb) {
+    for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) tile[static_cast<long long>(e / kB) * K + e % kB] = dinv[e];
     return;
   }
+  stage_tile(Ps, dinv, kB, true);    // P[r][k] = Dinv[jb][r][k]
+  stage_tile(Qs, tile, K, false);    // Q[k][c] = R[jb][kb][k][c]
+  __syncthreads();
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   double acc[4][4] = {};
-  for (int jb = kb; jb < ib; ++jb) {
-    __syncthreads();
-    stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB, K, true);  // L[ib][jb]
-    stage_tile(Qs, X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, false); // X[jb][kb]
-    __syncthreads();
-    tile_product(acc, Ps, Qs, tr, tc);
-  }
-  // X[ib][kb] = -Dinv[ib] S, S = acc (staged as Q[k][c] = S[k][c])
-  __syncthreads();
+  tile_product(acc, Ps, Qs, tr, tc);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) Qs[4 * tr + i][4 * tc + j] = acc[i][j];
-  stage_tile(Ps, Dinv + static_cast<long long>(ib) * kB * kB, kB, true);
+    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = acc[i][j];
+}
+
+// Update after step jb: CTA (blockIdx.x = kb <= jb, blockIdx.y = ib - jb - 1).
+__global__ void __launch_bounds__(256) gptq_trinv_update_kernel(const double* __restrict__ L, int K, int jb,
+                                                                double* __restrict__ X) {
+  extern __shared__ double sm[];
+  double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
+  double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
+  const int kb = blockIdx.x, ib = jb + 1 + blockIdx.y;
+  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB, K, true);   // L[ib][jb]
+  stage_tile(Qs, X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, false);  // X[jb][kb]
   __syncthreads();
-  double r[4][4] = {};
-  tile_product(r, Ps, Qs, tr, tc);
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  double acc[4][4] = {};
+  tile_product(acc, Ps, Qs, tr, tc);
+  double* tile = X + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
+  const bool first = kb == jb;  // R[ib][kb] is still the zero block of the identity
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) out[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = -r[i][j];
+    for (int j = 0; j < 4; ++j) {
+      double* d = tile + static_cast<long long>(4 * tr + i) * K + 4 * tc + j;
+      *d = first ? -acc[i][j] : *d - acc[i][j];
+    }
 }
 
 // G[K-1-i][K-1-j] = X[i][j] on and below the diagonal of X, 0 elsewhere.
@@ -445,7 +467,10 @@ cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspac
     e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_update_kernel),
                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
-    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_row_kernel),
+    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_final_kernel),
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_update_kernel),
                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   gptq_reverse_kernel<<<4 * device_sm_count(), 256, 0, st>>>(H, K, L);
@@ -458,8 +483,9 @@ cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspac
     }
     e = cudaGetLastError();
   }
-  for (int ib = 0; ib < nb && e == cudaSuccess; ++ib) {
-    gptq_trinv_row_kernel<<<ib + 1, 256, smem, st>>>(L, K, ib, Dinv, X);
+  for (int jb = 0; jb < nb && e == cudaSuccess; ++jb) {
+    gptq_trinv_final_kernel<<<jb + 1, 256, smem, st>>>(K, jb, Dinv, X);
+    if (jb + 1 < nb) gptq_trinv_update_kernel<<<dim3(jb + 1, nb - 1 - jb), 256, smem, st>>>(L, K, jb, X);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
