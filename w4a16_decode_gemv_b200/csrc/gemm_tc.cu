@@ -129,6 +129,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       : "memory");
 }
 
+// 32 lanes x 32 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns into registers: thread i reads lane (base + i).
@@ -574,33 +586,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (I8) {
           const uint32_t s2 = dv, zs4 = static_cast<uint32_t>(zv) * 0x01010101u;
           const uint32_t zlo7 = zs4 & 0x7F7F7F7Fu, ztop = ~zs4 & 0x80808080u;
+          uint32_t v[32];
 #pragma unroll
-          for (int c = 0; c < 4; c += 2) {
-            uint32_t v[16];
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              dq8_word((&cw[e][c].x)[k], s2, zlo7, ztop, v[2 * k], v[2 * k + 1]);
-              dq8_word((&cw[e][c + 1].x)[k], s2, zlo7, ztop, v[8 + 2 * k], v[8 + 2 * k + 1]);
-            }
-            tmem_st16(col + static_cast<uint32_t>(8 * c), v);
-          }
+            for (int k = 0; k < 4; ++k) dq8_word((&cw[e][c].x)[k], s2, zlo7, ztop, v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
+          tmem_st32(col, v);
         } else {
           const __half2 dd = as_h2(static_cast<uint32_t>(dv) | (static_cast<uint32_t>(dv) << 16));
           // -(1024 + z) as an fp16 pair (z is a small non-negative integer held in fp16)
           const __half zh = __hneg(__hadd(__ushort_as_half(zv), __float2half_rn(1024.0f)));
           const __half2 nz = __halves2half2(zh, zh);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t wv[4] = {cw[e][c].x, cw[e][c].y, cw[e][c].z, cw[e][c].w};
-            uint32_t v[16];
+          for (int c = 0; c < 4; c += 2) {
+            uint32_t v[32];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              v[4 * k + 0] = dq_pair(wv[k], nz, dd);
-              v[4 * k + 1] = dq_pair(wv[k] >> 4, nz, dd);
-              v[4 * k + 2] = dq_pair(wv[k] >> 8, nz, dd);
-              v[4 * k + 3] = dq_pair(wv[k] >> 12, nz, dd);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const uint32_t wv[4] = {cw[e][c + h2].x, cw[e][c + h2].y, cw[e][c + h2].z, cw[e][c + h2].w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                v[16 * h2 + 4 * k + 0] = dq_pair(wv[k], nz, dd);
+                v[16 * h2 + 4 * k + 1] = dq_pair(wv[k] >> 4, nz, dd);
+                v[16 * h2 + 4 * k + 2] = dq_pair(wv[k] >> 8, nz, dd);
+                v[16 * h2 + 4 * k + 3] = dq_pair(wv[k] >> 12, nz, dd);
+              }
             }
-            tmem_st16(col + static_cast<uint32_t>(16 * c), v);
+            tmem_st32(col + static_cast<uint32_t>(16 * c), v);
           }
         }
       }

@@ -48,14 +48,26 @@ namespace w4a16 {
 namespace {
 
 constexpr int kR = 4;                         // rows per unit (= rows per row block)
-constexpr int kUW = 256;                      // words per unit row (2048 channels)
-constexpr int kUB = kR * kUW * 4;             // 4 KiB of codes per unit
-constexpr int kUG = kUW / 16;                 // 16 groups per unit row
-constexpr int kStage = kUB + 2 * kR * kUG * 2;  // + Delta and z tiles (4 x 16 fp16 each)
-constexpr int kSlice = 36;                    // 4-byte words per 64-channel lane slice (33 used)
 constexpr int kXBatch = 4;                    // activation words a thread loads at once while staging
 constexpr int kMaxSmem = 227 * 1024;
 constexpr float kTwo24 = 16777216.0f;        // 2^24
+
+// The geometry of a unit of 4 rows x UW words: UW = 256 (2048 channels, 4 KiB
+// of codes) or 128 (1024 channels, 2 KiB).  Lane l owns kWPL = UW / 32
+// consecutive words (8 kWPL channels) of each unit row; its staged activations
+// are a slice of kSlice 4-byte words: the 8 kWPL fp16 values, 2^-24 times their
+// sum, padding (16 bytes, so that 128-bit reads of consecutive slices hit
+// distinct banks within a quarter-warp phase).
+template <int UW>
+struct Geo {
+  static constexpr int kUW = UW;
+  static constexpr int kWPL = UW / 32;
+  static constexpr int kUB = kR * UW * 4;              // codes per unit
+  static constexpr int kUG = UW / 16;                  // groups per unit row
+  static constexpr int kStage = kUB + 2 * kR * kUG * 2;  // + Delta and z tiles (4 x kUG fp16 each)
+  static constexpr int kSliceCh = 8 * kWPL;            // channels per lane slice
+  static constexpr int kSlice = 4 * kWPL + 4;          // 4-byte words per slice (4 kWPL + 1 used)
+};
 
 struct M1Args {
   const __half* x;
@@ -97,20 +109,24 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Issues the copies of unit (rb, kc) into a stage: lane 0 the 4 x 256-word
-// code box (one TMA op; rows past N and words past K/8 arrive as zeros), every
-// lane 4 bytes of the Delta tile and 4 of the z tile with cp.async (the group
-// count per row is even, so these pairs are 4-byte aligned).
+// Issues the copies of unit (rb, kc) into a stage: lane 0 the 4 x UW-word
+// code box (one TMA op; rows past N and words past K/8 arrive as zeros), lanes
+// (tile row, group pair) 4 bytes of the Delta tile and 4 of the z tile with
+// cp.async (the group count per row is even, so these pairs are 4-byte
+// aligned); every lane arrives once its copies have landed.
+template <int UW>
 __device__ __forceinline__ void issue_unit(const M1Args& a, const CUtensorMap* tmap, int rb, int kc, uint8_t* dst,
                                            uint64_t* bar, int lane, uint64_t pol) {
+  using G = Geo<UW>;
+  constexpr int kUB = G::kUB, kUG = G::kUG, kPairs = G::kUG / 2;
   const int n0 = rb * kR;
   if (lane == 0) {
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kUB));
-    tma_load_2d(dst, tmap, kc * kUW, n0, bar, pol);
+    tma_load_2d(dst, tmap, kc * UW, n0, bar, pol);
   }
   const int rows = min(kR, a.N - n0);
-  const int words = min(kUW, a.Kw - kc * kUW);
-  const int tr = lane >> 3, tc = lane & 7;  // tile row and group pair of this lane
+  const int words = min(UW, a.Kw - kc * UW);
+  const int tr = lane / kPairs, tc = lane % kPairs;  // tile row and group pair of this lane
   if (tr < rows && 2 * tc < words / 16) {
     const size_t o = static_cast<size_t>(n0 + tr) * a.Kg + kc * kUG + 2 * tc;
     __half* tile = reinterpret_cast<__half*>(dst + kUB);
@@ -129,11 +145,13 @@ __device__ __forceinline__ void issue_unit(const M1Args& a, const CUtensorMap* t
 // warps no longer leave HBM idle.  CTAS = 1: 16 warps (12 when 16 rings do not
 // fit beside the staged activations of a large K) owning the whole SM, with
 // only the first stage fetched before the wait.
-template <int WARPS, int CTAS>
+template <int WARPS, int CTAS, int UW>
 __global__ void __launch_bounds__(WARPS * 32, CTAS)
     gemv_m1_kernel(const M1Args a, const __grid_constant__ CUtensorMap tmap) {
+  using G = Geo<UW>;
   constexpr int kWarps = WARPS;
   constexpr int kThreads = WARPS * 32;
+  constexpr int kUW = UW, kWPL = G::kWPL, kUB = G::kUB, kUG = G::kUG, kStage = G::kStage, kSlice = G::kSlice;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.stages;
@@ -166,7 +184,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
   int rb_f = rb0 + warp / a.units_k, kc_f = warp % a.units_k;
   int jf = warp;
   auto issue_next = [&](int s) {
-    issue_unit(a, &tmap, rb_f, kc_f, ring + static_cast<size_t>(s) * kStage, &full[s], lane, pol);
+    issue_unit<UW>(a, &tmap, rb_f, kc_f, ring + static_cast<size_t>(s) * kStage, &full[s], lane, pol);
     jf += kWarps;
     rb_f += drb, kc_f += dkc;
     if (kc_f >= a.units_k) kc_f -= a.units_k, ++rb_f;
@@ -176,11 +194,12 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
   // x, y and anything earlier kernels produce are touched only after this
   griddep_wait();
 
-  // Word c of x (8 channels) is word c & 7 of lane slice c >> 3.  The slice's
-  // lane (c >> 3) & 31 reads its second 16-byte half first when bit 2 of the
-  // lane index is set (see swap1 below), so the words are stored in that order.
-  // Word 32 of each slice holds 2^-24 times the sum of its 64 channels.
-  // K / 8 is a multiple of 16, so the 8 words of a slice are 8 aligned lanes.
+  // Word c of x (8 channels) is word c % kWPL of lane slice c / kWPL.  With 8
+  // words per lane (UW = 256) the slice's lane (c >> 3) & 31 reads its second
+  // 16-byte half first when bit 2 of the lane index is set (see swap1 below),
+  // so the words are stored in that order.  Word 4 kWPL of each slice holds
+  // 2^-24 times the sum of its channels.  K / 8 is a multiple of 16, so the
+  // kWPL words of a slice are kWPL aligned lanes.
   // All of a thread's loads are issued before any is used, so the staging costs
   // one trip to L2 rather than one per word.
   // The loop bound is the warp's first word, so every lane runs every shuffle;
@@ -199,8 +218,8 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
       const bool valid = c < a.K / 8;
       const uint32_t hv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
       // position of word c in its owning lane's read order
-      const int jj = ((c & 7) - 4 * ((c >> 5) & 1)) & 7;
-      float* slice = xs + (c >> 3) * kSlice;
+      const int jj = kWPL == 8 ? ((c & 7) - 4 * ((c >> 5) & 1)) & 7 : c % kWPL;
+      float* slice = xs + (c / kWPL) * kSlice;
       float sum = 0.0f;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -208,10 +227,9 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
         sum += f.x + f.y;
       }
       if (valid) *reinterpret_cast<uint4*>(slice + 4 * jj) = v[q];
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      if (valid && (c & 7) == 0) slice[32] = sum * pow2f(-24);
+#pragma unroll
+      for (int o = 1; o < kWPL; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (valid && c % kWPL == 0) slice[4 * kWPL] = sum * pow2f(-24);
     }
   }
   __syncthreads();
@@ -222,14 +240,14 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
   // weight row first, so that the 32-byte lane stride does not put two lanes of
   // a quarter-warp phase on the same banks (their x slices are staged in the
   // same order).
-  const int swap1 = (lane >> 2) & 1;
+  const int swap1 = kWPL == 8 ? (lane >> 2) & 1 : 0;
   bool failed = false;
   int kc = warp % a.units_k;
   // this lane's staged activations for channel block xkc (reloaded only when the
   // warp's block changes; with 16 warps and K / 2048 dividing 16 it never does)
   int xkc = -1;
-  uint32_t xh[32];     // x as fp16 pairs, the lane's 8 words in read order
-  float xsum = 0.0f;  // 2^-24 x the sum of this lane's 64 activations
+  uint32_t xh[4 * kWPL];  // x as fp16 pairs, the lane's kWPL words in read order
+  float xsum = 0.0f;      // 2^-24 x the sum of this lane's activations
   for (int j = warp, i = 0; j < U; j += kWarps, ++i) {
     const int s = i % S;
     const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
@@ -237,15 +255,15 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
     kc += dkc;
     if (kc >= a.units_k) kc -= a.units_k;
 
-    const bool act = lane * 8 < min(kUW, a.Kw - ckc * kUW);
+    const bool act = lane * kWPL < min(kUW, a.Kw - ckc * kUW);
     if (ckc != xkc) {
       xkc = ckc;
       if (act) {
-        const float* sl = xs + (ckc * (kUW / 8) + lane) * kSlice;
-        xsum = sl[32];
+        const float* sl = xs + (ckc * 32 + lane) * kSlice;
+        xsum = sl[4 * kWPL];
         const uint4* xb = reinterpret_cast<const uint4*>(sl);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kWPL; ++k) {
           const uint4 v = xb[k];
           xh[4 * k] = v.x;
           xh[4 * k + 1] = v.y;
@@ -266,23 +284,28 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
     for (int r = 0; r < kR; ++r) acc[r] = 0.0f;
     uint8_t* stage = ring + static_cast<size_t>(s) * kStage;
     if (act) {
-      const ulonglong2* wq = reinterpret_cast<const ulonglong2*>(stage) + 2 * lane + swap1;
-      const __half* tile = reinterpret_cast<const __half*>(stage + kUB) + (lane >> 1);
+      // the lane's kWPL words of each row: one or two 16-byte reads (two: the
+      // half nearer the lane's bank first, as its activations were staged)
+      const uint4* wq = reinterpret_cast<const uint4*>(stage) + (kWPL / 4) * lane + swap1;
+      const __half* tile = reinterpret_cast<const __half*>(stage + kUB) + lane / (16 / kWPL);
 #pragma unroll
       for (int r = 0; r < kR; ++r) {
-        const ulonglong2 wa = wq[r * (kUW / 4)];
-        const ulonglong2 wb = wq[r * (kUW / 4) + 1 - 2 * swap1];
+        uint32_t hw[kWPL];
+        {
+          const uint4 wa = wq[r * (kUW / 4)];
+          hw[0] = wa.x, hw[1] = wa.y, hw[2] = wa.z, hw[3] = wa.w;
+          if constexpr (kWPL == 8) {
+            const uint4 wb = wq[r * (kUW / 4) + 1 - 2 * swap1];
+            hw[4] = wb.x, hw[5] = wb.y, hw[6] = wb.z, hw[7] = wb.w;
+          }
+        }
         const float zf = __half2float(tile[kR * kUG + r * kUG]);
         const float df = __half2float(tile[r * kUG]) * kTwo24;
         // u 2^-24 (bits 0..3 of each 16-bit half) and u 2^-20 (bits 4..7) are
         // fp16 subnormals; their products with x are exact in fp32
         float e0 = 0.0f, e1 = 0.0f, o0 = 0.0f, o1 = 0.0f;
-        const uint32_t hw[8] = {static_cast<uint32_t>(wa.x), static_cast<uint32_t>(wa.x >> 32),
-                                static_cast<uint32_t>(wa.y), static_cast<uint32_t>(wa.y >> 32),
-                                static_cast<uint32_t>(wb.x), static_cast<uint32_t>(wb.x >> 32),
-                                static_cast<uint32_t>(wb.y), static_cast<uint32_t>(wb.y >> 32)};
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kWPL; ++k) {
           const uint32_t w = hw[k], w8 = w >> 8;
           fma2_f16_f32(w & 0x000F000Fu, xh[4 * k], e0, e1);
           fma2_f16_f32(w & 0x00F000F0u, xh[4 * k + 1], o0, o1);
@@ -331,10 +354,14 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
 
 int round128(int b) { return (b + 127) / 128 * 128; }
 
-int x_bytes_for(int K) { return round128((K / 64) * kSlice * 4); }
+int slice_ch(int uw) { return uw == 256 ? Geo<256>::kSliceCh : Geo<128>::kSliceCh; }
+int slice_words(int uw) { return uw == 256 ? Geo<256>::kSlice : Geo<128>::kSlice; }
+int stage_bytes(int uw) { return uw == 256 ? Geo<256>::kStage : Geo<128>::kStage; }
 
-int smem_for(int warps, int stages, int x_bytes, int max_units) {
-  return x_bytes + warps * stages * kStage + round128(max_units * kR * 4) + warps * stages * 8;
+int x_bytes_for(int K, int uw) { return round128((K / slice_ch(uw)) * slice_words(uw) * 4); }
+
+int smem_for(int warps, int stages, int x_bytes, int max_units, int uw) {
+  return x_bytes + warps * stages * stage_bytes(uw) + round128(max_units * kR * 4) + warps * stages * 8;
 }
 
 // Shared memory of an SM (228 KiB) less 1 KiB the system reserves per CTA,
@@ -342,37 +369,40 @@ int smem_for(int warps, int stages, int x_bytes, int max_units) {
 constexpr int kMaxSmemPair = (228 * 1024) / 2 - 1024;
 
 struct M1Config {
-  int warps, ctas, stages, smem, grid, max_units;
+  int warps, ctas, uw, stages, smem, grid, max_units;
 };
 
 // Two 8-warp CTAs per SM when a CTA's ring holds all of its units, so that the
 // whole layer is fetched before the previous layer ends (on B200 that paid at
 // 4096 x 4096: 3.65 against 4.23 us per layer; for larger layers the shallower
 // rings of two CTAs lost more than the overlap gained: 10.5 against 9.2 us at
-// 8192 x 8192); else one CTA of 16 warps (12 if 16 two-stage rings do not
-// fit); the deepest ring (up to 6 stages) that fits.  False when nothing fits.
+// 8192 x 8192).  Else one CTA of 16 warps (12 if 16 two-stage rings do not
+// fit); the deepest ring (up to 6 stages) that fits.  Units are 4 rows x 2048
+// channels.  (Units of 1024 channels would balance the warps better, 6.5 to 7
+// units each instead of 3 or 4, but on B200 they were slower at every layer
+// shape, 11.3 against 9.2 us at 8192 x 8192: each unit costs its warp a tensor
+// copy issue and a barrier wait, both of which take a fixed, long time.)
+// False when nothing fits.
 bool m1_config(int N, int K, M1Config& c) {
   const int sms = device_sm_count();
   const int row_blocks = (N + kR - 1) / kR;
   c.grid = min(sms, row_blocks);
-  c.max_units = ((row_blocks + c.grid - 1) / c.grid) * ((K / 8 + kUW - 1) / kUW);
-  const int xb = x_bytes_for(K);
   const struct {
-    int warps, ctas, limit;
-  } shapes[3] = {{8, 2, kMaxSmemPair}, {16, 1, kMaxSmem}, {12, 1, kMaxSmem}};
+    int warps, ctas, uw, limit, max_stages;
+  } shapes[3] = {{8, 2, 256, kMaxSmemPair, 6}, {16, 1, 256, kMaxSmem, 6}, {12, 1, 256, kMaxSmem, 6}};
   for (const auto& sh : shapes) {
-    if (smem_for(sh.warps, 2, xb, c.max_units) > sh.limit) continue;
-    if (sh.ctas == 2) {
-      int st = 6;
-      while (st > 2 && smem_for(sh.warps, st, xb, c.max_units) > sh.limit) --st;
-      if (sh.warps * st < c.max_units) continue;  // the ring cannot hold the CTA's units
-    }
-    int st = 6;
-    while (st > 2 && smem_for(sh.warps, st, xb, c.max_units) > sh.limit) --st;
+    const int max_units = ((row_blocks + c.grid - 1) / c.grid) * ((K / 8 + sh.uw - 1) / sh.uw);
+    const int xb = x_bytes_for(K, sh.uw);
+    if (smem_for(sh.warps, 2, xb, max_units, sh.uw) > sh.limit) continue;
+    int st = sh.max_stages;
+    while (st > 2 && smem_for(sh.warps, st, xb, max_units, sh.uw) > sh.limit) --st;
+    if (sh.ctas == 2 && sh.warps * st < max_units) continue;  // the ring cannot hold the CTA's units
     c.warps = sh.warps;
     c.ctas = sh.ctas;
+    c.uw = sh.uw;
     c.stages = st;
-    c.smem = smem_for(sh.warps, st, xb, c.max_units);
+    c.max_units = max_units;
+    c.smem = smem_for(sh.warps, st, xb, max_units, sh.uw);
     return true;
   }
   return false;
@@ -412,23 +442,23 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   a.K = p.K;
   a.Kw = p.K / 8;
   a.Kg = p.K / kGroup;
-  a.units_k = (a.Kw + kUW - 1) / kUW;
-  a.row_blocks = (p.N + kR - 1) / kR;
   M1Config c;
   if (!m1_config(p.N, p.K, c)) return cudaErrorNotSupported;
+  a.units_k = (a.Kw + c.uw - 1) / c.uw;
+  a.row_blocks = (p.N + kR - 1) / kR;
   const int grid = c.grid;
   a.max_units = c.max_units;
-  a.x_bytes = x_bytes_for(p.K);
+  a.x_bytes = x_bytes_for(p.K, c.uw);
   a.stages = c.stages;
   const int smem = c.smem;
 
-  // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x 256.
+  // qweight as a 2-D tensor of u32: [N rows][K/8 words], boxes of 4 x UW.
   // The map depends only on the pointer and the shape, so the maps of the
   // last few weights this thread launched on are kept (a decode step visits
   // the same layers every token) and encoding is skipped for them.
   struct CachedMap {
     const uint32_t* ptr;
-    int n, kw;
+    int n, kw, uw;
     CUtensorMap map;
   };
   constexpr int kMapCache = 64;
@@ -436,13 +466,14 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
   thread_local int cache_next = 0;
   const CUtensorMap* tmap = nullptr;
   for (int i = 0; i < kMapCache && !tmap; ++i)
-    if (cache[i].ptr == p.qweight && cache[i].n == p.N && cache[i].kw == a.Kw) tmap = &cache[i].map;
+    if (cache[i].ptr == p.qweight && cache[i].n == p.N && cache[i].kw == a.Kw && cache[i].uw == c.uw)
+      tmap = &cache[i].map;
   if (!tmap) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.Kw), static_cast<cuuint64_t>(p.N)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.Kw) * 4};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kUW), static_cast<cuuint32_t>(kR)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(c.uw), static_cast<cuuint32_t>(kR)};
     const cuuint32_t estr[2] = {1, 1};
     CachedMap& slot = cache[cache_next];
     if (enc(&slot.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(p.qweight), dims, strides, box,
@@ -454,11 +485,13 @@ cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t 
     slot.ptr = p.qweight;
     slot.n = p.N;
     slot.kw = a.Kw;
+    slot.uw = c.uw;
     tmap = &slot.map;
     cache_next = (cache_next + 1) % kMapCache;
   }
 
-  auto kern = c.ctas == 2 ? gemv_m1_kernel<8, 2> : (c.warps == 16 ? gemv_m1_kernel<16, 1> : gemv_m1_kernel<12, 1>);
+  auto kern = c.ctas == 2 ? gemv_m1_kernel<8, 2, 256>
+                          : (c.warps == 16 ? gemv_m1_kernel<16, 1, 256> : gemv_m1_kernel<12, 1, 256>);
   cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e == cudaSuccess)
     e = ensure_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
