@@ -607,7 +607,7 @@ def other_workloads(args, dev):
                 e = {"M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(b / us / 1e3, 1),
                      "hbm_frac": round(b / us / 1e3 / hbm_peak, 4), "tflops": round(2 * M * N * K / us / 1e6, 2)}
                 if M > 4:
-                    e["path"] = "tcgen05 tensor cores" + (f", {-(-M // 128)} chunks of <= 128 tokens" if M > 128 else "")
+                    e["path"] = "tcgen05 tensor cores" + (f", {-(-M // 256)} chunks of <= 256 tokens" if M > 256 else "")
                     e["tensor_frac"] = round(2 * M * N * K / us / 1e6 / tc_peak, 4)
                 if M >= 16:
                     e["cublas_fp16_us"] = round(cublas_us(M, N, K), 3)

@@ -573,11 +573,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fetch(2 * i + e + kLook, pd[kLook - 1], pz[kLook - 1]);
         const int ga = 4 * i + gg, b = ga % kASlots;
-        const bool oka = ga < kASlots ||
-                         wait_or_abort(&aempty[b], static_cast<uint32_t>(ga / kASlots - 1) & 1u, abort_flag, a.status);
-        if (__any_sync(0xffffffffu, !oka)) {
-          ok = false;
-          break;
+        // Both of this warp's slots of the unit must be free.  The MMA thread
+        // commits the slots in group order and a commit arrives only once every
+        // earlier MMA has completed, so the wait for the later slot (group ga + 2)
+        // covers both: one barrier wait per unit (each costs hundreds of cycles).
+        if (e == 0) {
+          const int gl = ga + 2;
+          const bool oka = gl < kASlots || wait_or_abort(&aempty[gl % kASlots], static_cast<uint32_t>(gl / kASlots - 1) & 1u,
+                                                         abort_flag, a.status);
+          if (__any_sync(0xffffffffu, !oka)) {
+            ok = false;
+            break;
+          }
         }
         tc_fence_after();
         const uint32_t col = lane_base + static_cast<uint32_t>(b * AR::kACols);
@@ -617,9 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // the unit's x stages must have landed before the MMAs are released (the MMA
-      // thread then waits on one barrier per unit)
+      // thread then waits on one barrier per unit); one warp's wait is enough, as
+      // the barrier completes only with every warp's arrival
       bool okx = true;
-      for (int jx = i * xper; kXByDq && jx < (i + 1) * xper && okx; ++jx)
+      for (int jx = i * xper; kXByDq && warp == kDqWarp0 && jx < (i + 1) * xper && okx; ++jx)
         okx = wait_or_abort(&xfull[jx % Sx], static_cast<uint32_t>(jx / Sx) & 1u, abort_flag, a.status);
       if (__any_sync(0xffffffffu, !okx)) break;
       // both of this warp's groups of the unit are in tensor memory
