@@ -119,11 +119,13 @@ W4A16_API w4a16_status awq_quantize_pack(const void* W, const void* s, int N, in
 /*
  * w4a16_gemm_workspace_size -- bytes of workspace that w4a16_gemm needs.
  * Returns 0 for invalid sizes.  The workspace holds a device status word,
- * per-row-block arrival counters and fp32 split-K partial sums (M x N for
- * M <= 4); for M >= 5 it adds, after room for the M = 4 partial sums, two
- * 256 x MP fp32 slots per streaming multiprocessor of the current device for
- * the tensor-core path's partial sums (MP = M rounded up to 16 up to 64, then
- * 96 or 128).  For M > 128 it is the size for M = 128.
+ * 1024 partial-tile flags, per-row-block arrival counters and fp32 split-K
+ * partial sums (M x N for M <= 4); for M >= 5 it adds, after room for the
+ * M = 4 partial sums, one 128 x MP fp32 partial-tile slot per streaming
+ * multiprocessor of the current device for the tensor-core path (MP, the
+ * token tile, is one of 16, 32, 64, 96, 128, 192, 256: the smallest that
+ * holds M).  For M > 256 it is the size for M = 256.  Everything before the
+ * slots must be zero before the first call; every completed call leaves it so.
  */
 W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
 
@@ -133,16 +135,17 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  *   y[m][n] = fp16( sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k] )
  *
  * with fp32 accumulation.  M = 1..4 runs on the CUDA cores (M = 1: whole rows
- * per SM, no partial sums; M = 2..4: whole rows or split-K); M = 5..128 runs on
+ * per SM, no partial sums; M = 2..4: whole rows or split-K); M = 5..256 runs on
  * the tensor cores (tcgen05), with w_hat = Delta * (u - z) rounded once to fp16
  * before the MMA (so |w_hat| must stay below 65504).  Larger M (prefill) runs
- * as consecutive chunks of 128 tokens, each chunk as above, on the same
+ * as consecutive chunks of 256 tokens, each chunk as above, on the same
  * workspace.  x is the activation already divided by the AWQ scale s.
  * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
  * y_ref the exact product with the dequantized weight.  y is the same on every
- * call, bit for bit, except on the split-K CUDA-core GEMV, which serves M = 1..4
- * when the whole-row kernels do not apply (K / 128 odd, or activations too
- * large to stage) and whose partial sums may be added in another order.
+ * call, bit for bit, on every path: the split-K CUDA-core GEMV (M = 1..4 when
+ * the whole-row kernels do not apply: K / 128 odd, or activations too large
+ * to stage) adds at most two partial sums per output onto zero, and the
+ * tensor-core path adds its partial tiles in a fixed order.
  *
  *   x        fp16 [M][K], device.     y  fp16 [M][N], device (output).
  *   qweight, scales, zeros as produced by awq_quantize_pack (layout v1).
@@ -185,9 +188,7 @@ W4A16_API size_t awq_search_workspace_size(int N, int K, int T, int n_alpha, int
  * library's own entry point above, so the codes of the chosen alpha are the
  * ones awq_quantize_pack produces for it.  y is formed once, in fp32 on the
  * CUDA cores, from the exact fp16 products; each loss is an fp64 sum in a fixed
- * order, so the losses repeat exactly from call to call whenever the GEMM
- * outputs do (always unless a final chunk of 1 to 4 tokens runs on the split-K
- * GEMV, whose y may differ in the last bit).
+ * order, so the losses repeat exactly from call to call, as the GEMM outputs do.
  *
  *   W        fp16 [N][K], device.    X  fp16 [T][K] calibration tokens, device.
  *   alphas   double [n_alpha], host, finite (the pages search [0, 1]).

@@ -251,6 +251,23 @@ def test_gemv_skinny_m4(dev):
     assert np.all(np.abs(y.cpu().numpy()[:, rows].astype(np.float64) - y_ref) <= RTOL * B + ATOL)
 
 
+@pytest.mark.parametrize("M,N,K", [(4, 2048, 22016), (3, 513, 1152), (1, 300, 1152), (2, 512, 65536)])
+def test_split_k_gemv_repeats_bit_for_bit(dev, M, N, K):
+    """The split-K GEMV (activations too large to stage, or K / 128 odd) adds at most
+    two partial sums per output onto zero, so y is the same on every call."""
+    W, x = inputs.random_case(M * 13 + N, N, K, M)
+    qo, so, zo = oracle.quantize_pack(W[:64], None, 128, 4, oracle.ASYM)
+    qg, sg, zg = w4.awq_quantize_pack(to_dev(W, dev))
+    assert np.array_equal(qw_np(qg)[:64], qo)
+    xd = to_dev(x, dev)
+    ys = [w4.w4a16_gemm(xd, qg, sg, zg).cpu().numpy().view(np.uint16) for _ in range(6)]
+    for y in ys[1:]:
+        assert np.array_equal(y, ys[0])
+    y_ref, B = oracle.gemm(x, qo, so, zo)
+    err = np.abs(ys[0].view(np.float16)[:, :64].astype(np.float64) - y_ref)
+    assert np.all(err <= RTOL * B + ATOL)
+
+
 def test_workspace_left_zeroed_and_calls_repeat(dev):
     W, x = inputs.random_case(42, 300, 4096, 1)
     qo, so, zo = oracle.quantize_pack(W, None, 128, 4, oracle.ASYM)

@@ -1,5 +1,6 @@
 // C ABI of the w4a16 library: argument checks, error reporting, dispatch.
 // The operations themselves are specified in include/w4a16.h.
+#include <atomic>
 #include <vector>
 #include <mutex>
 #include <cmath>
@@ -46,15 +47,16 @@ constexpr long long kMaxElems = 1ll << 31;  // index arithmetic stays in 64 bits
 void set_last_error(const char* msg) { g_last_error = msg; }
 
 int device_sm_count() {
-  static int cached[128] = {0};
+  // per-device cache; threads that race on a first call store the same value
+  static std::atomic<int> cached[128];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 cudaError_t ensure_func_attr(const void* func, cudaFuncAttribute attr, int value) {

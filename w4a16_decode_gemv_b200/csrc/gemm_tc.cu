@@ -20,28 +20,34 @@
 // zero-filled by the tensor copy), fp32 accumulators in tensor memory.  Keeping
 // A out of shared memory leaves shared memory to the copies alone.
 //
-// Work split (stream-K).  Units are (tile of 128 rows, pair of groups = 256
-// inputs), ordered tile-major and dealt to a persistent grid (one CTA per SM) in
+// Work split (stream-K).  Units are (tile of 128 rows, 4 groups = 512 inputs),
+// ordered tile-major and dealt to a persistent grid (one CTA per SM) in
 // contiguous, equal ranges.  A CTA's range covers at most a few tiles; it
 // accumulates each one (a segment) in a tensor-memory accumulator.  A tile no
 // single CTA covers is finished by the lowest CTA that covers part of it (its
 // owner), for which the tile is the last segment: every other contributor has
 // the tile as its first segment, publishes its fp32 partial tile to a workspace
-// slot and sets a flag; the owner, after its own MMAs, waits for those flags
-// (bounded), adds the partials in CTA order and writes y.  y does not depend on
-// timing, and no second kernel is needed.
+// slot and adds 1 to its flag per epilogue warp; the owner, after its own MMAs,
+// waits for those flags (bounded), adds the partials in CTA order, writes y and
+// puts the flags back to 0.  y does not depend on timing, and no second kernel
+// is needed.
 //
 // Roles (16 warps):
-//   warp 0       one thread streams the code tiles: one tensor copy per unit
-//                (128 rows x 128 bytes, 128-byte swizzle) into a ring of Sc stages;
+//   warp 0       one thread streams the codes: per unit two adjacent tensor
+//                copies of 128 rows x 128 bytes (128-byte swizzle, 32 KiB in
+//                all) into a ring of Sc stages;
 //   warp 1       allocates tensor memory; one thread issues the MMAs (8 of
-//                128 x MP x 16 per group) and their commits;
-//   warp 2       one thread streams the x tiles (per group: two boxes of MP rows x
-//                64 inputs) into a ring of Sx stages, after griddepcontrol.wait;
+//                128 x MP x 16 per group, W4A16; 4 of 128 x MP x 32, W4A8) and
+//                their commits, waiting on one barrier per unit;
+//   warps 2, 3   one thread each streams x, alternating stages: one 3-D tensor
+//                copy of a [K / 64][M][64] view per stage (a unit's x up to
+//                MP = 32, half of it up to 128, one group above), after
+//                griddepcontrol.wait;
 //   warps 4-11   dequantization: warp w covers tensor-memory lane quarter w & 3
-//                (rows 32 (w & 3) .. + 31 of the tile) and group h = (w - 4) >> 2
-//                of each pair; lane i reads its row's 64 code bytes, converts them
-//                into 64 columns of w_hat and stores them with tcgen05.st;
+//                (rows 32 (w & 3) .. + 31 of the tile) and groups h and h + 2
+//                (h = (w - 4) >> 2) of each unit; lane i reads its row's 64 code
+//                bytes per group, converts them into w_hat and stores them with
+//                tcgen05.st;
 //   warps 12-15  epilogue: accumulator read-out, y, partial tiles, the owner's sums.
 // Dequantization of a code pair: (w >> 4t) & 0x000F000F | 0x64006400 (one LOP3)
 // reads as the fp16 pair 1024 + q; subtracting 1024 + z is exact and the

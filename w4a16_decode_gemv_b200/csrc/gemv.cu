@@ -21,6 +21,9 @@
 // block changes the warp reduces them with shuffles and either writes y (it
 // covered the whole row) or adds them into the fp32 workspace, the last
 // contributor of a row block converting to fp16 and zeroing the workspace behind it.
+// Every warp takes at least units_k - 1 units (fewer warps run when the units
+// are few), so a row block has at most two contributors; their two fp32 adds
+// onto zero commute, and y is the same on every call.
 //
 // This file holds the kernel for M = 2..4 (and for M = 1 when K is too large
 // for the dedicated M = 1 kernel of gemv_m1.cu): units of 4 rows, codes
@@ -50,6 +53,7 @@ struct GemvArgs {
   int Kw, Kg;          // words and groups per row
   int units_k;         // units per row block
   int total_units;
+  int warps;           // warps that take units (the first `warps` of the grid)
   int x_bytes;         // shared-memory bytes reserved for the activations
 };
 
@@ -70,7 +74,12 @@ __device__ __forceinline__ uint32_t ld_nc_u16(const __half* p) {
 // This warp's contiguous range [u0, u0 + cnt) of the units.
 __device__ __forceinline__ void warp_range(const GemvArgs& a, int warp, int& u0, int& cnt) {
   const int gw = blockIdx.x * kWarps + warp;
-  const int nw = gridDim.x * kWarps;
+  const int nw = a.warps;
+  if (gw >= nw) {
+    u0 = a.total_units;
+    cnt = 0;
+    return;
+  }
   const int base = a.total_units / nw;
   const int rem = a.total_units - base * nw;
   u0 = gw * base + min(gw, rem);
@@ -426,7 +435,13 @@ cudaError_t launch_gemv(const GemmProblem& p, const Workspace& ws, cudaStream_t 
     a.x_bytes = 0;
     stages = 4;
   }
-  const int grid = min(sms, (a.total_units + kWarps - 1) / kWarps);
+  // At most two warps contribute to a row block when every warp takes at least
+  // units_k - 1 units (a shorter range is what it takes to lie strictly inside
+  // a row block), and two partial sums added onto zero give the same fp32 sum in
+  // either order: y then does not depend on which contributor comes first.
+  a.warps = min(sms * kWarps, a.total_units);
+  if (a.units_k > 2) a.warps = max(1, min(a.warps, a.total_units / (a.units_k - 1)));
+  const int grid = (a.warps + kWarps - 1) / kWarps;
   switch (p.M) {
     case 1: return launch_multi<1>(a, grid, stages, st);
     case 2: return launch_multi<2>(a, grid, stages, st);

@@ -240,30 +240,30 @@ __global__ void gptq_reverse_kernel(const double* __restrict__ H, int K, double*
 }
 
 // Blocked factorization in 64 x 64 tiles (K is a multiple of 128).  Right-looking
-// Cholesky: for each block column kb, the diagonal tile is factored (and its
-// triangular inverse formed) by one CTA, the panel below becomes
+// Cholesky: for each block column kb, the diagonal tile is factored and its
+// triangular inverse formed by one CTA, the panel below becomes
 // L[ib][kb] = A[ib][kb] inv(L[kb][kb])^T, and the trailing lower triangle is
-// updated, A[ib][jb] -= L[ib][kb] L[jb][kb]^T.  Then X = L^-1 by block rows:
-// X[ib][ib] = inv(L[ib][ib]) and, for kb < ib,
-// X[ib][kb] = -inv(L[ib][ib]) sum_{jb = kb}^{ib-1} L[ib][jb] X[jb][kb].
-// Every tile product is a 64 x 64 x 64 fp64 product: 256 threads, 4 x 4
-// outputs each, operands staged in shared memory with k outermost.
+// updated, A[ib][jb] -= L[ib][kb] L[jb][kb]^T.  X = L^-1 follows by block rows
+// one step behind (see the schedule below).  Every tile product is a
+// 64 x 64 x 64 fp64 product: 256 threads, 4 x 4 outputs each (rows 4 tr + i,
+// columns tc + 16 j), both operands staged row by row in shared memory.
 constexpr int kB = 64;
-constexpr int kBP = kB + 2;  // padded row of a staged tile (doubles)
+constexpr int kBP = kB + 1;  // padded row (doubles): 16 rows read down one column hit 16 distinct bank pairs
+constexpr int kFactorSmem = (2 * kB * kBP + kB + 32) * 8;
 
-// dst[k][x] = src[x][k] (transpose) or src[k][x]; src row stride ld.
-__device__ __forceinline__ void stage_tile(double (*dst)[kBP], const double* src, long long ld, bool transpose) {
+// dst[r][c] = src[r ld + c]: coalesced reads, consecutive shared-memory words.
+__device__ __forceinline__ void stage_tile(double (*dst)[kBP], const double* src, long long ld) {
   for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
-    const int a = e / kB, b = e % kB;  // b runs fastest: coalesced reads of src row a
-    const double v = src[static_cast<long long>(a) * ld + b];
-    if (transpose)
-      dst[b][a] = v;  // src[a][b] = P[x = a][k = b]
-    else
-      dst[a][b] = v;  // src[a][b] = Q[k = a][x = b]
+    const int r = e / kB, c = e % kB;
+    dst[r][c] = src[static_cast<long long>(r) * ld + c];
   }
 }
 
-// acc[i][j] += sum_k Ps[k][4 tr + i] * Qs[k][4 tc + j]
+// acc[i][j] += sum_k P[4 tr + i][k] Q(k, tc + 16 j), with Q(k, c) = Qs[c][k] when
+// QT (the staged tile is the transpose of the right operand), else Qs[k][c].  A
+// warp reads two P addresses (broadcasts) and 16 consecutive, or column-wise
+// conflict-free, Q words per load.
+template <bool QT>
 __device__ __forceinline__ void tile_product(double (&acc)[4][4], const double (*Ps)[kBP], const double (*Qs)[kBP],
                                              int tr, int tc) {
 #pragma unroll 4
@@ -271,8 +271,8 @@ __device__ __forceinline__ void tile_product(double (&acc)[4][4], const double (
     double p[4], q[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      p[i] = Ps[k][4 * tr + i];
-      q[i] = Qs[k][4 * tc + i];
+      p[i] = Ps[4 * tr + i][k];
+      q[i] = QT ? Qs[tc + 16 * i][k] : Qs[k][tc + 16 * i];
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -281,99 +281,180 @@ __device__ __forceinline__ void tile_product(double (&acc)[4][4], const double (
   }
 }
 
-// Diagonal tile kb: L[kb][kb] (lower) in place and Dinv[kb] = its inverse.
-__global__ void __launch_bounds__(256) gptq_chol_diag_kernel(double* __restrict__ L, int K, int kb,
-                                                             double* __restrict__ Dinv) {
-  extern __shared__ double sm[];
-  double(*a)[kB + 1] = reinterpret_cast<double(*)[kB + 1]>(sm);
-  double(*x)[kB + 1] = reinterpret_cast<double(*)[kB + 1]>(sm + kB * (kB + 1));
+// Lower Cholesky factor of the 32 x 32 block at a[o..o+31][o..o+31], in place,
+// by one warp, lane i keeping row o + i in registers: at column j every lane
+// takes rs = 1/sqrt(a_jj) from lane j's register (a shuffle), L_jj = a_jj rs,
+// lane i > j forms l_ij = a_ij rs and publishes it in col[i], and every lane
+// updates its row, a_ic -= l_ij l_cj for j < c <= i (l_cj a broadcast read).
+// rd[o + j] receives 1 / L_jj.  Entries above the diagonal become 0.
+__device__ __forceinline__ void chol32_warp(double (*a)[kBP], double* col, double* rd, int o) {
+  const int i = threadIdx.x & 31;
+  double r[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) r[c] = c <= i ? a[o + i][o + c] : 0.0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const double ajj = __shfl_sync(0xffffffffu, r[j], j);
+    const double rs = rsqrt(ajj);
+    const double l = r[j] * rs;
+    col[i] = l;
+    __syncwarp();
+#pragma unroll
+    for (int c = j + 1; c < 32; ++c)
+      if (i >= c) r[c] = fma(-l, col[c], r[c]);
+    __syncwarp();  // col is rewritten for the next column
+    if (i == j) {
+      r[j] = ajj * rs;
+      rd[o + j] = rs;
+    } else if (i < j) {
+      r[j] = 0.0;
+    } else {
+      r[j] = l;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 32; ++c) a[o + i][o + c] = r[c];
+}
+
+// X = L^-1 for the lower-triangular 32 x 32 block L = a[o..][o..], into
+// x[o..][o..], by one warp: lane c forms column c by forward substitution,
+// X[i][c] = -(sum_{k<i} L[i][k] X[k][c]) / L[i][i] (X[k][c] = 0 for k < c, so the
+// sum may start at 0), X[c][c] = 1 / L[c][c]; rd holds the 32 reciprocals.
+// L is read by broadcasts, each lane's column of X is its own; two partial
+// sums halve the dependent chain.
+__device__ __forceinline__ void inv32_warp(const double (*a)[kBP], double (*x)[kBP], const double* rd, int o) {
+  const int c = threadIdx.x & 31;
+  for (int i = 0; i < 32; ++i) {
+    double s0 = 0.0, s1 = 0.0;
+    for (int k = 0; k + 1 < i; k += 2) {
+      s0 = fma(a[o + i][o + k], x[o + k][o + c], s0);
+      s1 = fma(a[o + i][o + k + 1], x[o + k + 1][o + c], s1);
+    }
+    if (i & 1) s0 = fma(a[o + i][o + i - 1], x[o + i - 1][o + c], s0);
+    x[o + i][o + c] = i < c ? 0.0 : (i == c ? rd[o + i] : -(s0 + s1) * rd[o + i]);
+  }
+}
+
+// Diagonal tile kb: L[kb][kb] (lower, zeros above) in place and Dinv[kb] = its
+// inverse, by one CTA of 256 threads, as 2 x 2 blocks of 32: L11 = chol(A11),
+// X11 = L11^-1, L21 = A21 X11^T, A22 -= L21 L21^T, L22 = chol(A22), X22 = L22^-1,
+// X21 = -X22 (L21 X11).  The two Cholesky factors and inverses are single-warp
+// steps; the four 32 x 32 products use every thread (4 outputs each).
+__device__ void chol_diag_tile(double* sm, double* __restrict__ L, int K, int kb, double* __restrict__ Dinv) {
+  double(*a)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
+  double(*x)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
+  double* rd = sm + 2 * kB * kBP;  // 1 / L_jj
+  double* col = rd + kB;             // a column of the 32 x 32 factor in progress
   double* tile = L + static_cast<long long>(kb) * kB * K + static_cast<long long>(kb) * kB;
-  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) a[e / kB][e % kB] = tile[static_cast<long long>(e / kB) * K + e % kB];
+  const int warp = threadIdx.x >> 5;
+  const int pr = threadIdx.x >> 3, pc = threadIdx.x & 7;  // 32 rows x 8 threads, columns pc + 8 j
+  __syncthreads();  // the shared memory may hold a tile product of this CTA
+  stage_tile(a, tile, K);
   __syncthreads();
-  // Column j: d = sqrt(a[j][j]) (kept at a[j][j]); the trailing lower triangle
-  // takes a[i][c] -= a[i][j] a[c][j] / d^2 from the unscaled column, which is
-  // divided by d only once every later column is done.  Two barriers per column.
-  for (int j = 0; j < kB; ++j) {
-    if (threadIdx.x == 0) a[j][j] = sqrt(a[j][j]);
-    __syncthreads();
-    const double inv_d2 = 1.0 / (a[j][j] * a[j][j]);
-    for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
-      const int i = e / kB, c = e % kB;
-      if (c > j && c <= i) a[i][c] = fma(-a[i][j] * inv_d2, a[c][j], a[i][c]);
-    }
-    __syncthreads();
-  }
-  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
-    const int i = e / kB, c = e % kB;
-    if (i > c) a[i][c] /= a[c][c];
+  if (warp == 0) {
+    chol32_warp(a, col, rd, 0);
+    __syncwarp();
+    inv32_warp(a, x, rd, 0);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
-    const int i = e / kB, c = e % kB;
-    tile[static_cast<long long>(i) * K + c] = c <= i ? a[i][c] : 0.0;
-  }
-  // inverse by forward substitution, one column per thread
-  if (threadIdx.x < kB) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < c; ++i) x[i][c] = 0.0;
-    x[c][c] = 1.0 / a[c][c];
-    for (int i = c + 1; i < kB; ++i) {
-      double sum = 0.0;
-      for (int k = c; k < i; ++k) sum = fma(a[i][k], x[k][c], sum);
-      x[i][c] = -sum / a[i][i];
+  {  // L21 = A21 X11^T (X11 is 0 above its diagonal)
+    double s[4] = {};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const double v = a[32 + pr][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[j] = fma(v, x[pc + 8 * j][k], s[j]);
     }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a[32 + pr][pc + 8 * j] = s[j];
+  }
+  __syncthreads();
+  // A22 -= L21 L21^T on and below the diagonal
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = pc + 8 * j;
+    if (c <= pr) {
+      double s = 0.0;
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) s = fma(a[32 + pr][k], a[32 + c][k], s);
+      a[32 + pr][32 + c] -= s;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    chol32_warp(a, col, rd, 32);
+    __syncwarp();
+    inv32_warp(a, x, rd, 32);
+  }
+  __syncthreads();
+  {  // T = L21 X11 into the unused upper-right block of x
+    double s[4] = {};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const double v = a[32 + pr][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[j] = fma(v, x[k][pc + 8 * j], s[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[pr][32 + pc + 8 * j] = s[j];
+  }
+  __syncthreads();
+  {  // X21 = -X22 T
+    double s[4] = {};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const double v = x[32 + pr][32 + k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[j] = fma(v, x[k][32 + pc + 8 * j], s[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[32 + pr][pc + 8 * j] = -s[j];
   }
   __syncthreads();
   double* dinv = Dinv + static_cast<long long>(kb) * kB * kB;
-  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) dinv[e] = x[e / kB][e % kB];
+  for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) {
+    const int r = e / kB, c = e % kB;
+    tile[static_cast<long long>(r) * K + c] = c <= r ? a[r][c] : 0.0;
+    dinv[e] = c <= r ? x[r][c] : 0.0;
+  }
 }
 
-// Panel of block column kb: block row ib = kb + 1 + blockIdx.x,
-// L[ib][kb] = A[ib][kb] Dinv[kb]^T.
-__global__ void __launch_bounds__(256) gptq_chol_panel_kernel(double* __restrict__ L, int K, int kb,
-                                                              const double* __restrict__ Dinv) {
-  extern __shared__ double sm[];
+// Panel of block column kb, block row ib > kb: L[ib][kb] = A[ib][kb] Dinv[kb]^T.
+__device__ void chol_panel_tile(double* sm, double* __restrict__ L, int K, int kb, int ib,
+                                const double* __restrict__ Dinv) {
   double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
   double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
-  const int ib = kb + 1 + blockIdx.x;
   double* tile = L + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
-  stage_tile(Ps, tile, K, true);                                           // P[r][k] = A[ib][kb][r][k]
-  stage_tile(Qs, Dinv + static_cast<long long>(kb) * kB * kB, kB, true);   // Q[k][c] = Dinv[c][k]
+  stage_tile(Ps, tile, K);
+  stage_tile(Qs, Dinv + static_cast<long long>(kb) * kB * kB, kB);
   __syncthreads();
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   double acc[4][4] = {};
-  tile_product(acc, Ps, Qs, tr, tc);
+  tile_product<true>(acc, Ps, Qs, tr, tc);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = acc[i][j];
+    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + tc + 16 * j] = acc[i][j];
 }
 
-// Trailing update after block column kb: tile (ib, jb) with kb < jb <= ib, numbered
-// row by row over the lower triangle; A[ib][jb] -= L[ib][kb] L[jb][kb]^T.
-__global__ void __launch_bounds__(256) gptq_chol_update_kernel(double* __restrict__ L, int K, int kb) {
-  extern __shared__ double sm[];
+// Trailing update after block column kb of tile (ib, jb), kb < jb <= ib:
+// A[ib][jb] -= L[ib][kb] L[jb][kb]^T.
+__device__ void chol_update_tile(double* sm, double* __restrict__ L, int K, int kb, int ib, int jb) {
   double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
   double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
-  // blockIdx.x = t (t + 1) / 2 + c for tile row t, column c <= t of the trailing triangle
-  const int b = blockIdx.x;
-  int t = static_cast<int>((sqrt(8.0 * b + 1.0) - 1.0) / 2.0);
-  while ((t + 1) * (t + 2) / 2 <= b) ++t;
-  while (t * (t + 1) / 2 > b) --t;
-  const int c = b - t * (t + 1) / 2;
-  const int ib = kb + 1 + t, jb = kb + 1 + c;
-  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB, K, true);
-  stage_tile(Qs, L + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, true);
+  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB, K);
+  stage_tile(Qs, L + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K);
   __syncthreads();
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   double acc[4][4] = {};
-  tile_product(acc, Ps, Qs, tr, tc);
+  tile_product<true>(acc, Ps, Qs, tr, tc);
   double* tile = L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      double* d = tile + static_cast<long long>(4 * tr + i) * K + 4 * tc + j;
+      double* d = tile + static_cast<long long>(4 * tr + i) * K + tc + 16 * j;
       *d -= acc[i][j];
     }
 }
@@ -383,53 +464,101 @@ __global__ void __launch_bounds__(256) gptq_chol_update_kernel(double* __restric
 // X[jb][kb] = Dinv[jb] R[jb][kb] for kb < jb and X[jb][jb] = Dinv[jb]; then every
 // later block row is updated, R[ib][kb] -= L[ib][jb] X[jb][kb] for kb <= jb < ib
 // (R starts as the identity: its first update, at jb = kb, is a plain product).
-// Each step is parallel over its tiles, so the critical path is 2 K / 64 launches.
-__global__ void __launch_bounds__(256) gptq_trinv_final_kernel(int K, int jb, const double* __restrict__ Dinv,
-                                                               double* __restrict__ X) {
-  extern __shared__ double sm[];
+
+// Tile kb <= jb of the final block row jb.
+__device__ void trinv_final_tile(double* sm, int K, int jb, int kb, const double* __restrict__ Dinv,
+                                 double* __restrict__ X) {
   double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
   double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
-  const int kb = blockIdx.x;  // 0 .. jb
   double* tile = X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB;
   const double* dinv = Dinv + static_cast<long long>(jb) * kB * kB;
   if (kb == jb) {
     for (int e = threadIdx.x; e < kB * kB; e += blockDim.x) tile[static_cast<long long>(e / kB) * K + e % kB] = dinv[e];
     return;
   }
-  stage_tile(Ps, dinv, kB, true);    // P[r][k] = Dinv[jb][r][k]
-  stage_tile(Qs, tile, K, false);    // Q[k][c] = R[jb][kb][k][c]
+  stage_tile(Ps, dinv, kB);
+  stage_tile(Qs, tile, K);
   __syncthreads();
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   double acc[4][4] = {};
-  tile_product(acc, Ps, Qs, tr, tc);
+  tile_product<false>(acc, Ps, Qs, tr, tc);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + 4 * tc + j] = acc[i][j];
+    for (int j = 0; j < 4; ++j) tile[static_cast<long long>(4 * tr + i) * K + tc + 16 * j] = acc[i][j];
 }
 
-// Update after step jb: CTA (blockIdx.x = kb <= jb, blockIdx.y = ib - jb - 1).
-__global__ void __launch_bounds__(256) gptq_trinv_update_kernel(const double* __restrict__ L, int K, int jb,
-                                                                double* __restrict__ X) {
-  extern __shared__ double sm[];
+// Update after step jb of tile (ib, kb), kb <= jb < ib: R[ib][kb] -= L[ib][jb] X[jb][kb].
+__device__ void trinv_update_tile(double* sm, const double* __restrict__ L, int K, int jb, int kb, int ib,
+                                  double* __restrict__ X) {
   double(*Ps)[kBP] = reinterpret_cast<double(*)[kBP]>(sm);
   double(*Qs)[kBP] = reinterpret_cast<double(*)[kBP]>(sm + kB * kBP);
-  const int kb = blockIdx.x, ib = jb + 1 + blockIdx.y;
-  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB, K, true);   // L[ib][jb]
-  stage_tile(Qs, X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K, false);  // X[jb][kb]
+  stage_tile(Ps, L + static_cast<long long>(ib) * kB * K + static_cast<long long>(jb) * kB, K);
+  stage_tile(Qs, X + static_cast<long long>(jb) * kB * K + static_cast<long long>(kb) * kB, K);
   __syncthreads();
   const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
   double acc[4][4] = {};
-  tile_product(acc, Ps, Qs, tr, tc);
+  tile_product<false>(acc, Ps, Qs, tr, tc);
   double* tile = X + static_cast<long long>(ib) * kB * K + static_cast<long long>(kb) * kB;
   const bool first = kb == jb;  // R[ib][kb] is still the zero block of the identity
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      double* d = tile + static_cast<long long>(4 * tr + i) * K + 4 * tc + j;
+      double* d = tile + static_cast<long long>(4 * tr + i) * K + tc + 16 * j;
       *d = first ? -acc[i][j] : *d - acc[i][j];
     }
+}
+
+// The schedule: two launches per block column s, the inverse one step behind
+// the factorization, and the next diagonal tile factored by the CTA that
+// applies its last update (so it overlaps the rest of that update):
+//   launch A(s): the panel of block column s (nb - 1 - s CTAs) and the update
+//                after block row s - 1 of X (s (nb - s) CTAs);
+//   launch B(s): the trailing update after block column s (one CTA per tile of
+//                the lower triangle; CTA 0 holds tile (s + 1, s + 1) and goes on
+//                to factor it) and the final block row s of X (s + 1 CTAs).
+// A(s) needs Dinv[s] and the updated block column s (from B(s - 1)), L's block
+// column s - 1 (A(s - 1)) and X's block row s - 1 (B(s - 1)); B(s) needs the
+// panel and the update of X's block row s (A(s)).  A diagonal tile 0 launch
+// starts it.
+__global__ void __launch_bounds__(256) gptq_factor_diag0_kernel(double* __restrict__ L, int K,
+                                                                double* __restrict__ Dinv) {
+  extern __shared__ double sm[];
+  chol_diag_tile(sm, L, K, 0, Dinv);
+}
+
+__global__ void __launch_bounds__(256) gptq_factor_a_kernel(double* __restrict__ L, int K, int s, int nb,
+                                                            const double* __restrict__ Dinv,
+                                                            double* __restrict__ X) {
+  extern __shared__ double sm[];
+  const int m = nb - 1 - s;
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < m) {
+    chol_panel_tile(sm, L, K, s, s + 1 + b, Dinv);
+    return;
+  }
+  const int e = b - m;  // over kb = 0 .. s - 1 (fastest), ib = s .. nb - 1
+  trinv_update_tile(sm, L, K, s - 1, e % s, s + e / s, X);
+}
+
+__global__ void __launch_bounds__(256, 2) gptq_factor_b_kernel(double* __restrict__ L, int K, int s, int nb,
+                                                            double* __restrict__ Dinv, double* __restrict__ X) {
+  extern __shared__ double sm[];
+  const int m = nb - 1 - s;
+  const int nu = m * (m + 1) / 2;
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < nu) {
+    // b = t (t + 1) / 2 + c for tile row t, column c <= t of the trailing triangle
+    int t = static_cast<int>((sqrt(8.0 * b + 1.0) - 1.0) / 2.0);
+    while ((t + 1) * (t + 2) / 2 <= b) ++t;
+    while (t * (t + 1) / 2 > b) --t;
+    const int c = b - t * (t + 1) / 2;
+    chol_update_tile(sm, L, K, s, s + 1 + t, s + 1 + c);
+    if (b == 0) chol_diag_tile(sm, L, K, s + 1, Dinv);  // tile (s + 1, s + 1) took its last update
+    return;
+  }
+  trinv_final_tile(sm, K, s, b - nu, Dinv, X);
 }
 
 // G[K-1-i][K-1-j] = X[i][j] on and below the diagonal of X, 0 elsewhere.
@@ -457,35 +586,20 @@ cudaError_t launch_gptq_factor(const double* H, int K, double* G, void* workspac
   double* X = reinterpret_cast<double*>(ws + align256(static_cast<size_t>(K) * K * 8));
   double* Dinv = reinterpret_cast<double*>(ws + 2 * align256(static_cast<size_t>(K) * K * 8));
   const int nb = K / kB;
-  const int smem = 2 * kB * kBP * 8, smem_diag = 2 * kB * (kB + 1) * 8;
-  cudaError_t e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_diag_kernel),
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_diag);
-  if (e == cudaSuccess)
-    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_panel_kernel),
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_chol_update_kernel),
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_final_kernel),
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = ensure_func_attr(reinterpret_cast<const void*>(gptq_trinv_update_kernel),
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaSuccess;
+  for (const void* f : {reinterpret_cast<const void*>(gptq_factor_diag0_kernel),
+                        reinterpret_cast<const void*>(gptq_factor_a_kernel),
+                        reinterpret_cast<const void*>(gptq_factor_b_kernel)})
+    if (e == cudaSuccess) e = ensure_func_attr(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kFactorSmem);
   if (e != cudaSuccess) return e;
   gptq_reverse_kernel<<<4 * device_sm_count(), 256, 0, st>>>(H, K, L);
-  for (int kb = 0; kb < nb && e == cudaSuccess; ++kb) {
-    gptq_chol_diag_kernel<<<1, 256, smem_diag, st>>>(L, K, kb, Dinv);
-    const int m = nb - 1 - kb;
-    if (m > 0) {
-      gptq_chol_panel_kernel<<<m, 256, smem, st>>>(L, K, kb, Dinv);
-      gptq_chol_update_kernel<<<m * (m + 1) / 2, 256, smem, st>>>(L, K, kb);
-    }
-    e = cudaGetLastError();
-  }
-  for (int jb = 0; jb < nb && e == cudaSuccess; ++jb) {
-    gptq_trinv_final_kernel<<<jb + 1, 256, smem, st>>>(K, jb, Dinv, X);
-    if (jb + 1 < nb) gptq_trinv_update_kernel<<<dim3(jb + 1, nb - 1 - jb), 256, smem, st>>>(L, K, jb, X);
+  gptq_factor_diag0_kernel<<<1, 256, kFactorSmem, st>>>(L, K, Dinv);
+  e = cudaGetLastError();
+  for (int s = 0; s < nb && e == cudaSuccess; ++s) {
+    const int m = nb - 1 - s;
+    const int ga = m + s * (nb - s);
+    if (ga > 0) gptq_factor_a_kernel<<<ga, 256, kFactorSmem, st>>>(L, K, s, nb, Dinv, X);
+    gptq_factor_b_kernel<<<m * (m + 1) / 2 + s + 1, 256, kFactorSmem, st>>>(L, K, s, nb, Dinv, X);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;

@@ -87,7 +87,7 @@ LLAMA7B = dict(seed=1, sigma=0.02, M=1, layers=[
 LLAMA65B = dict(seed=2, sigma=0.015, M=1, layers=[
     ("attn_8192x8192", 8192, 8192), ("up_22016x8192", 22016, 8192),
     ("down_8192x22016", 8192, 22016)])
-SKINNY_M = (1, 4, 16, 32, 64)
+SKINNY_M = (1, 4, 8, 12, 16, 32, 64)
 SKINNY = dict(seed=3, sigma=0.015, M=max(SKINNY_M), layers=[("skinny_8192", 8192, 8192)])
 QUANT = dict(seed=0, sigma=0.02, N=11008, K=4096, alpha=0.5)
 
