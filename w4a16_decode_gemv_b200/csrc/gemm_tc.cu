@@ -32,7 +32,7 @@
 // puts the flags back to 0.  y does not depend on timing, and no second kernel
 // is needed.
 //
-// Roles (16 warps):
+// Roles (24 warps):
 //   warp 0       one thread streams the codes: per unit two adjacent tensor
 //                copies of 128 rows x 128 bytes (128-byte swizzle, 32 KiB in
 //                all) into a ring of Sc stages;
@@ -43,12 +43,12 @@
 //                copy of a [K / 64][M][64] view per stage (a unit's x up to
 //                MP = 32, half of it up to 128, one group above), after
 //                griddepcontrol.wait;
-//   warps 4-11   dequantization: warp w covers tensor-memory lane quarter w & 3
-//                (rows 32 (w & 3) .. + 31 of the tile) and groups h and h + 2
-//                (h = (w - 4) >> 2) of each unit; lane i reads its row's 64 code
-//                bytes per group, converts them into w_hat and stores them with
-//                tcgen05.st;
-//   warps 12-15  epilogue: accumulator read-out, y, partial tiles, the owner's sums.
+//   warps 4-19   dequantization: warp w covers tensor-memory lane quarter w & 3
+//                (rows 32 (w & 3) .. + 31 of the tile) and group h = (w - 4) >> 2
+//                of each unit; lane i reads its row's 64 code bytes, converts
+//                them into w_hat and stores them with tcgen05.st (four warps per
+//                lane quarter, so that their latencies overlap);
+//   warps 20-23  epilogue: accumulator read-out, y, partial tiles, the owner's sums.
 // Dequantization of a code pair: (w >> 4t) & 0x000F000F | 0x64006400 (one LOP3)
 // reads as the fp16 pair 1024 + q; subtracting 1024 + z is exact and the
 // multiply by Delta rounds once (Lecture 13 guide, §TinyChat, slides 36-37;
@@ -68,11 +68,13 @@ constexpr int kCodeStage = kRows * 256;    // 32 KiB: the codes of one unit (4 g
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
-constexpr int kWarps = 16;
+constexpr int kWarps = 24;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCodeWarp = 0, kMmaWarp = 1, kXWarp = 2, kXWarp2 = 3;
-constexpr int kDqWarp0 = 4, kDqWarps = 8;
-constexpr int kEpiWarp0 = 12, kEpiWarps = 4;
+constexpr int kDqWarp0 = 4, kDqWarps = 16;
+constexpr int kDqSets = kDqWarps / 4;   // dequantizing warps per tensor-memory lane quarter
+constexpr int kGpw = 4 / kDqSets;       // groups of a unit per dequantizing warp
+constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps, kEpiWarps = 4;
 constexpr int kCtrlBytes = 1024;
 constexpr uint32_t kTmemCols = 512;
 
@@ -107,31 +109,32 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
 
+// The MMA issue is warp-collective: the whole warp runs the issue loop with its
+// operands the same in every lane, and one elected lane issues each instruction.
+// On B200 that issues a 128 x 16 x 16 MMA every 25 cycles, against 50 when a
+// single lane runs the loop alone (a one-warp microbenchmark, A in tensor memory).
+
 // D[tmem] (+)= A[tmem] * B[smem]^T: A is 128 rows x 16 inputs (fp16 pairs in 8
 // consecutive columns), B is described by a shared-memory matrix descriptor.
+// Called by all 32 lanes of the warp with the same arguments.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                            bool accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
       : "memory");
 }
 
-// Arrives once on `bar` when every MMA this thread issued so far has completed.
+// Arrives once on `bar` when every MMA issued so far by the elected lanes of this
+// warp has completed (called by all 32 lanes; one commits).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (base + i).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
@@ -265,8 +268,7 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
 template <bool I8>
 struct Arith {
   static constexpr int kACols = I8 ? 32 : 64;          // tensor-memory columns of A per group
-  static constexpr int kChunks = I8 ? 1 : 2;           // 128-byte x chunks per group
-  static constexpr int kMmas = 4 * kChunks;            // MMAs per group
+  static constexpr int kChunks = I8 ? 1 : 2;           // 128-byte x chunks per group (4 MMAs each)
 };
 
 // kind::i8 instruction descriptor: s32 D, signed 8-bit A and B, both K-major, M = 128, N = n.
@@ -278,9 +280,10 @@ __host__ __device__ constexpr uint32_t idesc_i8(int n) {
 __device__ __forceinline__ void mma_i8_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           bool accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
       : "memory");
 }
@@ -449,74 +452,73 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (latest[s] >= 0) mbar_wait_bounded(&xfull[s], static_cast<uint32_t>(latest[s] / Sx) & 1u);
     }
   } else if (warp == kMmaWarp) {
-    // ---------------- MMA issuer ----------------
-    // A wait on an mbarrier between MMAs costs this thread about as much as 5
-    // MMAs of 128 x 16 x 16 (B200 measurement), even when the phase is already
-    // complete, so w_hat is signalled per unit (32 MMAs), not per group.
-    if (lane == 0) {
-      bool any = false, ok = true;
-      int seg = 0;
-      for (int i = 0; i < cnt && ok; ++i) {
-        const int u = u0 + i, q4 = u % Q;
-        const bool first = (i == 0) || (q4 == 0);
-        const bool last = (i == cnt - 1) || (q4 == Q - 1);
-        const int ab = seg % kAcc;
-        if (first && seg >= kAcc &&
-            !wait_or_abort(&accempty[ab], static_cast<uint32_t>(seg / kAcc - 1) & 1u, abort_flag, a.status))
+    // ---------------- MMA issuer (the whole warp; one lane issues) ----------------
+    // A wait on an mbarrier between MMAs costs about as much as 5 MMAs of
+    // 128 x 16 x 16 (B200 measurement), even when the phase is already complete,
+    // so w_hat is signalled per unit (32 MMAs), not per group.  Every lane waits
+    // and the outcome is agreed on by the warp, so the lanes stay converged.
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag, a.status));
+    };
+    bool any = false, ok = true;
+    int seg = 0;
+    for (int i = 0; i < cnt && ok; ++i) {
+      const int u = u0 + i, q4 = u % Q;
+      const bool first = (i == 0) || (q4 == 0);
+      const bool last = (i == cnt - 1) || (q4 == Q - 1);
+      const int ab = seg % kAcc;
+      if (first && seg >= kAcc && !wait_all(&accempty[ab], static_cast<uint32_t>(seg / kAcc - 1) & 1u)) break;
+      const uint32_t d = tbase + static_cast<uint32_t>(ab * MP);
+      // the unit's w_hat (all four groups) is in tensor memory (and, when kXByDq,
+      // its x stages have landed: the dequantizing warps wait for those first)
+      if (!wait_all(&afull[i & 1], static_cast<uint32_t>(i >> 1) & 1u)) break;
+      tc_fence_after();
+      for (int gg = 0; gg < 4; ++gg) {
+        const int j = i * xper + gg / kXG;  // x stage of this group
+        const int s = j % Sx;
+        if (!kXByDq && gg % kXG == 0 && !wait_all(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u)) {
+          ok = false;
           break;
-        const uint32_t d = tbase + static_cast<uint32_t>(ab * MP);
-        // the unit's w_hat (all four groups) is in tensor memory (and, when kXByDq,
-        // its x stages have landed: the dequantizing warps wait for those first)
-        if (!wait_or_abort(&afull[i & 1], static_cast<uint32_t>(i >> 1) & 1u, abort_flag, a.status)) break;
-        tc_fence_after();
-        for (int gg = 0; gg < 4; ++gg) {
-          const int j = i * xper + gg / kXG;  // x stage of this group
-          const int s = j % Sx;
-          if (!kXByDq && gg % kXG == 0 &&
-              !wait_or_abort(&xfull[s], static_cast<uint32_t>(j / Sx) & 1u, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          // every group position of a unit takes its w_hat slot, a position past the
-          // last group (K / 128 not a multiple of 4) with no MMAs, so that each slot's
-          // uses follow one another in order
-          const int ga = 4 * i + gg, b = ga % kASlots;
-          if (4 * q4 + gg < a.G) {
-            const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * AR::kACols);
-            const uint8_t* xg = xstage + s * kXStage + (gg % kXG) * AR::kChunks * kXChunk;
+        }
+        // every group position of a unit takes its w_hat slot, a position past the
+        // last group (K / 128 not a multiple of 4) with no MMAs, so that each slot's
+        // uses follow one another in order
+        const int ga = 4 * i + gg, b = ga % kASlots;
+        if (4 * q4 + gg < a.G) {
+          const uint32_t acol = tbase + kACol0 + static_cast<uint32_t>(b * AR::kACols);
+          const uint8_t* xg = xstage + s * kXStage + (gg % kXG) * AR::kChunks * kXChunk;
 #pragma unroll
-            for (int c = 0; c < AR::kChunks; ++c) {
-              const uint64_t bd = sw128_desc(xg + c * kXChunk);
+          for (int c = 0; c < AR::kChunks; ++c) {
+            const uint64_t bd = sw128_desc(xg + c * kXChunk);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                // the descriptor's start address advances 32 bytes (2 x 16) per MMA
-                const uint32_t at = acol + 8u * (4 * c + kk);
-                const bool accum = !(first && gg == 0 && c == 0 && kk == 0);
-                if constexpr (I8)
-                  mma_i8_ts(d, at, bd + 2u * kk, kIdesc, accum);
-                else
-                  mma_f16_ts(d, at, bd + 2u * kk, kIdesc, accum);
-              }
+            for (int kk = 0; kk < 4; ++kk) {
+              // the descriptor's start address advances 32 bytes (2 x 16) per MMA
+              const uint32_t at = acol + 8u * (4 * c + kk);
+              const bool accum = !(first && gg == 0 && c == 0 && kk == 0);
+              if constexpr (I8)
+                mma_i8_ts(d, at, bd + 2u * kk, kIdesc, accum);
+              else
+                mma_f16_ts(d, at, bd + 2u * kk, kIdesc, accum);
             }
-            any = true;
           }
-          mma_commit(&aempty[b]);
-          if (gg % kXG == kXG - 1) mma_commit(&xempty[s]);
+          any = true;
         }
-        if (!ok) break;
-        if (last) {
-          mma_commit(&accfull[ab]);
-          ++seg;
-        }
+        mma_commit(&aempty[b]);
+        if (gg % kXG == kXG - 1) mma_commit(&xempty[s]);
       }
-      if (any) {
-        mma_commit(tdown);
-        mbar_wait_bounded(tdown, 0);
+      if (!ok) break;
+      if (last) {
+        mma_commit(&accfull[ab]);
+        ++seg;
       }
+    }
+    if (any) {
+      mma_commit(tdown);
+      mbar_wait_bounded(tdown, 0);
     }
   } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
     // ---------------- dequantization into tensor memory ----------------
-    // warp (q, h): rows 32 q .. 32 q + 31 of the tile, groups h and h + 2 of each unit
+    // warp (q, h): rows 32 q .. 32 q + 31 of the tile, groups h + kDqSets e of each unit
     const int q = warp & 3, h = (warp - kDqWarp0) >> 2;
     const int r = q * 32 + lane;  // row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
@@ -526,9 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t pd[kLook], pz[kLook];
     auto fetch = [&](int it, uint16_t& dv, uint16_t& zv) {
       dv = zv = 0;
-      const int i = it >> 1;
+      const int i = it / kGpw;
       if (i < cnt) {
-        const int u = u0 + i, t = u / Q, g = 4 * (u - t * Q) + h + 2 * (it & 1);
+        const int u = u0 + i, t = u / Q, g = 4 * (u - t * Q) + h + kDqSets * (it % kGpw);
         const int n = t * kRows + r;
         if (n < a.N && g < a.G) {
           const size_t o = static_cast<size_t>(n) * a.G + g;
@@ -550,12 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = i % Sc;
       const bool okc = wait_or_abort(&cfull[s], static_cast<uint32_t>(i / Sc) & 1u, abort_flag, a.status);
       if (__any_sync(0xffffffffu, !okc)) break;
-      // this lane's 64 code bytes of groups h and h + 2 (box h... the pair box gg / 2, half gg % 2)
-      uint4 cw[2][4];
-      bool valid[2];
+      // this lane's 64 code bytes of each of its groups gg (the pair box gg / 2, half gg % 2)
+      uint4 cw[kGpw][4];
+      bool valid[kGpw];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int gg = h + 2 * e;
+      for (int e = 0; e < kGpw; ++e) {
+        const int gg = h + kDqSets * e;
         valid[e] = 4 * q4 + gg < a.G;
         if (valid[e]) {
           const uint32_t row = smem_u32(cstage) + static_cast<uint32_t>(s * kCodeStage + (gg >> 1) * (kCodeStage / 2) + r * 128);
@@ -569,22 +571,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&cempty[s]);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int gg = h + 2 * e;
+      for (int e = 0; e < kGpw; ++e) {
+        const int gg = h + kDqSets * e;
         const uint16_t dv = pd[0], zv = pz[0];
 #pragma unroll
         for (int l = 0; l + 1 < kLook; ++l) {
           pd[l] = pd[l + 1];
           pz[l] = pz[l + 1];
         }
-        fetch(2 * i + e + kLook, pd[kLook - 1], pz[kLook - 1]);
+        fetch(kGpw * i + e + kLook, pd[kLook - 1], pz[kLook - 1]);
         const int ga = 4 * i + gg, b = ga % kASlots;
-        // Both of this warp's slots of the unit must be free.  The MMA thread
+        // Each of this warp's slots of the unit must be free.  The MMA warp
         // commits the slots in group order and a commit arrives only once every
-        // earlier MMA has completed, so the wait for the later slot (group ga + 2)
-        // covers both: one barrier wait per unit (each costs hundreds of cycles).
+        // earlier MMA has completed, so the wait for the warp's last slot of the
+        // unit covers all: one barrier wait per unit (each costs hundreds of cycles).
         if (e == 0) {
-          const int gl = ga + 2;
+          const int gl = ga + kDqSets * (kGpw - 1);
           const bool oka = gl < kASlots || wait_or_abort(&aempty[gl % kASlots], static_cast<uint32_t>(gl / kASlots - 1) & 1u,
                                                          abort_flag, a.status);
           if (__any_sync(0xffffffffu, !oka)) {

@@ -53,15 +53,18 @@ __global__ void __launch_bounds__(kAsWarps * 32) act_scale_kernel(const __half* 
 }
 
 // ---------------------------------------------------------------------------
-// Quantize + pack.  A group of 128 input channels is handled by a half-warp:
-// lane h of the half-warp owns channels 8h .. 8h+7, i.e. exactly one packed
-// word of layout v1.  Group statistics are shuffle reductions over the 16 lanes.
-// Each warp iteration covers two groups; kQpUnroll iterations are loaded before
-// any is computed so that enough bytes are in flight.
+// Quantize + pack.  A group of 128 input channels is handled by four lanes (a
+// quad): lane q of the quad owns channels 32q .. 32q+31, i.e. four packed words
+// of layout v1, read as four 16-byte vectors and written as one.  Group
+// statistics are shuffle reductions over the quad (two levels), and the
+// per-group step and zero point, worked out by each lane of the quad, are
+// shared by 32 values per lane.  Each warp iteration covers eight groups;
+// kQpUnroll iterations are loaded before any is computed so that enough bytes
+// are in flight.
 // ---------------------------------------------------------------------------
 constexpr int kQpThreads = 256;
-constexpr int kQpHalfWarps = kQpThreads / 16;
-constexpr int kQpUnroll = 4;
+constexpr int kQpQuads = kQpThreads / 4;  // groups per CTA and iteration
+constexpr int kQpUnroll = 2;
 constexpr int kQpBlocksPerSm = 3;  // resident CTAs per SM the register budget allows
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
@@ -109,9 +112,10 @@ __global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kern
   const int Kg = K / kGroup;
   const int Kw = K / 8;
   const long long total = static_cast<long long>(N) * Kg;
-  const int hl = threadIdx.x & 15, hw = threadIdx.x >> 4;
-  const long long stride = static_cast<long long>(gridDim.x) * kQpHalfWarps;
-  long long g0 = static_cast<long long>(blockIdx.x) * kQpHalfWarps + hw;
+  const int ql = threadIdx.x & 3, qd = threadIdx.x >> 2;  // lane in the quad, quad in the CTA
+  const int qw = qd & 7;                                   // quad in the warp
+  const long long stride = static_cast<long long>(gridDim.x) * kQpQuads;
+  long long g0 = static_cast<long long>(blockIdx.x) * kQpQuads + qd;
   // (row, group) of g0 and of the stride, kept in step with g0 without dividing again
   int n0 = static_cast<int>(g0 / Kg), gi0 = static_cast<int>(g0 - static_cast<long long>(n0) * Kg);
   const int sn = static_cast<int>(stride / Kg), sr = static_cast<int>(stride - static_cast<long long>(sn) * Kg);
@@ -121,23 +125,22 @@ __global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kern
     if (gi >= Kg) gi -= Kg, ++n;
   };
 
-  // both half-warps of a warp run every iteration (the reductions shuffle over 32 lanes)
-  for (; g0 - (hw & 1) < total; g0 += stride * kQpUnroll) {
+  // every quad of a warp runs every iteration (the reductions shuffle over 32 lanes)
+  for (; g0 - qw < total; g0 += stride * kQpUnroll) {
     int nn[kQpUnroll], gg[kQpUnroll];
-    uint4 wv[kQpUnroll];
-    uint4 sv[kQpUnroll];
+    uint4 wv[kQpUnroll][4];
 #pragma unroll
     for (int u = 0; u < kQpUnroll; ++u) {
       nn[u] = u ? nn[u - 1] : n0;
       gg[u] = u ? gg[u - 1] : gi0;
       if (u) step(nn[u], gg[u]);
       const long long g = g0 + u * stride;
-      wv[u] = make_uint4(0, 0, 0, 0);
-      sv[u] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // 1.0
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wv[u][c] = make_uint4(0, 0, 0, 0);
       if (g < total) {
-        const int k = gg[u] * kGroup + hl * 8;
-        wv[u] = ldg_stream(W + static_cast<size_t>(nn[u]) * K + k);
-        if (HAS_S) sv[u] = __ldg(reinterpret_cast<const uint4*>(s + k));
+        const __half* wr = W + static_cast<size_t>(nn[u]) * K + gg[u] * kGroup + ql * 32;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) wv[u][c] = ldg_stream(wr + 8 * c);
       }
     }
     n0 = nn[kQpUnroll - 1];
@@ -146,28 +149,38 @@ __global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kern
 #pragma unroll
     for (int u = 0; u < kQpUnroll; ++u) {
       const long long g = g0 + u * stride;
-      // a1: w' = fp16(W * s), the exact product rounded once (mul.rn.f16x2)
-      __half2 w2[4];
-      w2[0] = as_h2(wv[u].x);
-      w2[1] = as_h2(wv[u].y);
-      w2[2] = as_h2(wv[u].z);
-      w2[3] = as_h2(wv[u].w);
-      if (HAS_S) {
-        w2[0] = __hmul2(w2[0], as_h2(sv[u].x));
-        w2[1] = __hmul2(w2[1], as_h2(sv[u].y));
-        w2[2] = __hmul2(w2[2], as_h2(sv[u].z));
-        w2[3] = __hmul2(w2[3], as_h2(sv[u].w));
+      // a1: w' = fp16(W * s), the exact product rounded once (mul.rn.f16x2);
+      // w2[4c + t] holds channels 32q + 8c + 2t and + 1
+      // (s is one row of K values shared by every row of W: read where it is used, from L1)
+      __half2 w2[16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        w2[4 * c + 0] = as_h2(wv[u][c].x);
+        w2[4 * c + 1] = as_h2(wv[u][c].y);
+        w2[4 * c + 2] = as_h2(wv[u][c].z);
+        w2[4 * c + 3] = as_h2(wv[u][c].w);
+        if (HAS_S && g < total) {
+          const uint4 sv = __ldg(reinterpret_cast<const uint4*>(s + gg[u] * kGroup + ql * 32 + 8 * c));
+          w2[4 * c + 0] = __hmul2(w2[4 * c + 0], as_h2(sv.x));
+          w2[4 * c + 1] = __hmul2(w2[4 * c + 1], as_h2(sv.y));
+          w2[4 * c + 2] = __hmul2(w2[4 * c + 2], as_h2(sv.z));
+          w2[4 * c + 3] = __hmul2(w2[4 * c + 3], as_h2(sv.w));
+        }
       }
-      // a2: group statistics over the half-warp (all 32 lanes take part)
+      // a2: group statistics over the quad (all 32 lanes take part)
       __half d;
       float zf;
       if (MODE == 0) {
         // (max, -min) in one fp16 pair, so one max per level reduces both
-        const __half2 hi = __hmax2(__hmax2(w2[0], w2[1]), __hmax2(w2[2], w2[3]));
-        const __half2 nlo = __hmax2(__hmax2(__hneg2(w2[0]), __hneg2(w2[1])), __hmax2(__hneg2(w2[2]), __hneg2(w2[3])));
+        __half2 hi = w2[0], nlo = __hneg2(w2[0]);
+#pragma unroll
+        for (int p = 1; p < 16; ++p) {
+          hi = __hmax2(hi, w2[p]);
+          nlo = __hmax2(nlo, __hneg2(w2[p]));
+        }
         __half2 mm = __hmax2(__lows2half2(hi, nlo), __highs2half2(hi, nlo));
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) mm = __hmax2(mm, as_h2(__shfl_xor_sync(0xffffffffu, as_u32(mm), o)));
+        for (int o = 2; o >= 1; o >>= 1) mm = __hmax2(mm, as_h2(__shfl_xor_sync(0xffffffffu, as_u32(mm), o)));
         // a3: Delta = fp16((max - min) / (2^N - 1)), the exact quotient rounded
         // once to fp16; a zero step becomes the unit range.  When max - min is
         // exact in fp32 (its TwoSum error term is zero), the correctly rounded
@@ -191,10 +204,12 @@ __global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kern
         const float dz = __half2float(d);
         zf = fminf(fmaxf(round_quotient(nmn, dz, __frcp_rn(dz)), 0.0f), static_cast<float>(kQmax)) + 0.0f;
       } else {
-        __half2 a = __hmax2(__hmax2(__habs2(w2[0]), __habs2(w2[1])), __hmax2(__habs2(w2[2]), __habs2(w2[3])));
+        __half2 a = __habs2(w2[0]);
+#pragma unroll
+        for (int p = 1; p < 16; ++p) a = __hmax2(a, __habs2(w2[p]));
         __half am = __hmax(__low2half(a), __high2half(a));
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) {
+        for (int o = 2; o >= 1; o >>= 1) {
           const __half other = __ushort_as_half(
               static_cast<unsigned short>(__shfl_xor_sync(0xffffffffu, static_cast<unsigned>(__half_as_ushort(am)), o)));
           am = __hmax(am, other);
@@ -207,49 +222,59 @@ __global__ void __launch_bounds__(kQpThreads, kQpBlocksPerSm) quantize_pack_kern
       }
       if (g >= total) continue;
       // a4: u = clamp(Round(w' / Delta) + z, 0, 2^N - 1);  a5: pack into layout v1.
-      // Two values at a time (elements 2t, 2t + 1, bound for bits 4t and
-      // 16 + 4t).  q + z = w * inv_d + z is clamped to [-1/4, 2^N - 3/4] (which
-      // changes no clamped code) and rounded to an integer by the magic add.
-      // The product is within 2^-19 of w / d for the quotients that are not
+      // Two values at a time (elements 2t, 2t + 1 of a word, bound for bits 4t
+      // and 16 + 4t).  q + z = w * inv_d + z is clamped to [-1/4, 2^N - 3/4]
+      // (which changes no clamped code) and rounded to an integer by the magic
+      // add.  The product is within 2^-19 of w / d for the quotients that are not
       // clamped (|w / d| < 2^5), so the integer is the exact Round unless q + z
-      // lies within 2^-16 of a half-integer; then the group is redone with
-      // round_quotient, which decides every case exactly.
+      // lies within 2^-16 of a half-integer; then the lane's values are redone
+      // with round_quotient, which decides every case exactly.
       const float df = __half2float(d);
       const float inv_d = __frcp_rn(df);
       const uint64_t inv2 = f2_pack(inv_d, inv_d), z2 = f2_pack(zf, zf);
       const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
-      uint64_t u2[4];
+      // Per word, the two 16-bit halves are summed as integers in floats on a
+      // 2^23 base (exact: below 2^16), so their low 16 bits are the packed nibbles.
+      uint32_t word[4];
       bool near = false;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 wf = __half22float2(w2[t]);
-        const float2 qz = f2_unpack(f2_fma(f2_pack(wf.x, wf.y), inv2, z2));
-        const uint64_t c2 = f2_pack(fminf(fmaxf(qz.x, -0.25f), static_cast<float>(kQmax) + 0.25f),
-                                    fminf(fmaxf(qz.y, -0.25f), static_cast<float>(kQmax) + 0.25f));
-        u2[t] = f2_sub(f2_add(c2, magic2), magic2);
-        const float2 off = f2_unpack(f2_sub(c2, u2[t]));
-        near |= fabsf(off.x) >= 0.5f - 0x1p-16f || fabsf(off.y) >= 0.5f - 0x1p-16f;
-      }
-      if (near) {
+      for (int c = 0; c < 4; ++c) {
+        uint64_t acc = f2_pack(8388608.0f, 8388608.0f);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float2 wf = __half22float2(w2[t]);
-          u2[t] = f2_pack(fminf(fmaxf(round_quotient(wf.x, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)),
-                          fminf(fmaxf(round_quotient(wf.y, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)));
+          const float2 wf = __half22float2(w2[4 * c + t]);
+          const float2 qz = f2_unpack(f2_fma(f2_pack(wf.x, wf.y), inv2, z2));
+          const uint64_t c2 = f2_pack(fminf(fmaxf(qz.x, -0.25f), static_cast<float>(kQmax) + 0.25f),
+                                      fminf(fmaxf(qz.y, -0.25f), static_cast<float>(kQmax) + 0.25f));
+          const uint64_t u2 = f2_sub(f2_add(c2, magic2), magic2);
+          const float2 off = f2_unpack(f2_sub(c2, u2));
+          near |= fabsf(off.x) >= 0.5f - 0x1p-16f || fabsf(off.y) >= 0.5f - 0x1p-16f;
+          const float sc = static_cast<float>(1 << (4 * t));
+          acc = f2_fma(u2, f2_pack(sc, sc), acc);
+        }
+        const float2 lh = f2_unpack(acc);
+        word[c] = __byte_perm(__float_as_uint(lh.x), __float_as_uint(lh.y), 0x5410);
+      }
+      if (near) {  // a value near a half-integer: the lane's codes again, each decided exactly
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint64_t acc = f2_pack(8388608.0f, 8388608.0f);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 wf = __half22float2(w2[4 * c + t]);
+            const uint64_t u2 =
+                f2_pack(fminf(fmaxf(round_quotient(wf.x, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)),
+                        fminf(fmaxf(round_quotient(wf.y, df, inv_d) + zf, 0.0f), static_cast<float>(kQmax)));
+            const float sc = static_cast<float>(1 << (4 * t));
+            acc = f2_fma(u2, f2_pack(sc, sc), acc);
+          }
+          const float2 lh = f2_unpack(acc);
+          word[c] = __byte_perm(__float_as_uint(lh.x), __float_as_uint(lh.y), 0x5410);
         }
       }
-      // the two 16-bit halves of the word summed as integers in floats on a 2^23
-      // base (exact: below 2^16), so their low 16 bits are the packed nibbles
-      uint64_t acc = f2_pack(8388608.0f, 8388608.0f);
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float sc = static_cast<float>(1 << (4 * t));
-        acc = f2_fma(u2[t], f2_pack(sc, sc), acc);
-      }
-      const float2 lh = f2_unpack(acc);
-      const uint32_t word = __byte_perm(__float_as_uint(lh.x), __float_as_uint(lh.y), 0x5410);
-      qweight[static_cast<size_t>(nn[u]) * Kw + gg[u] * 16 + hl] = word;
-      if (hl == 0) {
+      *reinterpret_cast<uint4*>(qweight + static_cast<size_t>(nn[u]) * Kw + gg[u] * 16 + ql * 4) =
+          make_uint4(word[0], word[1], word[2], word[3]);
+      if (ql == 0) {
         scales[static_cast<size_t>(nn[u]) * Kg + gg[u]] = d;
         zeros[static_cast<size_t>(nn[u]) * Kg + gg[u]] = __float2half_rn(zf);
       }
@@ -261,8 +286,8 @@ template <int BITS, int MODE, bool HAS_S>
 cudaError_t launch_qp(const __half* W, const __half* s, int N, int K, uint32_t* qw, __half* sc, __half* zr,
                       cudaStream_t st) {
   const long long groups = static_cast<long long>(N) * (K / kGroup);
-  const long long half_warps_needed = (groups + kQpUnroll - 1) / kQpUnroll;
-  long long blocks = (half_warps_needed + kQpHalfWarps - 1) / kQpHalfWarps;
+  const long long quads_needed = (groups + kQpUnroll - 1) / kQpUnroll;
+  long long blocks = (quads_needed + kQpQuads - 1) / kQpQuads;
   const long long cap = static_cast<long long>(device_sm_count()) * kQpBlocksPerSm;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
