@@ -251,6 +251,55 @@ def test_gemv_skinny_m4(dev):
     assert np.all(np.abs(y.cpu().numpy()[:, rows].astype(np.float64) - y_ref) <= RTOL * B + ATOL)
 
 
+# w4a16_gemm, M = 2..8 with K a multiple of 256: register-sourced MMAs (gemv_mma.cu)
+@pytest.mark.parametrize("M,N,K", [
+    (2, 1, 256),        # one row, one unit per row (15 of 16 warps idle)
+    (3, 17, 1280),      # ragged 16-row block, 5 units per row
+    (5, 300, 4096),
+    (8, 1000, 2048),    # every token column of the MMA used
+    (6, 33, 8192),
+    (2, 64, 11008),     # 43 units per row: warps with 2 and 3 units
+    (7, 129, 512),
+])
+def test_gemv_mma_shapes(dev, M, N, K):
+    _gemm_case(dev, M, N, K, seed=M * 7717 + N)
+
+
+def test_gemv_mma_edge_values(dev):
+    """Zero points 0 and 15, steps from tiny to large, outlier activations, rows past
+    a 16-row block; every output checked."""
+    rng = np.random.default_rng(3)
+    N, K, M = 37, 1024, 4
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    W[0] = np.abs(W[0])                      # a row of one sign: z = 0
+    W[1] = -np.abs(W[1])                     # z = 15
+    W[2] *= np.float16(1e-3)                 # tiny steps
+    W[3] = (rng.standard_normal(K) * 2).astype(np.float16)  # large steps
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    x[:, :11] *= np.float16(40)              # outlier channels
+    qo, so, zo = oracle.quantize_pack(W, None, 128, 4, oracle.ASYM)
+    y = w4.w4a16_gemm(to_dev(x, dev), to_dev(qo.view(np.int32), dev), to_dev(so, dev), to_dev(zo, dev))
+    torch.cuda.synchronize()
+    assert_close(y.cpu().numpy(), x, qo, so, zo)
+
+
+@pytest.mark.parametrize("M", [2, 4, 8])
+def test_gemv_mma_workload_rows_and_repeats(dev, M):
+    """The K = N = 8192 skinny layer at M = 2, 4, 8 (the bench's launches): sampled rows
+    against the oracle, and y bit-identical over repeated calls."""
+    (layer,) = inputs.layer_set(inputs.SKINNY)
+    x = layer.x[:M]
+    qg, sg, zg = w4.awq_quantize_pack(to_dev(layer.W, dev))
+    xd = to_dev(x, dev)
+    ys = [w4.w4a16_gemm(xd, qg, sg, zg).cpu().numpy() for _ in range(4)]
+    for yy in ys[1:]:
+        assert np.array_equal(yy.view(np.uint16), ys[0].view(np.uint16))
+    rows = np.unique(np.concatenate([np.random.default_rng(M).choice(layer.N, 250, replace=False),
+                                     [0, 15, 16, layer.N - 1]]))
+    y_ref, B = oracle.gemm_ref(x, oracle.dequant(qw_np(qg)[rows], sg.cpu().numpy()[rows], zg.cpu().numpy()[rows]))
+    assert np.all(np.abs(ys[0][:, rows].astype(np.float64) - y_ref) <= RTOL * B + ATOL)
+
+
 @pytest.mark.parametrize("M,N,K", [(4, 2048, 22016), (3, 513, 1152), (1, 300, 1152), (2, 512, 65536)])
 def test_split_k_gemv_repeats_bit_for_bit(dev, M, N, K):
     """The split-K GEMV (activations too large to stage, or K / 128 odd) adds at most

@@ -90,6 +90,12 @@ __device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32
 // 2-D tiled tensor copy global -> this CTA's shared memory (TMA), completion
 // counted on `bar` in bytes.  x is the innermost coordinate (elements); x times
 // the element size must be a multiple of 16 bytes.
+// Brings a tensor map (a __grid_constant__ kernel parameter) into the
+// descriptor cache ahead of the first tensor copy that uses it.
+__device__ __forceinline__ void prefetch_tensor_map(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar,
                                             uint64_t policy) {
   asm volatile(

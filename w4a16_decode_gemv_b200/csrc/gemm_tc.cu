@@ -407,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kCodeWarp) {
     // ---------------- codes: two adjacent 16 KiB boxes per unit ----------------
     if (lane == 0) {
+      prefetch_tensor_map(&tq);
       const uint64_t pol = l2_evict_first_policy();
       int issued = 0;
       // the weights do not depend on the previous kernel: no griddepcontrol.wait
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kXWarp || warp == kXWarp2) {
     // ---------------- x: one 3-D box per stage; the two x warps alternate stages ----------------
     if (lane == 0) {
+      prefetch_tensor_map(&tx);
       const uint64_t pol = l2_evict_last_policy();
       griddep_wait();  // x may be the previous kernel's output
       const int total_x = cnt * xper;

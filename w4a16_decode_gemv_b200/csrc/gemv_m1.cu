@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS)
   // the next kernel on the stream may start its own prologue right away
   griddep_launch_dependents();
   if (lane == 0) {
+    prefetch_tensor_map(&tmap);
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 33);  // expect-tx arrival + 32 cp.async arrivals
     fence_mbar_init();
   }

@@ -67,6 +67,12 @@ struct GemmProblem {
 bool gemv_m1_supports(int N, int K);
 cudaError_t launch_gemv_m1(const GemmProblem& p, uint32_t* status, cudaStream_t st);
 
+// The M = 2..8 GEMV on mma.sync (gemv_mma.cu): whole rows per CTA, no
+// workspace; false when K is not a multiple of 256 or the staged activations of
+// M tokens leave no room for two ring stages.
+bool gemv_mma_supports(int M, int N, int K);
+cudaError_t launch_gemv_mma(const GemmProblem& p, uint32_t* status, cudaStream_t st);
+
 // The M = 2..4 GEMV (gemv_mt.cu): whole rows per CTA, no workspace; false when
 // the staged activations of M tokens do not fit in shared memory.
 bool gemv_mt_supports(int M, int N, int K);

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_gemv_kernel(const W8Args a, 
 
   griddep_launch_dependents();
   if (lane == 0) {
+    prefetch_tensor_map(&tmap);
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
   }
