@@ -134,12 +134,15 @@ W4A16_API size_t w4a16_gemm_workspace_size(int M, int N, int K, int group);
  *
  *   y[m][n] = fp16( sum_g Delta[n][g] * sum_{k in g} (u[n][k] - z[n][g]) * x[m][k] )
  *
- * with fp32 accumulation.  M = 1..4 runs on the CUDA cores (M = 1: whole rows
- * per SM, no partial sums; M = 2..4: whole rows or split-K); M = 5..256 runs on
- * the tensor cores (tcgen05), with w_hat = Delta * (u - z) rounded once to fp16
- * before the MMA (so |w_hat| must stay below 65504).  Larger M (prefill) runs
- * as consecutive chunks of 256 tokens, each chunk as above, on the same
- * workspace.  x is the activation already divided by the AWQ scale s.
+ * with fp32 accumulation.  M = 1 runs on the CUDA cores (whole rows per SM, no
+ * partial sums).  M = 2..8 runs on register-sourced tensor-core MMAs
+ * (mma.sync, the integers u - z exact in fp16, Delta applied per group in
+ * fp32) when K is a multiple of 256 and the activations of M tokens fit in
+ * shared memory; otherwise M = 2..4 runs on the CUDA cores (whole rows or
+ * split-K).  The rest, up to 256 tokens per launch, runs on the tcgen05 tensor
+ * cores, with w_hat = Delta * (u - z) rounded once to fp16 before the MMA (so
+ * |w_hat| must stay below 65504).  Larger M (prefill) runs as consecutive
+ * chunks of 256 tokens, each chunk as above, on the same workspace.  x is the activation already divided by the AWQ scale s.
  * Accuracy: |y - y_ref| <= 2e-3 * sum_k |x[m][k] * w_hat[n][k]| + 1e-3 per element,
  * y_ref the exact product with the dequantized weight.  y is the same on every
  * call, bit for bit, on every path: the split-K CUDA-core GEMV (M = 1..4 when

@@ -164,15 +164,20 @@ __global__ void __launch_bounds__(32 * kSweepRows) gptq_block_kernel(const Sweep
 }
 
 // ---- the block's corrections to every column right of it ------------------------
-// Wc[r][j] -= sum_i e[r][i] G[b0 + i][j], i = 0..127 added in order.  64 x 64
-// tiles of (rows, columns), 4 x 4 per thread; e and G staged 16 columns of the
-// block at a time.  For the first block, the columns come from W itself.
+// Wc[r][j] -= sum_i e[r][i] G[b0 + i][j], i = 0..127 added in order (each
+// product and each sum rounded once: the order the oracle fixes).  64 x 64 tiles
+// of (rows, columns); thread (ty, tx) holds rows 4 ty + p and columns tx + 16 q,
+// so that a warp's reads of G are 16 consecutive words (no bank conflicts) and
+// its reads of e two broadcasts.  e and G are staged kUChunk columns of the block
+// at a time, with coalesced global reads (e is row-major by row: consecutive
+// threads take consecutive i of a row; the padded row keeps those stores on
+// distinct banks).  For the first block, the columns come from W itself.
 constexpr int kUTile = 64;
-constexpr int kUChunk = 16;
+constexpr int kUChunk = 32;
 
 __global__ void __launch_bounds__(256) gptq_update_kernel(const SweepArgs a, int b0) {
-  __shared__ double es[kUChunk][kUTile];  // [i][row]
-  __shared__ double gs[kUChunk][kUTile];  // [i][column]
+  __shared__ double es[kUChunk][kUTile + 1];  // [i][row]
+  __shared__ double gs[kUChunk][kUTile];      // [i][column]
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int r0 = blockIdx.x * kUTile;
   const int b1 = b0 + kGroupCols;
@@ -180,16 +185,27 @@ __global__ void __launch_bounds__(256) gptq_update_kernel(const SweepArgs a, int
   double acc[4][4] = {};
   for (int i0 = 0; i0 < kGroupCols; i0 += kUChunk) {
     for (int e = threadIdx.x; e < kUChunk * kUTile; e += 256) {
-      const int c = e % kUTile, i = e / kUTile;
-      es[i][c] = r0 + c < a.N ? a.errs[static_cast<size_t>(r0 + c) * kGroupCols + i0 + i] : 0.0;
-      gs[i][c] = j0 + c < a.K ? a.G[static_cast<size_t>(b0 + i0 + i) * a.K + j0 + c] : 0.0;
+      {  // e: row c, column i of the chunk (i fastest: contiguous in errs)
+        const int c = e / kUChunk, i = e % kUChunk;
+        es[i][c] = r0 + c < a.N ? a.errs[static_cast<size_t>(r0 + c) * kGroupCols + i0 + i] : 0.0;
+      }
+      {  // G: row i of the chunk, column c (c fastest: contiguous in G)
+        const int c = e % kUTile, i = e / kUTile;
+        gs[i][c] = j0 + c < a.K ? a.G[static_cast<size_t>(b0 + i0 + i) * a.K + j0 + c] : 0.0;
+      }
     }
     __syncthreads();
+#pragma unroll 4
     for (int i = 0; i < kUChunk; ++i) {
+      double ev[4], gv[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) ev[p] = es[i][ty * 4 + p];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) gv[q] = gs[i][tx + 16 * q];
 #pragma unroll
       for (int p = 0; p < 4; ++p)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = __dadd_rn(acc[p][q], __dmul_rn(es[i][ty * 4 + p], gs[i][tx * 4 + q]));
+        for (int q = 0; q < 4; ++q) acc[p][q] = __dadd_rn(acc[p][q], __dmul_rn(ev[p], gv[q]));
     }
     __syncthreads();
   }
@@ -200,7 +216,7 @@ __global__ void __launch_bounds__(256) gptq_update_kernel(const SweepArgs a, int
     const size_t row = static_cast<size_t>(r) * a.K;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int j = j0 + tx * 4 + q;
+      const int j = j0 + tx + 16 * q;
       if (j >= a.K) continue;
       const double w = b0 == 0 ? static_cast<double>(__half2float(a.W[row + j])) : a.Wc[row + j];
       a.Wc[row + j] = __dsub_rn(w, acc[p][q]);
