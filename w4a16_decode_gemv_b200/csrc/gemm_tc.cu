@@ -525,9 +525,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = q * 32 + lane;  // row within the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
-    // per-group parameters of the next items (unit, group), fetched a few items ahead
-    constexpr int kLook = 4;
-    uint16_t pd[kLook], pz[kLook];
+    // Per-group parameters, fetched two units ahead into one of two register
+    // sets (even and odd units): a value is first read two units after its load
+    // was issued, so the load's latency (HBM, under the code stream) is hidden.
+    // (A look-ahead by shifting a register array reads each value one unit after
+    // its load: every shift waits for the previous unit's load.)
+    uint16_t pd[2][kGpw], pz[2][kGpw];
     auto fetch = [&](int it, uint16_t& dv, uint16_t& zv) {
       dv = zv = 0;
       const int i = it / kGpw;
@@ -547,13 +550,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 #pragma unroll
-    for (int l = 0; l < kLook; ++l) fetch(l, pd[l], pz[l]);
+    for (int par = 0; par < 2; ++par)
+#pragma unroll
+      for (int e = 0; e < kGpw; ++e) fetch(kGpw * par + e, pd[par][e], pz[par][e]);
     bool ok = true;
-    for (int i = 0; i < cnt && ok; ++i) {
+    for (int i2 = 0; i2 < cnt && ok; i2 += 2)
+#pragma unroll
+    for (int par = 0; par < 2; ++par) {
+      const int i = i2 + par;
+      if (i >= cnt || !ok) break;
       const int u = u0 + i, t = u / Q, q4 = u - t * Q;
       const int s = i % Sc;
       const bool okc = wait_or_abort(&cfull[s], static_cast<uint32_t>(i / Sc) & 1u, abort_flag, a.status);
-      if (__any_sync(0xffffffffu, !okc)) break;
+      if (__any_sync(0xffffffffu, !okc)) {
+        ok = false;
+        break;
+      }
       // this lane's 64 code bytes of each of its groups gg (the pair box gg / 2, half gg % 2)
       uint4 cw[kGpw][4];
       bool valid[kGpw];
@@ -575,13 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < kGpw; ++e) {
         const int gg = h + kDqSets * e;
-        const uint16_t dv = pd[0], zv = pz[0];
-#pragma unroll
-        for (int l = 0; l + 1 < kLook; ++l) {
-          pd[l] = pd[l + 1];
-          pz[l] = pz[l + 1];
-        }
-        fetch(kGpw * i + e + kLook, pd[kLook - 1], pz[kLook - 1]);
+        const uint16_t dv = pd[par][e], zv = pz[par][e];
+        fetch(kGpw * (i + 2) + e, pd[par][e], pz[par][e]);
         const int ga = 4 * i + gg, b = ga % kASlots;
         // Each of this warp's slots of the unit must be free.  The MMA warp
         // commits the slots in group order and a commit arrives only once every
@@ -639,7 +646,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool okx = true;
       for (int jx = i * xper; kXByDq && warp == kDqWarp0 && jx < (i + 1) * xper && okx; ++jx)
         okx = wait_or_abort(&xfull[jx % Sx], static_cast<uint32_t>(jx / Sx) & 1u, abort_flag, a.status);
-      if (__any_sync(0xffffffffu, !okx)) break;
+      if (__any_sync(0xffffffffu, !okx)) {
+        ok = false;
+        break;
+      }
       // both of this warp's groups of the unit are in tensor memory
       tmem_wait_st();
       tc_fence_before();
