@@ -143,7 +143,34 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_gemv_kernel(const W8Args a, 
   const int swap1 = (lane >> 2) & 1;  // bank spread of the 32-byte lane strides, as the W4A16 GEMV
   bool failed = false;
   int kc = warp % a.units_k;
-  for (int j = warp, i = 0; j < U; j += kWarps, ++i) {
+  // s2 and zs of this lane's group in each row of unit jj (0 past the matrix),
+  // fetched two units ahead into one of two register sets (even and odd units of
+  // the warp), so that each load has two units' time before its value is read
+  auto load_s2zs = [&](int jj, int (&s2o)[kR], int (&zso)[kR]) {
+#pragma unroll
+    for (int r = 0; r < kR; ++r) s2o[r] = zso[r] = 0;
+    if (jj < U) {
+      const int kcj = jj % a.units_k;
+      const bool actj = lane * 8 < min(kUW, a.Kw - kcj * kUW);
+      const int g = kcj * kUG + (lane >> 1);
+      const int n0 = (rb0 + jj / a.units_k) * kR;
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        const bool in = actj && n0 + r < a.N && g < a.G;
+        const size_t o = static_cast<size_t>(n0 + r) * a.G + g;
+        s2o[r] = in ? static_cast<int>(ld_nc_u8(a.s2 + o)) : 0;
+        zso[r] = in ? static_cast<int>(ld_nc_u8(a.zs + o)) : 0;
+      }
+    }
+  };
+  int s2set[2][kR], zsset[2][kR];
+  load_s2zs(warp, s2set[0], zsset[0]);
+  load_s2zs(warp + kWarps, s2set[1], zsset[1]);
+  for (int j2 = warp, i2 = 0; j2 < U && !failed; j2 += 2 * kWarps, i2 += 2)
+#pragma unroll
+  for (int par = 0; par < 2; ++par) {
+    const int j = j2 + par * kWarps, i = i2 + par;
+    if (j >= U) break;
     const int s = i % S;
     const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
     const int ckc = kc;
@@ -170,19 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_gemv_kernel(const W8Args a, 
         xsm[m] = xsum[m * (a.K / 64) + slice];
       }
     }
-    // s2 and zs of this lane's group in each of the unit's rows (0 past the matrix)
     int s2r[kR], zsr[kR];
-    {
-      const int g = ckc * kUG + (lane >> 1);
-      const int n0 = (rb0 + j / a.units_k) * kR;
 #pragma unroll
-      for (int r = 0; r < kR; ++r) {
-        const bool in = act && n0 + r < a.N && g < a.G;
-        const size_t o = static_cast<size_t>(n0 + r) * a.G + g;
-        s2r[r] = in ? static_cast<int>(ld_nc_u8(a.s2 + o)) : 0;
-        zsr[r] = in ? static_cast<int>(ld_nc_u8(a.zs + o)) : 0;
-      }
+    for (int r = 0; r < kR; ++r) {
+      s2r[r] = s2set[par][r];
+      zsr[r] = zsset[par][r];
     }
+    load_s2zs(j + 2 * kWarps, s2set[par], zsset[par]);
     if (!mbar_wait_bounded(&full[s], parity)) {
       if (lane == 0) atomicOr(a.status, kDevWaitTimeout);
       failed = true;
