@@ -126,8 +126,8 @@ Workspace carve_workspace(void* base, int M, int N, int K) {
 // The kernels for an M x N x K problem with M <= kMaxM: M = 1 on whole rows when
 // the activation fits the kernel's staging; M = 2..8 on whole rows with
 // register-sourced MMAs when K is a multiple of 256 and the activations fit,
-// else M = 2..4 on whole rows or split-K on the CUDA cores; the rest (M = 5..256)
-// on the tcgen05 tensor cores.
+// else M = 2..4 on whole rows or split-K on the CUDA cores; the rest (up to 256
+// tokens) on the tcgen05 tensor cores.
 static cudaError_t dispatch_gemm(const GemmProblem& p, const Workspace& ws, cudaStream_t st) {
   if (p.M == 1 && gemv_m1_supports(p.N, p.K)) return launch_gemv_m1(p, ws.status, st);
   if (gemv_mma_supports(p.M, p.N, p.K)) return launch_gemv_mma(p, ws.status, st);

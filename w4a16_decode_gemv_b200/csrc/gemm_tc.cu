@@ -1,5 +1,7 @@
-// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05), M = 5..256 per
-// launch (larger M runs as chunks of 256 tokens, one launch per chunk).
+// W4A16 skinny GEMM on the 5th-generation tensor cores (tcgen05), up to 256
+// tokens per launch (larger M runs as chunks of 256 tokens, one launch per
+// chunk); from 9 tokens, or from 2 where the register-sourced MMA GEMV does not
+// apply.
 //
 //   y[m][n] = sum_k x[m][k] * w_hat[n][k],   w_hat = Delta[n][g] * (u[n][k] - z[n][g])
 //
